@@ -1,0 +1,18 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a B200 (sm_100) GPU and the built CUDA library")
+    config.addinivalue_line("markers", "slow: large-shape CPU work (still part of the default run)")
+
+
+@pytest.fixture(scope="session")
+def repo_root():
+    return ROOT

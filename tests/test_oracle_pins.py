@@ -1,0 +1,424 @@
+"""Pins for the CPU oracle: closed forms, invariants, brute force and special cases.
+
+Each test checks the oracle against something other than itself: the format
+definitions of E2M1 / UE4M3 / INT4 written out from their bit layouts, the
+algebraic identities that the SVDQuant model card's stages 1-3 fix, the
+Eckart-Young optimality of a truncated SVD, brute-force loops in a different
+order, and hand-computed tiny cases.  A plausible slip in the oracle (a wrong
+tie rule, a dropped term, a transposed factor, an inverted smoothing
+direction) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import svdq_oracle as O
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _f32(x):
+    return np.float32(x)
+
+
+def _next_up(x):
+    return np.nextafter(np.float32(x), np.float32(np.inf), dtype=np.float32)
+
+
+def _next_down(x):
+    return np.nextafter(np.float32(x), np.float32(-np.inf), dtype=np.float32)
+
+
+# ---------------------------------------------------------------- formats
+
+
+def e2m1_closed_form(code: int) -> float:
+    """E2M1 from its bits: sign | 2-bit exponent (bias 1) | 1 mantissa bit."""
+    s = -1.0 if code & 8 else 1.0
+    e = (code >> 1) & 3
+    m = code & 1
+    mag = m * 0.5 if e == 0 else 2.0 ** (e - 1) * (1.0 + m / 2.0)
+    return s * mag
+
+
+def ue4m3_closed_form(code: int) -> float:
+    e = (code >> 3) & 0xF
+    m = code & 7
+    return m * 2.0 ** -9 if e == 0 else 2.0 ** (e - 7) * (1.0 + m / 8.0)
+
+
+def test_e2m1_table_matches_bit_definition():
+    for c in range(16):
+        v = float(O.e2m1_value(np.array([c]))[0])
+        assert v == e2m1_closed_form(c) or (v == 0 and e2m1_closed_form(c) == 0)
+    assert float(O.e2m1_value(np.array([7]))[0]) == 6.0
+
+
+def test_e2m1_encode_grid_midpoints_ties_saturation_sign():
+    mags = [e2m1_closed_form(c) for c in range(8)]
+    for c, v in enumerate(mags):
+        assert int(O.e2m1_encode(np.array([v], np.float32))[0]) == c
+        if v != 0:
+            assert int(O.e2m1_encode(np.array([-v], np.float32))[0]) == c | 8
+    for c in range(7):
+        a, b = mags[c], mags[c + 1]
+        mid = _f32((a + b) / 2)  # exact: a few significant bits
+        assert int(O.e2m1_encode(np.array([_next_down(mid)]))[0]) == c
+        assert int(O.e2m1_encode(np.array([_next_up(mid)]))[0]) == c + 1
+        even = c if c % 2 == 0 else c + 1  # ties go to the even mantissa bit
+        assert int(O.e2m1_encode(np.array([mid]))[0]) == even
+    # hand-listed ties from the rounding rule
+    ties = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0}
+    for x, want in ties.items():
+        got = float(O.e2m1_value(O.e2m1_encode(np.array([x], np.float32)))[0])
+        assert got == want, (x, got, want)
+    for big in (6.0001, 7.0, 1e30):
+        assert int(O.e2m1_encode(np.array([big], np.float32))[0]) == 7
+        assert int(O.e2m1_encode(np.array([-big], np.float32))[0]) == 15
+    # negative values that round to zero keep the sign bit (reading R6)
+    assert int(O.e2m1_encode(np.array([-0.1], np.float32))[0]) == 8
+    assert int(O.e2m1_encode(np.array([0.1], np.float32))[0]) == 0
+
+
+def test_ue4m3_table_roundtrip_midpoints_saturation_underflow():
+    for c in range(0x7F):
+        assert float(O.ue4m3_value(np.array([c]))[0]) == ue4m3_closed_form(c)
+        assert int(O.ue4m3_encode(np.array([ue4m3_closed_form(c)], np.float32))[0]) == c
+    assert ue4m3_closed_form(0x7E) == 448.0
+    for c in range(0x7E):
+        a, b = ue4m3_closed_form(c), ue4m3_closed_form(c + 1)
+        mid = _f32((a + b) / 2)
+        assert float(mid) == (a + b) / 2
+        assert int(O.ue4m3_encode(np.array([_next_down(mid)]))[0]) == c
+        assert int(O.ue4m3_encode(np.array([_next_up(mid)]))[0]) == c + 1
+        assert int(O.ue4m3_encode(np.array([mid]))[0]) == (c if c % 2 == 0 else c + 1)
+    for big in (448.0001, 464.0, 480.0, 1e9):
+        assert int(O.ue4m3_encode(np.array([big], np.float32))[0]) == 0x7E
+    # half the smallest subnormal is a tie between 0 and 2^-9: goes to 0 (even)
+    assert int(O.ue4m3_encode(np.array([2.0 ** -10], np.float32))[0]) == 0
+    assert int(O.ue4m3_encode(np.array([_next_up(2.0 ** -10)], np.float32))[0]) == 1
+    assert int(O.ue4m3_encode(np.array([2.0 ** -11], np.float32))[0]) == 0
+
+
+def test_int4_rounding_half_even_and_clamp():
+    # one group of 64 with amax 7 -> scale exactly 1, so codes are rint(v)
+    v = np.zeros((1, 64), np.float32)
+    vals = [7.0, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.49, -6.51, 0.0]
+    v[0, :len(vals)] = vals
+    codes, scales = O.quantize_rows(v, O.INT4)
+    assert scales[0, 0] == np.float32(1.0)
+    q = O.int4_value(O.unpack_nibbles(codes))[0, :len(vals)]
+    assert list(q) == [7, 0, 2, 2, 0, -2, -2, 3, -7, 0]
+    # clamp: an element above amax cannot occur; a direct rint beyond 7 is clipped
+    assert np.clip(np.rint(7.6), -8, 7) == 7
+
+
+def test_packing_low_nibble_first():
+    nib = np.array([[1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 0]], np.uint8)
+    p = O.pack_nibbles(nib)
+    assert list(p[0]) == [0x21, 0x43, 0x65, 0x87, 0xA9, 0xCB, 0xED, 0x0F]
+    assert np.array_equal(O.unpack_nibbles(p), nib)
+
+
+def test_bf16_rounding_against_closed_form_and_torch():
+    import torch
+
+    one = 1.0
+    cases = {one + 2.0 ** -8: one, one + 3 * 2.0 ** -8: one + 2.0 ** -6, one + 2.0 ** -8 + 2.0 ** -20: one + 2.0 ** -7,
+             -(one + 2.0 ** -8): -one, 3.0: 3.0}
+    for x, want in cases.items():
+        got = O.bf16_to_f32(O.f32_to_bf16(np.array([x], np.float32)))[0]
+        assert float(got) == want, (x, got, want)
+    rng = np.random.default_rng(0)
+    x = (rng.standard_normal(100000) * np.exp2(rng.integers(-20, 20, 100000))).astype(np.float32)
+    ours = O.f32_to_bf16(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+# ---------------------------------------------------------------- quantizer
+
+
+def _random_on_grid_nvfp4(rng, rows, K, lo=0x08, hi=0x7E):
+    G = 16
+    nblk = K // G
+    scodes = rng.integers(lo, hi, size=(rows, nblk))  # normal UE4M3 scales
+    nib = rng.integers(0, 16, size=(rows, nblk, G)).astype(np.uint8)
+    pos = rng.integers(0, G, size=(rows, nblk))
+    sign = rng.integers(0, 2, size=(rows, nblk)).astype(np.uint8) << 3
+    nib[np.arange(rows)[:, None], np.arange(nblk)[None, :], pos] = 7 | sign  # a +-6 in every block
+    vals = np.array([e2m1_closed_form(int(c)) for c in range(16)])[nib]
+    sval = np.array([ue4m3_closed_form(int(c)) for c in range(0x7F)])[scodes]
+    v = (vals * sval[:, :, None]).reshape(rows, K).astype(np.float32)
+    return v, nib.reshape(rows, K), scodes.astype(np.uint8)
+
+
+def test_nvfp4_values_on_grid_roundtrip_exactly():
+    rng = np.random.default_rng(1)
+    v, nib, scodes = _random_on_grid_nvfp4(rng, 32, 256)
+    codes, scales = O.quantize_rows(v, O.NVFP4)
+    assert np.array_equal(scales, scodes)
+    got = O.unpack_nibbles(codes)
+    # +-0 both decode to 0; the encoder keeps the sign of -0.0 inputs
+    assert np.array_equal(got, nib)
+    assert np.array_equal(O.dequantize_rows(codes, scales, O.NVFP4), v.astype(np.float64))
+
+
+def test_int4_values_on_grid_roundtrip_exactly():
+    rng = np.random.default_rng(2)
+    rows, K, G = 16, 256, 64
+    # scales with <= 20 significant bits so that 7 * s is exact in fp32
+    s = (rng.integers(1 << 19, 1 << 20, size=(rows, K // G)) * 2.0 ** -25).astype(np.float32)
+    q = rng.integers(-7, 8, size=(rows, K // G, G))
+    q[:, :, 0] = 7 * np.where(rng.integers(0, 2, size=(rows, K // G)) > 0, 1, -1)
+    v = (q * s[:, :, None].astype(np.float64)).reshape(rows, K).astype(np.float32)
+    codes, scales = O.quantize_rows(v, O.INT4)
+    assert np.array_equal(scales, s)
+    assert np.array_equal(O.int4_value(O.unpack_nibbles(codes)).reshape(rows, K // G, G), q)
+
+
+def test_quantize_dequantize_idempotent():
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((64, 512)) * np.exp2(rng.integers(-6, 6, (64, 1)))).astype(np.float32)
+    c1, s1 = O.quantize_rows(x, O.NVFP4)
+    d1 = O.dequantize_rows(c1, s1, O.NVFP4).astype(np.float32)
+    c2, s2 = O.quantize_rows(d1, O.NVFP4)
+    nib1 = O.unpack_nibbles(c1).reshape(64, 32, 16)
+    blk6 = np.max(nib1 & 7, axis=2) == 7
+    assert blk6.mean() > 0.5
+    assert np.array_equal(s1[blk6], s2[blk6])
+    nib2 = O.unpack_nibbles(c2).reshape(64, 32, 16)
+    assert np.array_equal(nib1[blk6], nib2[blk6])
+    # INT4: codes equal, scale within one ulp (RN(RN(7s)/7) may move by an ulp)
+    c1, s1 = O.quantize_rows(x, O.INT4)
+    d1 = O.dequantize_rows(c1, s1, O.INT4).astype(np.float32)
+    c2, s2 = O.quantize_rows(d1, O.INT4)
+    assert np.array_equal(c1, c2)
+    ulp = np.spacing(s1)
+    assert np.all(np.abs(s2 - s1) <= ulp)
+
+
+def test_zero_and_underflow_blocks():
+    v = np.zeros((2, 32), np.float32)
+    v[1, :16] = -1e-30  # amax/6 underflows UE4M3 -> zero block, all codes +0
+    v[1, 16:] = 3.0
+    codes, scales = O.quantize_rows(v, O.NVFP4)
+    assert scales[0, 0] == 0 and scales[0, 1] == 0 and scales[1, 0] == 0
+    assert np.all(O.unpack_nibbles(codes)[:, :16] == 0) and np.all(O.unpack_nibbles(codes)[0] == 0)
+    assert float(O.ue4m3_value(scales[1, 1:2])[0]) == 0.5 and np.all(O.unpack_nibbles(codes)[1, 16:] == 7)
+    ci, si = O.quantize_rows(np.zeros((1, 64), np.float32), O.INT4)
+    assert si[0, 0] == 0 and np.all(ci == 0)
+
+
+def test_nvfp4_quantizer_brute_force_scalar_loop():
+    """Scalar restatement of one block with Python floats (fp32 via numpy scalars)."""
+    rng = np.random.default_rng(4)
+    v = (rng.standard_normal((3, 16)) * 3).astype(np.float32)
+    codes, scales = O.quantize_rows(v, O.NVFP4)
+    mags = [e2m1_closed_form(c) for c in range(8)]
+    for r in range(3):
+        amax = max(abs(float(t)) for t in v[r])
+        s = np.float32(np.float32(amax) / np.float32(6.0))
+        # nearest UE4M3, ties to even, by scanning every code
+        best = min(range(0x7F), key=lambda c: (abs(ue4m3_closed_form(c) - float(s)), c % 2))
+        assert scales[r, 0] == best
+        sd = np.float32(ue4m3_closed_form(best))
+        for k in range(16):
+            q = float(np.float32(v[r, k] / sd))
+            c = min(range(8), key=lambda i: (abs(mags[i] - abs(q)), i % 2))
+            want = c | (8 if q < 0 else 0)
+            got = int(O.unpack_nibbles(codes)[r, k])
+            assert got == want
+
+
+# ---------------------------------------------------------------- smoothing + SVD
+
+
+def test_smoothing_closed_form_and_product_invariance():
+    W = np.array([[1.0, -5.0, 0.0], [0.5, 2.0, 0.0]])
+    a = np.array([4.0, 0.0, 9.0])
+    lam = O.smoothing_factors(a, W)
+    assert list(lam) == [2.0, 1.0, 1.0]  # sqrt(4/1); a=0 -> 1; w=0 -> 1
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((7, 12))
+    X[:, 3] *= 40
+    W = rng.standard_normal((5, 12)) * 0.02
+    lam = O.smoothing_factors(np.max(np.abs(X), 0), W)
+    assert np.all(lam > 0)
+    Xh = X / lam[None, :]
+    Wh = O.smooth_weight(W, lam)
+    assert np.allclose(Xh @ Wh.T, X @ W.T, rtol=1e-13, atol=1e-15)
+    # smoothing migrates the outlier: column 3 of X_hat is no longer an outlier
+    assert np.max(np.abs(Xh[:, 3])) < np.max(np.abs(X[:, 3])) / 4
+    # the fp32 activation path divides by lam (multiplies by 1/lam), not the reverse
+    xb = O.f32_to_bf16(X.astype(np.float32))
+    xs = O.smooth_activations(xb, O.inv_lambda_f32(lam)).astype(np.float64)
+    assert np.allclose(xs, O.bf16_to_f32(xb) / lam[None, :], rtol=2e-7)
+
+
+def _householder(rng, n):
+    Q = np.eye(n)
+    for _ in range(3):
+        v = rng.standard_normal(n)
+        v /= np.linalg.norm(v)
+        Q = Q @ (np.eye(n) - 2.0 * np.outer(v, v))
+    return Q
+
+
+def test_svd_recovers_constructed_spectrum():
+    rng = np.random.default_rng(6)
+    K, N = 20, 14
+    Q1 = _householder(rng, K)[:, :N]
+    Q2 = _householder(rng, N)
+    sig = np.linspace(10.0, 1.0, N) ** 2
+    Wkn = Q1 @ np.diag(sig) @ Q2.T
+    r = 5
+    L1, L2, S, U_r, S_r, Vt_r = O.svd_split(Wkn.T, r)
+    assert np.allclose(S, sig, rtol=1e-12)
+    assert L1.shape == (K, r) and L2.shape == (r, N)
+    trunc = Q1[:, :r] @ np.diag(sig[:r]) @ Q2[:, :r].T
+    assert np.linalg.norm(L1 @ L2 - trunc) <= 1e-12 * np.linalg.norm(trunc)
+    for i in range(r):
+        j = int(np.argmax(np.abs(U_r[:, i])))
+        assert U_r[j, i] > 0
+    # balanced split: both factors carry sqrt(sigma)
+    assert np.allclose(np.linalg.norm(L1, axis=0), np.sqrt(sig[:r]), rtol=1e-12)
+    assert np.allclose(np.linalg.norm(L2, axis=1), np.sqrt(sig[:r]), rtol=1e-12)
+
+
+def test_full_rank_residual_is_zero_and_eckart_young():
+    rng = np.random.default_rng(7)
+    N, K = 12, 16
+    W = rng.standard_normal((N, K))
+    L1, L2, S, U_r, S_r, Vt_r = O.svd_split(W, min(N, K))
+    R = O.residual_f32(W, U_r, S_r, Vt_r)
+    assert np.linalg.norm(R.astype(np.float64)) <= 1e-12 * np.linalg.norm(W) + 1e-6 * 0
+    for r in (1, 4, 9):
+        L1, L2, S, U_r, S_r, Vt_r = O.svd_split(W, r)
+        Rr = W - ((U_r * S_r) @ Vt_r).T
+        assert math.isclose(np.sum(Rr ** 2), np.sum(S[r:] ** 2), rel_tol=1e-10)
+        # fp32 residual agrees with the fp64 residual to fp32 rounding
+        assert np.allclose(O.residual_f32(W, U_r, S_r, Vt_r), Rr, rtol=1e-6, atol=1e-6)
+
+
+# ---------------------------------------------------------------- GEMM + forward
+
+
+def test_gemm_4bit_brute_force_grouped_loops():
+    rng = np.random.default_rng(8)
+    for prec, G in ((O.NVFP4, 16), (O.INT4, 64)):
+        M, N, K = 3, 4, 2 * G
+        x = rng.standard_normal((M, K)).astype(np.float32)
+        w = rng.standard_normal((N, K)).astype(np.float32) * 0.1
+        cx, sx = O.quantize_rows(x, prec)
+        cw, sw = O.quantize_rows(w, prec)
+        Y = O.gemm_4bit(cx, sx, cw, sw, prec)
+        nx = O.unpack_nibbles(cx)
+        nw = O.unpack_nibbles(cw)
+
+        def code_val(n):
+            if prec == O.NVFP4:
+                return e2m1_closed_form(int(n))
+            n = int(n)
+            return float(n - 16 if n >= 8 else n)
+
+        def scale_val(s):
+            return ue4m3_closed_form(int(s)) if prec == O.NVFP4 else float(s)
+
+        for m in range(M):
+            for n in range(N):
+                acc = 0.0
+                for g in reversed(range(K // G)):  # a different order from the library matmul
+                    part = 0.0
+                    for k in range(g * G, (g + 1) * G):
+                        part += code_val(nx[m, k]) * code_val(nw[n, k])
+                    acc += scale_val(sx[m, g]) * scale_val(sw[n, g]) * part
+                assert math.isclose(Y[m, n], acc, rel_tol=1e-12, abs_tol=1e-12)
+
+
+def test_forward_lossless_on_grid_equals_exact_product():
+    """lam = 1, r = 0, operands already on the 4-bit grid: quantization is lossless,
+    so the forward equals X W^T + b exactly."""
+    rng = np.random.default_rng(9)
+    v, _, _ = _random_on_grid_nvfp4(rng, 8, 64, 0x20, 0x50)
+    w, _, _ = _random_on_grid_nvfp4(rng, 6, 64, 0x20, 0x50)
+    xb = O.f32_to_bf16(v)
+    assert np.array_equal(O.bf16_to_f32(xb), v)  # on-grid values are bf16 exact
+    inv = np.ones(64, np.float32)
+    xh, cx, sx = O.quantize_activations(xb, inv, O.NVFP4)
+    cw, sw = O.quantize_rows(w, O.NVFP4)
+    bias = O.f32_to_bf16(rng.standard_normal(6).astype(np.float32))
+    Y = O.forward(cx, sx, np.zeros((8, 0), np.uint16), cw, sw, np.zeros((0, 6), np.uint16), bias, O.NVFP4)
+    exact = v.astype(np.float64) @ w.astype(np.float64).T + O.bf16_to_f32(bias)[None, :]
+    assert np.array_equal(Y, exact)
+
+
+def test_lowrank_branch_hand_computed():
+    """x_hat = e_0, L1 row 0 = [1, 2], L2 = [[1,0,0,...],[0,1,0,...]], W = 0, b = 0.5:
+    T = [1, 2], T L2 = [1, 2, 0, ...], Y = [1.5, 2.5, 0.5, ...]."""
+    K, N, r = 16, 5, 2
+    x = np.zeros((1, K), np.float32)
+    x[0, 0] = 1.0
+    L1 = np.zeros((K, r), np.float32)
+    L1[0] = [1.0, 2.0]
+    L2 = np.zeros((r, N), np.float32)
+    L2[0, 0] = 1.0
+    L2[1, 1] = 1.0
+    T = O.lowrank_down(x, O.f32_to_bf16(L1))
+    assert list(O.bf16_to_f32(T)[0]) == [1.0, 2.0]
+    cx, sx = O.quantize_rows(x, O.NVFP4)
+    cw, sw = O.quantize_rows(np.zeros((N, K), np.float32), O.NVFP4)
+    bias = O.f32_to_bf16(np.full(N, 0.5, np.float32))
+    Y = O.forward(cx, sx, T, cw, sw, O.f32_to_bf16(L2), bias, O.NVFP4)
+    assert list(Y[0]) == [1.5, 2.5, 0.5, 0.5, 0.5]
+    # r = 0: the branch is empty and Y is the 4-bit path plus bias
+    T0 = O.lowrank_down(x, np.zeros((K, 0), np.uint16))
+    assert T0.shape == (1, 0)
+
+
+def test_prepare_and_linear_reconstruct_exact_at_full_rank():
+    """Full rank: L1 L2 reproduces W_hat, so the low-rank branch alone (with W's 4-bit
+    part ~0) approximates X W^T to bf16 precision -- pins the orientation of L1/L2."""
+    rng = np.random.default_rng(10)
+    M, K, N = 4, 32, 16
+    X = O.f32_to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    W = O.f32_to_bf16((rng.standard_normal((N, K)) * 0.05).astype(np.float32))
+    a = np.max(np.abs(O.bf16_to_f32(X)), axis=0)
+    ops = O.prepare(W, None, a, O.NVFP4, rank=N)
+    assert np.max(np.abs(ops["R"])) < 1e-6
+    out = O.linear(X, ops, O.NVFP4)
+    exact = O.exact_linear(X, W, None)
+    assert O.rel_fro(out["Y"], exact) < 2e-2
+
+
+def test_svdquant_error_ordering_on_outlier_data():
+    """Model card stage 1-3 claim: smoothing helps 4-bit quantization of outlier
+    activations, and the low-rank branch helps further."""
+    import synth
+
+    spec = synth.get("tiny_256x512x512_r16")
+    X = synth.activations_bf16(spec)
+    W = synth.weight_bf16(spec)
+    b = synth.bias_bf16(spec)
+    exact = O.exact_linear(X, W, b)
+    a = np.max(np.abs(O.bf16_to_f32(X)), axis=0)
+    for prec in (O.NVFP4, O.INT4):
+        plain = O.prepare(W, b, np.zeros_like(a), prec, rank=0)  # a = 0 -> lam = 1
+        smooth = O.prepare(W, b, a, prec, rank=0)
+        svdq = O.prepare(W, b, a, prec, rank=16)
+        e_plain = O.rel_fro(O.linear(X, plain, prec)["Y"], exact)
+        e_smooth = O.rel_fro(O.linear(X, smooth, prec)["Y"], exact)
+        e_svdq = O.rel_fro(O.linear(X, svdq, prec)["Y"], exact)
+        assert e_svdq < e_smooth < e_plain, (prec, e_svdq, e_smooth, e_plain)
+
+
+def test_pages_quantization_config_matches_oracle_groups():
+    with open(os.path.join(HERE, "golden", "quantization_config.json")) as f:
+        cfg = json.load(f)
+    assert cfg["svdq_w4a4"]["precision"] == O.NVFP4
+    assert O.GROUP[O.NVFP4] == cfg["svdq_w4a4"]["group_size"] == 16
+    assert cfg["svdq_w4a4"]["rank"] == 32
+    assert O.GROUP[O.INT4] == 64
