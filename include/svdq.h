@@ -1,0 +1,185 @@
+/*
+ * svdq.h -- C ABI of the B200 (sm_100a) SVDQuant W4A4 rank-corrected smoothed linear layer.
+ *
+ *   Y = Q4(X diag(lam)^-1) (x) Q4(R) + (X diag(lam)^-1 L1) L2 + b
+ *
+ * Sources (the pages this library restates):
+ *   [MC]  SVDQuant model card, huggingface mit-han-lab/svdq-int4-flux.1-depth-dev:
+ *         "Quantization Method -- SVDQuant" (stages 1-3: smoothing migrates outliers
+ *         from X into W, SVD splits the smoothed W into a 16-bit low-rank branch
+ *         L1 L2 and a 4-bit residual R) and "Nunchaku Engine Design" (a)(b)
+ *         (Down Projection fused with Quantize on the shared input; Up Projection
+ *         fused with 4-Bit Compute on the shared output).
+ *   [ND]  "Nunchaku in Diffusers" blog: "Introducing Nunchaku Lite" (svdq_w4a4 kernel
+ *         family, INT4 and NVFP4 variants), "Native loading in Diffusers"
+ *         (quantization_config: precision nvfp4, group_size 16, rank 32,
+ *         compute_dtype bfloat16), "Hardware support" (the GPU capability is checked at
+ *         load time and a clear error is raised instead of wrong outputs).
+ *
+ * Conventions for every call
+ *   - Shapes are nn.Linear shapes: X is M x K, W is N x K (output x input features),
+ *     Y is M x N.  bf16 tensors are passed as uint16_t bit patterns (host) or as
+ *     untyped device pointers.
+ *   - "host" pointers are ordinary CPU memory; "device" pointers are global memory of
+ *     the device the weights were prepared on.  The library never frees caller memory.
+ *   - Every call returns an svdq_status.  Nothing aborts, traps or throws across the
+ *     ABI; svdq_last_error() gives a human-readable message for the calling thread.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Device calls are asynchronous on that stream and never synchronise it, except
+ *     where stated.
+ *   - Precisions: SVDQ_NVFP4 = E2M1 values with one UE4M3 scale per 16 elements along
+ *     K; SVDQ_INT4 = signed 4-bit integers with one fp32 scale per 64 elements along K.
+ *   - Shape limits: K % 256 == 0, N % 8 == 0, 0 <= rank <= 128 with rank % 16 == 0,
+ *     rank <= min(N, K); M >= 0 (any M; row tails are masked); ldx, ldy multiples of 8
+ *     elements; X, Y and workspace 16-byte aligned.
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SVDQ_ABI_VERSION 1
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,        /* null pointer, bad shape, misalignment, workspace too small */
+  SVDQ_ERR_UNSUPPORTED_DEVICE = 2, /* device is not compute capability 10.0 ([ND] "Hardware support") */
+  SVDQ_ERR_CUDA = 3,               /* a CUDA runtime call failed (message in svdq_last_error) */
+  SVDQ_ERR_OOM = 4,                /* a device or host allocation in svdq_prepare_weights failed */
+  SVDQ_ERR_TIMEOUT = 5,            /* a kernel's bounded wait gave up (see svdq_get_device_error) */
+  SVDQ_ERR_INTERNAL = 6
+} svdq_status;
+
+typedef enum { SVDQ_NVFP4 = 0, SVDQ_INT4 = 1 } svdq_precision;
+
+/* Opaque prepared layer: device buffers owned by the library until svdq_free_weights. */
+typedef struct svdq_weights svdq_weights;
+
+/* Offline parameters, the C mirror of [ND] quantization_config's svdq_w4a4 block. */
+typedef struct {
+  int precision;   /* svdq_precision */
+  int rank;        /* r of the low-rank branch; 0 disables it ([MC] stage 3) */
+  float alpha;     /* smoothing exponent: lam_k = a_k^alpha * w_k^(alpha-1); 0.5 gives sqrt(a/w) */
+  int svd_iters;   /* subspace iterations of the randomized SVD; <= 0 selects the default (12) */
+  uint64_t seed;   /* seed of the randomized SVD's Gaussian test matrix */
+} svdq_prepare_params;
+
+/* Shapes and group size of a prepared layer. */
+typedef struct {
+  int N, K, rank, precision, group, device;
+} svdq_weights_info;
+
+/* ------------------------------------------------------------------ status / device */
+
+/* Static string for a status code; never NULL. */
+const char* svdq_status_string(svdq_status s);
+
+/* Detailed message of the last failing call on this thread ("" if none).  The pointer
+ * stays valid until the next call on the same thread. */
+const char* svdq_last_error(void);
+
+/* Load-time capability validation ([ND] "Hardware support": raise a clear error instead
+ * of producing incorrect outputs).  OK only for compute capability 10.0 (B200/GB200). */
+svdq_status svdq_check_device(int device);
+
+/* Synchronises `stream`, then reads and clears the device error word that kernels set
+ * when a bounded wait gives up.  SVDQ_ERR_TIMEOUT if any bit was set, else SVDQ_OK. */
+svdq_status svdq_get_device_error(void* stream);
+
+/* ------------------------------------------------------------------ offline prepare */
+
+/* [MC] stages 2-3, once per layer, on the host except the final uploads:
+ *   lam_k = a_k^alpha w_k^(alpha-1) (a_k = act_absmax[k], w_k = max_n |W[n,k]|; 1 if either is 0),
+ *   W_hat = W diag(lam) (fp64),  top-`rank` SVD of W_hat by randomized subspace iteration,
+ *   L1 = U_r sqrt(S), L2 = sqrt(S) V_r^T (bf16),  R = W_hat - U_r S V_r^T (fp32),
+ *   R quantized per group along K (same quantizer as the activations).
+ * W_bf16:     host, N x K row-major bf16 bits (nn.Linear weight).
+ * bias_bf16:  host, N bf16 bits, or NULL for no bias.
+ * act_absmax: host, K fp32, the calibration statistic max_m |X[m,k]|.
+ * device:     CUDA ordinal that will run the forward; `stream` orders the uploads, and the
+ *             call synchronises it before returning.
+ * out:        receives the handle; free it with svdq_free_weights.
+ * Errors: INVALID_ARG (shape/params), UNSUPPORTED_DEVICE, OOM, CUDA. */
+svdq_status svdq_prepare_weights(const uint16_t* W_bf16, int N, int K, const uint16_t* bias_bf16,
+                                 const float* act_absmax, const svdq_prepare_params* params,
+                                 int device, void* stream, svdq_weights** out);
+
+svdq_status svdq_free_weights(svdq_weights* w);
+
+svdq_status svdq_get_weights_info(const svdq_weights* w, svdq_weights_info* info);
+
+/* Canonical (row-major, untiled) host copies of the prepared operands, for checking the
+ * layer against an independent implementation.  Any pointer may be NULL to skip it.
+ *   inv_lambda: K fp32 (fp32 of 1/lam)         codes_w: N x K/2 bytes (element 2i in bits 3:0)
+ *   scales_w:   NVFP4 N x K/16 UE4M3 bytes;   INT4 N x K/64 fp32
+ *   L1: K x rank bf16    L2: rank x N bf16    bias: N bf16 (zeros when prepared without bias)
+ *   sigma: rank fp64 singular values of W_hat (descending). */
+svdq_status svdq_export_weights(const svdq_weights* w, float* inv_lambda, uint8_t* codes_w,
+                                void* scales_w, uint16_t* L1, uint16_t* L2, uint16_t* bias,
+                                double* sigma);
+
+/* ------------------------------------------------------------------ the hot path */
+
+/* Bytes of device workspace svdq_linear_forward needs for M rows (0 when M == 0). */
+svdq_status svdq_workspace_size(const svdq_weights* w, int M, size_t* bytes);
+
+/* The forward ([MC] "Nunchaku Engine Design"): two kernels on `stream`.
+ *   kernel 1 (Quantize + Down Projection): reads X once; per token and K-group computes
+ *     x_hat = fp32(x) * inv_lambda_k, the group scale and the 4-bit codes, and the bf16
+ *     low-rank product T = bf16(x_hat) L1 (fp32 accumulation, rounded to bf16);
+ *   kernel 2 (4-Bit Compute + Up Projection): block-scaled 4-bit GEMM of the codes against
+ *     Q4(R) on the tensor cores, plus T L2 and the bias into the same fp32 accumulator;
+ *     writes Y = bf16_rn(acc) once.
+ * X:  device, M rows of K bf16, row stride ldx elements.   Y: device, M x N bf16, stride ldy.
+ * workspace: device, >= svdq_workspace_size(w, M) bytes, 256-byte aligned; holds the codes,
+ *   scales and T between the two kernels; contents are scratch.
+ * No allocation, no synchronisation.  Errors: INVALID_ARG, CUDA (launch failure). */
+svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Kernel 1 alone (same arguments as the forward minus Y): fills the workspace. */
+svdq_status svdq_quant_down(const svdq_weights* w, const void* X, int M, int ldx, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* Kernel 2 alone: consumes a workspace filled by svdq_quant_down for the same M. */
+svdq_status svdq_gemm_up(const svdq_weights* w, int M, void* Y, int ldy, const void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Copies kernel 1's outputs out of `workspace` into canonical host layouts (synchronises
+ * `stream`): codes_x M x K/2 bytes, scales_x (NVFP4: M x K/16 UE4M3 bytes; INT4: M x K/64
+ * fp32), T M x rank bf16.  Any output pointer may be NULL. */
+svdq_status svdq_export_activations(const svdq_weights* w, const void* workspace, size_t workspace_bytes,
+                                    int M, uint8_t* codes_x, void* scales_x, uint16_t* T, void* stream);
+
+/* ------------------------------------------------------------------ host-only helpers */
+
+/* The library's host quantizer on fp32 rows (the one svdq_prepare_weights applies to R):
+ * V host rows x K fp32; codes rows x K/2; scales as in svdq_export_weights.  No GPU. */
+svdq_status svdq_quantize_rows_host(const float* V, int rows, int K, int precision, uint8_t* codes,
+                                    void* scales);
+
+/* The offline prepare without a device: same arithmetic as svdq_prepare_weights, results
+ * in the canonical layouts of svdq_export_weights (each output may be NULL). */
+svdq_status svdq_prepare_host(const uint16_t* W_bf16, int N, int K, const uint16_t* bias_bf16,
+                              const float* act_absmax, const svdq_prepare_params* params,
+                              float* inv_lambda, uint8_t* codes_w, void* scales_w, uint16_t* L1,
+                              uint16_t* L2, double* sigma, float* R_out);
+
+/* ------------------------------------------------------------------ failure detection */
+
+/* Launches a one-block kernel that waits, with the library's bounded-wait routine, on a
+ * shared-memory barrier that nothing signals, for at most `spin_limit` polls; on giving up
+ * it sets the device error word and returns.  Lets a test check that a wait that runs out
+ * is reported as SVDQ_ERR_TIMEOUT by svdq_get_device_error while the context stays usable. */
+svdq_status svdq_selftest_wait_timeout(int spin_limit, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */

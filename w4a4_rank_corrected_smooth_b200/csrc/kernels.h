@@ -1,0 +1,40 @@
+// Host launchers of the device kernels (defined in kernels.cu).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace svdq {
+
+struct QuantDownArgs {
+  const uint16_t* X;       // M x K bf16, row stride ldx
+  int M, K, ldx, rank, precision;
+  const float* inv_lambda; // K
+  const uint8_t* l1;       // tiled L1 (layout.h l1_offset)
+  uint8_t* codes;          // workspace: tiled activation codes
+  uint8_t* sf;             // workspace: tiled activation scales
+  uint8_t* t;              // workspace: tiled bf16 T
+};
+
+struct GemmArgs {
+  int M, N, K, rank, precision, ldy;
+  const uint8_t* a_codes;
+  const uint8_t* a_sf;
+  const uint8_t* t;
+  const uint8_t* b_codes;
+  const uint8_t* b_sf;
+  const uint8_t* l2;
+  const float* bias;  // N (padded to a multiple of 256)
+  uint16_t* Y;
+};
+
+// Returns a cudaError_t of the launch (cudaSuccess when the launch was queued).
+cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_selftest_wait(int spin_limit, cudaStream_t stream);
+cudaError_t read_and_clear_device_error(unsigned int* value, cudaStream_t stream);
+
+// Split-K factor (cluster size) kernel 1 uses for a given shape.
+int quant_down_splits(int M, int K, int num_sms);
+
+}  // namespace svdq
