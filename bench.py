@@ -1,0 +1,465 @@
+#!/usr/bin/env python
+"""Benchmark of the SVDQuant W4A4 + rank-32 linear (NVFP4) on the FLUX fused-QKV layer
+(M = 4608 tokens, K = 3072, N = 9216, rank 32) on B200.
+
+One step = one pass of the hot path on one batch: kernel 1 (smoothing + 4-bit quantization +
+bf16 down projection) and kernel 2 (block-scaled 4-bit GEMM + up projection + bias).  Three
+independent copies of the layer (inputs, outputs, workspace and prepared weights; ~400 MB, over
+3x the 126 MB L2) are used in rotation, so no step finds its operands in L2.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead.
+Multi-GPU (torchrun): every rank runs its own replica of the layer (weak scaling, no
+data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4+rank-32 linear TFLOP/s & % FP4 peak; low-rank overhead % on one B200"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "flux_qkv_4608x3072x9216_r32"
+FP4_PER_BF16 = 4.0  # nominal dense ratio: 9 PFLOP/s fp4 / 2.25 PFLOP/s bf16
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCE = os.path.join(ROOT, "w4a4_rank_corrected_smooth_b200", "csrc", "kernels.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=30)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--precision", default="nvfp4")
+    ap.add_argument("--sets", type=int, default=3, help="rotating copies of the layer")
+    ap.add_argument("--no-extras", action="store_true", help="skip overhead, e2e and CPU-baseline legs")
+    ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    with open(KERNEL_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def stored_traffic(kernel: str, workload: str):
+    """dram bytes per launch from a committed ncu summary, if taken on the current kernel source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        e = d[kernel][workload]
+        if e.get("source_sha256") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.tmp = tempfile.NamedTemporaryFile(prefix="svdq_clk_", suffix=".csv", delete=False)
+        self.proc = None
+        self.device_index = device_index
+        self.t_start = self.t_stop = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", str(self.device_index)], stdout=self.tmp, stderr=subprocess.DEVNULL)
+            time.sleep(1.0)
+        except Exception:
+            self.proc = None
+
+    def mark(self, start: bool):
+        if start:
+            self.t_start = time.time()
+        else:
+            self.t_stop = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        self.tmp.close()
+        rows = []
+        try:
+            with open(self.tmp.name) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        finally:
+            os.unlink(self.tmp.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        # nvidia-smi rows carry no timestamps here: keep the loaded ones (power above idle).
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        pw = [num(r[3]) for r in rows]
+        pmax = max([p for p in pw if p is not None] or [0.0])
+        loaded = [r for r, p in zip(rows, pw) if p is not None and p >= 0.5 * pmax] or rows
+        sm = [num(r[1]) for r in loaded if num(r[1]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in loaded:
+            for name, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(loaded[0][2]),
+                "reasons": sorted(reasons), "samples": len(loaded), "power_w_max": pmax}
+
+
+# ---------------------------------------------------------------- helpers
+
+
+def bf16_device(x_bits, device):
+    import numpy as np
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def dist_info():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """Max of a per-rank float over all ranks (identity at world size 1)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def oracle_cpu_baseline(X, ops, precision, spec, budget_s: float = 10.0):
+    """Times the oracle's forward on a row sample of the workload (all N, all K)."""
+    import numpy as np
+    from oracle import svdq_oracle as O
+
+    try:
+        from threadpoolctl import threadpool_info
+
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        cores = os.cpu_count()
+    def timed(rows):
+        t0 = time.perf_counter()
+        O.linear(X[:rows], ops, precision)
+        return time.perf_counter() - t0
+
+    # t(rows) ~ a + b * rows (a: per-call dequantization of W); size the sample for the budget.
+    t_small, t_big = timed(64), timed(512)
+    slope = max((t_big - t_small) / 448.0, 1e-9)
+    fixed = max(t_small - 64 * slope, 0.0)
+    rows = int((budget_s - fixed) / slope)
+    rows = max(64, min(spec.M, rows // 64 * 64))
+    dt = timed(rows)
+    flops = 2 * rows * spec.N * spec.K + 2 * rows * spec.rank * (spec.K + spec.N)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": f"oracle.linear (fp64) on rows 0..{rows - 1} of {spec.M} (all {spec.N} outputs, K={spec.K}), "
+                      f"one call, {dt:.2f} s wall"}
+
+
+# ---------------------------------------------------------------- reference arm
+
+
+def run_reference(args):
+    """The CPU oracle, as it stands, on the same workload/metric: each step is oracle.linear on a
+    block of output rows x columns sized so that warm-up + steps end within a few minutes."""
+    import numpy as np
+
+    import synth
+    from oracle import svdq_oracle as O
+
+    world, rank, _ = dist_info()
+    if rank != 0:
+        return
+    spec = synth.get(args.workload)
+    X = synth.activations_bf16(spec)
+    W = synth.weight_bf16(spec)
+    b = synth.bias_bf16(spec)
+    a = synth.act_absmax(X)
+    ops = O.prepare(W, b, a, args.precision, spec.rank)
+    try:
+        from threadpoolctl import threadpool_info
+
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        cores = os.cpu_count()
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    rows, cols = 16, 64
+
+    def sliced(c0, cols):
+        d = dict(ops)
+        d["codes_w"] = ops["codes_w"][c0:c0 + cols]
+        d["scales_w"] = ops["scales_w"][c0:c0 + cols]
+        d["L2"] = ops["L2"][:, c0:c0 + cols]
+        d["bias"] = ops["bias"][c0:c0 + cols]
+        return d
+
+    t0 = time.perf_counter()
+    O.linear(X[:rows], sliced(0, cols), args.precision)
+    dt = time.perf_counter() - t0
+    while dt * 4 < budget and (rows < spec.M or cols < spec.N):
+        if cols < spec.N:
+            cols = min(spec.N, cols * 2)
+        else:
+            rows = min(spec.M, rows * 2)
+        t0 = time.perf_counter()
+        O.linear(X[:rows], sliced(0, cols), args.precision)
+        dt = time.perf_counter() - t0
+    flops = 2 * rows * cols * spec.K + 2 * rows * spec.rank * (spec.K + cols)
+    rng = np.random.default_rng(0)
+    for i in range(args.warmup):
+        r0 = int(rng.integers(0, spec.M - rows + 1))
+        c0 = int(rng.integers(0, (spec.N - cols) // 8 + 1)) * 8
+        O.linear(X[r0:r0 + rows], sliced(c0, cols), args.precision)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        r0 = int(rng.integers(0, spec.M - rows + 1))
+        c0 = int(rng.integers(0, (spec.N - cols) // 8 + 1)) * 8
+        O.linear(X[r0:r0 + rows], sliced(c0, cols), args.precision)
+    total = time.perf_counter() - t0
+    value = flops * args.steps / total / 1e12
+    sample = f"per step: oracle.linear on a {rows} x {cols} block of Y (K={spec.K}) of {spec.M} x {spec.N}"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "rank": spec.rank,
+                   "precision": args.precision},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(cores), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+
+
+def time_loop(layers, sets, steps, stream):
+    """Runs `steps` steps rotating over `sets`; returns (total_ms, mean k1 ms, mean k2 ms)."""
+    import torch
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        lin = layers[i % len(layers)]
+        X, Y, ws = sets[i % len(sets)]
+        M = X.shape[0]
+        ev[i][0].record(stream)
+        lin.svdq_quant_down(X, M, X.stride(0), ws, ws.numel(), stream)
+        ev[i][1].record(stream)
+        lin.svdq_gemm_up(M, Y, Y.stride(0), ws, ws.numel(), stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    total = ev[0][0].elapsed_time(ev[-1][2])
+    k1 = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+    k2 = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+    return total, k1, k2
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    import synth
+    import w4a4_rank_corrected_smooth_b200 as S
+
+    world, rank, local = dist_info()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    S.svdq_check_device(local)
+    stream = torch.cuda.current_stream(dev)
+    spec = synth.get(args.workload)
+    X = synth.activations_bf16(spec)
+    W = synth.weight_bf16(spec)
+    b = synth.bias_bf16(spec)
+    a = synth.act_absmax(X)
+    lin = S.SVDQLinear(W, b, a, args.precision, spec.rank, device=local)
+    layers = [lin] + [lin.clone() for _ in range(args.sets - 1)]
+    Xd = bf16_device(X, dev)
+    sets = []
+    for s in range(args.sets):
+        perm = torch.randperm(spec.M, generator=torch.Generator().manual_seed(s)).to(dev)
+        Xs = Xd if s == 0 else Xd[perm].contiguous()
+        Ys = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=dev)
+        ws = lin.new_workspace(spec.M)
+        sets.append((Xs, Ys, ws))
+    peaks, peak_src = load_peaks()
+
+    sampler = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local])
+                           if os.environ.get("CUDA_VISIBLE_DEVICES") else local)
+    if not args.no_clocks:
+        sampler.start()
+    time_loop(layers, sets, max(3, args.warmup), stream)
+    S.svdq_get_device_error(stream)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.mark(True)
+    total_ms, k1_ms, k2_ms = time_loop(layers, sets, args.steps, stream)
+    torch.cuda.synchronize()
+    sampler.mark(False)
+    barrier(world)
+    clocks = sampler.stop() if not args.no_clocks else None
+    S.svdq_get_device_error(stream)
+    total_ms = max_over_ranks(total_ms, world)
+
+    flops = spec.flops
+    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    k2_flops = spec.flops_4bit + 2 * spec.M * spec.rank * spec.N
+    k2_tflops = k2_flops / (k2_ms / 1e3) / 1e12
+    fp4_peak_sustained = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
+    fp4_peak_burst = peaks["bf16_tflops"] * FP4_PER_BF16
+    k1_bytes = (2 * spec.M * spec.K + spec.M * spec.K // 2 + spec.M * spec.K // 16 + 2 * spec.K * spec.rank
+                + 2 * spec.M * spec.rank)
+    k2_bytes = (spec.M * spec.K // 2 + spec.M * spec.K // 16 + spec.N * spec.K // 2 + spec.N * spec.K // 16
+                + 2 * spec.M * spec.rank + 2 * spec.N * spec.rank + 4 * spec.N + 2 * spec.M * spec.N)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4" if args.precision == "nvfp4" else "int4",
+        "data": "synthetic (seeded FLUX-shaped activations with 0.5% x30 outlier channels, W ~ N(0, 0.02))",
+        "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "rank": spec.rank,
+                   "precision": args.precision, "parallelism": f"replicas x{world}",
+                   "l2": f"{args.sets} rotating copies of X/Y/workspace/weights (> 3x L2), no flush"},
+        "fp4_peak_frac": value / world / fp4_peak_sustained,
+        "kernel_ms": {"quant_down": k1_ms, "gemm": k2_ms},
+        "roofline": {"bound": "tensor", "achieved": k2_tflops, "peak": fp4_peak_sustained, "unit": "TFLOP/s",
+                     "frac": k2_tflops / fp4_peak_sustained, "traffic": stored_traffic("gemm", spec.name),
+                     "kernel": "gemm_nvfp4_kernel",
+                     "peak_source": f"{peak_src} bf16 sustained x {FP4_PER_BF16:g} (nominal fp4/bf16)",
+                     "frac_of_burst_peak": k2_tflops / fp4_peak_burst,
+                     "algorithmic_flops_per_launch": k2_flops},
+        "quant_down_roofline": {"bound": "hbm", "achieved": k1_bytes / (k1_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                                "unit": "GB/s", "frac": k1_bytes / (k1_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                                "traffic": stored_traffic("quant_down", spec.name),
+                                "algorithmic_bytes_per_launch": k1_bytes},
+        "gemm_algorithmic_bytes_per_launch": k2_bytes,
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+
+    if not args.no_extras:
+        # Low-rank overhead: the same layer prepared with rank 0, timed the same way.
+        lin0 = S.SVDQLinear(W, b, a, args.precision, 0, device=local)
+        layers0 = [lin0] + [lin0.clone() for _ in range(args.sets - 1)]
+        sets0 = [(x, y, lin0.new_workspace(spec.M)) for (x, y, _) in sets]
+        n_over = min(args.steps, 1000)
+        time_loop(layers0, sets0, max(3, args.warmup), stream)
+        _, k1_0, k2_0 = time_loop(layers0, sets0, n_over, stream)
+        _, k1_r, k2_r = time_loop(layers, sets, n_over, stream)
+        S.svdq_get_device_error(stream)
+        over = (k1_r + k2_r - k1_0 - k2_0)
+        line["lowrank_overhead_pct"] = 100.0 * over / k2_0
+        line["lowrank_overhead_detail"] = {
+            "rank": spec.rank, "ms_rank": {"quant_down": k1_r, "gemm": k2_r},
+            "ms_rank0": {"quant_down": k1_0, "gemm": k2_0},
+            "pct_of_bare_gemm": 100.0 * over / k2_0, "pct_of_bare_layer": 100.0 * over / (k1_0 + k2_0)}
+        for l0 in layers0:
+            l0.close()
+        # End to end through the public API: pinned host X -> device, forward, Y -> pinned host.
+        Xh = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).pin_memory()
+        Yh = torch.empty((spec.M, spec.N), dtype=torch.bfloat16).pin_memory()
+        Xe, Ye, wse = sets[0]
+        n_e2e = min(args.steps, 30)
+        for _ in range(3):
+            Xe.copy_(Xh, non_blocking=True)
+            lin.svdq_linear_forward(Xe, spec.M, spec.K, Ye, spec.N, wse, wse.numel(), stream)
+            Yh.copy_(Ye, non_blocking=True)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            Xe.copy_(Xh, non_blocking=True)
+            lin.svdq_linear_forward(Xe, spec.M, spec.K, Ye, spec.N, wse, wse.numel(), stream)
+            Yh.copy_(Ye, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
+        line["e2e"] = {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+                       "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yh.numel() * 2),
+                       "ms_per_step": e2e_ms, "steps": n_e2e}
+        if world == 1:
+            line["cpu_baseline"] = oracle_cpu_baseline(X, lin.export_weights(), args.precision, spec)
+    for l in layers:
+        l.close()
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, _, _ = dist_info()
+    if world != args.gpus and not (world == 1 and args.gpus == 1):
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

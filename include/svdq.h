@@ -111,6 +111,11 @@ svdq_status svdq_prepare_weights(const uint16_t* W_bf16, int N, int K, const uin
 
 svdq_status svdq_free_weights(svdq_weights* w);
 
+/* A second, independent handle holding device copies of `src`'s buffers (same device, same
+ * operands; copies ordered on `stream`, which the call synchronises).  Useful to run several
+ * instances of a layer without repeating the offline SVD.  Errors: INVALID_ARG, OOM, CUDA. */
+svdq_status svdq_clone_weights(const svdq_weights* src, void* stream, svdq_weights** out);
+
 svdq_status svdq_get_weights_info(const svdq_weights* w, svdq_weights_info* info);
 
 /* Canonical (row-major, untiled) host copies of the prepared operands, for checking the

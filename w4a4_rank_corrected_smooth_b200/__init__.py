@@ -43,7 +43,7 @@ class WeightsInfo(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m w4a4_rank_corrected_smooth_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python w4a4_rank_corrected_smooth_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     sig = {
@@ -53,6 +53,7 @@ def _load() -> ctypes.CDLL:
         "svdq_get_device_error": ([vp], i),
         "svdq_prepare_weights": ([vp, i, i, vp, vp, ctypes.POINTER(PrepareParams), i, vp, ctypes.POINTER(vp)], i),
         "svdq_free_weights": ([vp], i),
+        "svdq_clone_weights": ([vp, vp, ctypes.POINTER(vp)], i),
         "svdq_get_weights_info": ([vp, ctypes.POINTER(WeightsInfo)], i),
         "svdq_export_weights": ([vp, vp, vp, vp, vp, vp, vp, vp], i),
         "svdq_workspace_size": ([vp, i, ctypes.POINTER(sz)], i),
@@ -74,7 +75,7 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 DECLARED_SYMBOLS = tuple(sorted([
     "svdq_status_string", "svdq_last_error", "svdq_check_device", "svdq_get_device_error", "svdq_prepare_weights",
-    "svdq_free_weights", "svdq_get_weights_info", "svdq_export_weights", "svdq_workspace_size", "svdq_linear_forward",
+    "svdq_free_weights", "svdq_clone_weights", "svdq_get_weights_info", "svdq_export_weights", "svdq_workspace_size", "svdq_linear_forward",
     "svdq_quant_down", "svdq_gemm_up", "svdq_export_activations", "svdq_quantize_rows_host", "svdq_prepare_host",
     "svdq_selftest_wait_timeout"]))
 
@@ -181,6 +182,15 @@ class SVDQLinear:
         _check(_lib.svdq_prepare_weights(_ptr(W), self.N, self.K, _ptr(b), _ptr(a), ctypes.byref(p), device,
                                          _stream(stream), ctypes.byref(h)))
         self._h = h
+
+    def clone(self, stream=None) -> "SVDQLinear":
+        """An independent copy of this prepared layer (device buffers duplicated, no re-prepare)."""
+        h = ctypes.c_void_p()
+        _check(_lib.svdq_clone_weights(self._h, _stream(stream), ctypes.byref(h)))
+        other = object.__new__(SVDQLinear)
+        other.N, other.K, other.rank, other.precision, other.device = self.N, self.K, self.rank, self.precision, self.device
+        other._h = h
+        return other
 
     def close(self) -> None:
         if self._h is not None:

@@ -1,6 +1,7 @@
 """Builds the C-ABI shared library ``lib/libsvdq_b200.so`` in-tree for sm_100a.
 
-Usage: ``python -m w4a4_rank_corrected_smooth_b200.build [--force]``.  nvcc cross-compiles,
+Usage: ``python w4a4_rank_corrected_smooth_b200/build.py [--force]`` (run by path: importing the
+package loads the library this script builds).  nvcc cross-compiles,
 so this runs on a machine without a GPU.  Objects go to ``_build/`` next to this file.
 """
 from __future__ import annotations

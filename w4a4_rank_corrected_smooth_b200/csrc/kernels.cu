@@ -16,6 +16,7 @@
 // (kind::mxf4nvf4 with UE4M3 scales copied into tensor memory by tcgen05.cp) into the same fp32
 // accumulator in tensor memory; eight epilogue warps drain the accumulator, add the bias and
 // write bf16 Y once.
+#include <cuda.h>
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -26,14 +27,19 @@ namespace svdq {
 
 // ============================================================================ kernel 1
 
-constexpr int kQdStages = 4;
-constexpr int kQdWorkerWarps = 8;
-constexpr int kQdThreads = (kQdWorkerWarps + 1) * 32;
-constexpr int kXsBytes = kBM * 128;  // bf16 x_hat: 128 rows x 64 columns, 128-byte swizzle
+constexpr int kQdMaxStages = 8;
+constexpr int kQdWorkerWarps = 16;
+constexpr int kQdMmaWarp = kQdWorkerWarps;        // tcgen05 MMA issuer (+ TMEM owner)
+constexpr int kQdTmaWarp = kQdWorkerWarps + 1;    // TMA producer
+constexpr int kQdThreads = (kQdWorkerWarps + 2) * 32;
+constexpr uint32_t kXsBytes = kBM * 128;  // one stage of X: 128 rows x 64 bf16, 128-byte swizzle
+constexpr size_t kQdSmemBudget = 220 * 1024;
+// Relative nudges that bracket a correctly rounded quotient (see the worker loop).
+constexpr float kNudgeLo = 1.0f - 0x1p-20f;
+constexpr float kNudgeHi = 1.0f + 0x1p-20f;
 
 struct QdParams {
-  const uint16_t* X;
-  int M, K, ldx, rank, KB, splits;
+  int M, K, rank, KB, splits, stages;
   const float* inv_lambda;
   const uint8_t* l1;
   uint8_t* codes;
@@ -41,71 +47,107 @@ struct QdParams {
   uint8_t* t;
 };
 
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Quantizes this lane's 8 smoothed values (a 16-group spans a lane pair; a 64-group spans the 8
-// lanes of a row).  Returns the packed codes (element 2i in the low nibble of byte i) and, in
-// `scale_bits`, the group scale (UE4M3 byte or fp32 bits).
-template <int PREC>
-__device__ __forceinline__ uint32_t quantize8(const float (&xh)[8], uint32_t& scale_bits) {
-  float amax = 0.0f;
+// Two fp32 lanes in one 64-bit register for the packed (f32x2) FP pipe of sm_100.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// Element-wise round-to-nearest product of two fp32 pairs.
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// E2M1 codes (RNE, saturating) of the 8 values held as 4 fp32 pairs; element 2i in the low nibble.
+__device__ __forceinline__ uint32_t e2m1x8_pairs(const uint64_t (&v)[4]) {
+  float a[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(xh[j]));
-  uint32_t codes = 0;
-  if (PREC == 0) {
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    const float s = __fdiv_rn(amax, 6.0f);
-    const uint32_t sc = cvt_e4m3(s);
-    const float sd = e4m3_to_f32(sc);
-    scale_bits = sc;
-    if (sd != 0.0f) {
+  for (int t = 0; t < 4; ++t) f2unpack(v[t], a[2 * t], a[2 * t + 1]);
+  uint32_t c;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(c)
+      : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]), "f"(a[7]));
+  return c;
+}
+
+// E2M1 codes of x[j] * mul (each product rounded to nearest), element 2i in the low nibble of byte i.
+__device__ __forceinline__ uint32_t e2m1x8_scaled(const uint64_t (&x)[4], float mul) {
+  const uint64_t m = f2pack(mul, mul);
+  uint64_t q[4];
 #pragma unroll
-      for (int t = 0; t < 4; ++t)
-        codes |= cvt_e2m1x2(__fdiv_rn(xh[2 * t], sd), __fdiv_rn(xh[2 * t + 1], sd)) << (8 * t);
-    }
-  } else {
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-    const float s = __fdiv_rn(amax, 7.0f);
-    scale_bits = __float_as_uint(s);
-    if (s != 0.0f) {
+  for (int t = 0; t < 4; ++t) q[t] = f2mul(x[t], m);
+  return e2m1x8_pairs(q);
+}
+
+// The exact codes E2M1_rne(RN(x / sd)) with IEEE divisions (rare path).
+__device__ __forceinline__ uint32_t e2m1x8_div(const float (&v)[8], float sd) {
+  uint32_t c = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        int q = __float2int_rn(__fdiv_rn(xh[j], s));
-        q = max(-8, min(7, q));
-        codes |= (static_cast<uint32_t>(q) & 0xFu) << (4 * j);
-      }
-    }
+  for (int t = 0; t < 4; ++t) c |= cvt_e2m1x2(__fdiv_rn(v[2 * t], sd), __fdiv_rn(v[2 * t + 1], sd)) << (8 * t);
+  return c;
+}
+
+__device__ __forceinline__ uint32_t int4x8(const float (&v)[8], float mul) {
+  uint32_t c = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float q = fminf(7.0f, fmaxf(-8.0f, rintf(__fmul_rn(v[j], mul))));
+    c |= (static_cast<uint32_t>(static_cast<int>(q)) & 0xFu) << (4 * j);
   }
-  return codes;
+  return c;
+}
+
+__device__ __forceinline__ uint32_t int4x8_div(const float (&v)[8], float s) {
+  uint32_t c = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int q = max(-8, min(7, __float2int_rn(__fdiv_rn(v[j], s))));
+    c |= (static_cast<uint32_t>(q) & 0xFu) << (4 * j);
+  }
+  return c;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
 }
 
 template <int PREC>
-__global__ void __launch_bounds__(kQdThreads, 1) quant_down_kernel(const QdParams p) {
-  extern __shared__ uint8_t smem_raw[];
+__global__ void __launch_bounds__(kQdThreads, 1)
+    quant_down_kernel(const __grid_constant__ CUtensorMap tmap_x, const QdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ float rcp_tbl[128];  // RN(1 / UE4M3 value) for every finite scale code
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int r = p.rank;
+  const int NS = p.stages;
   const bool has_lr = r > 0;
-  const uint32_t l1_stage_bytes = static_cast<uint32_t>(r) * 128u;
-  uint8_t* xs = smem;                                              // kQdStages x 16 KB
-  uint8_t* l1s = smem + kQdStages * kXsBytes;                      // kQdStages x r*128
-  uint64_t* bars = reinterpret_cast<uint64_t*>(l1s + kQdStages * align_up(l1_stage_bytes, 1024));
-  uint64_t* xfull = bars;                   // workers -> MMA (count 8)
-  uint64_t* l1full = bars + kQdStages;      // L1 copy landed (count 1 + tx)
-  uint64_t* empty = bars + 2 * kQdStages;   // MMA done reading the stage (tcgen05.commit)
-  uint64_t* done = bars + 3 * kQdStages;    // all MMAs of this CTA complete
+  const uint32_t l1_bytes = static_cast<uint32_t>(r) * 128u;
+  const uint32_t l1_stride = static_cast<uint32_t>(align_up(l1_bytes, 1024));
+  uint8_t* xs = smem;                       // NS x 16 KB (X, then bf16 x_hat in place)
+  uint8_t* l1s = smem + NS * kXsBytes;      // NS x r*128 (L1 chunk)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(l1s + NS * l1_stride);
+  uint64_t* full = bars;                    // TMA landed: X tile (+ L1 chunk)
+  uint64_t* xready = bars + NS;             // workers wrote x_hat (one arrive per worker warp)
+  uint64_t* empty = bars + 2 * NS;          // stage free again
+  uint64_t* done = bars + 3 * NS;           // all MMAs of this CTA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -117,16 +159,17 @@ __global__ void __launch_bounds__(kQdThreads, 1) quant_down_kernel(const QdParam
   const uint32_t tmem_cols = r <= 32 ? 32u : (r <= 64 ? 64u : 128u);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kQdStages; ++s) {
-      mbar_init(&xfull[s], kQdWorkerWarps);
-      mbar_init(&l1full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&xready[s], kQdWorkerWarps);
+      mbar_init(&empty[s], has_lr ? 1 : kQdWorkerWarps);
     }
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (has_lr && warp == kQdWorkerWarps) {
+  if (PREC == 0 && threadIdx.x < 128) rcp_tbl[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __frcp_rn(e4m3_to_f32(threadIdx.x));
+  if (has_lr && warp == kQdMmaWarp) {
     tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
   }
@@ -137,130 +180,187 @@ __global__ void __launch_bounds__(kQdThreads, 1) quant_down_kernel(const QdParam
 
   if (warp < kQdWorkerWarps) {
     // ------------------------------------------------------------ workers
+    // Lane (sub, kg) of warp w handles 8 consecutive columns (16-byte unit kg) of rows
+    // 8w + sub and 8w + 4 + sub.  Quantization is exact (codes = E2M1_rne(RN(x / s)), resp.
+    // rint): the quotient is bracketed between x * RN(RN(1/s)(1 -+ 2^-20)); both roundings are
+    // monotonic, so when the two bracketing codes agree they are the exact codes, and
+    // otherwise (x/s within ~2^-20 of a threshold) the IEEE division decides.
     const int sub = lane >> 3, kg = lane & 7;
-    const uint8_t* xrow[4];
-    bool rvalid[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int row = mt * kBM + warp * 16 + i * 4 + sub;
-      rvalid[i] = row < p.M;
-      xrow[i] = reinterpret_cast<const uint8_t*>(p.X + static_cast<size_t>(rvalid[i] ? row : 0) * p.ldx);
-    }
-    uint4 cur[4], nxt[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int col = c0 * 64 + kg * 8;
-      cur[i] = rvalid[i] ? ld_stream_v4(xrow[i] + static_cast<size_t>(col) * 2) : make_uint4(0, 0, 0, 0);
-    }
+    const float kInv6 = __frcp_rn(6.0f);
     for (int c = 0; c < nch; ++c) {
-      const int gc = c0 + c;
-      if (c + 1 < nch) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int col = (gc + 1) * 64 + kg * 8;
-          nxt[i] = rvalid[i] ? ld_stream_v4(xrow[i] + static_cast<size_t>(col) * 2) : make_uint4(0, 0, 0, 0);
-        }
+      const int st = c % NS;
+      const bool ok = !*abort_flag && wait_parity_bounded(&full[st], (c / NS) & 1, kErrWaitQuantDown);
+      if (!__all_sync(0xffffffffu, ok)) {
+        *abort_flag = 1;
+        break;
       }
+      const int gc = c0 + c;
       const int col = gc * 64 + kg * 8;
       const float4 il0 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + col));
       const float4 il1 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + col + 4));
       const float il[8] = {il0.x, il0.y, il0.z, il0.w, il1.x, il1.y, il1.z, il1.w};
       const int kb = gc >> 2, cc = gc & 3;
-      const int st = c % kQdStages;
-      if (has_lr && c >= kQdStages) {
-        if (!wait_parity_bounded(&empty[st], ((c / kQdStages) - 1) & 1, kErrWaitQuantDown)) {
-          *abort_flag = 1;
-          break;
-        }
-      }
       uint8_t* codes_chunk = p.codes + codes_chunk_offset(mt, kb, p.KB, kBM);
       uint8_t* sf_chunk = p.sf + sf_chunk_offset(mt, kb, p.KB, kBM);
+      uint8_t* xt = xs + st * kXsBytes;
+      int row[2];
+      uint4* cell[2];
+      float xh[2][8];
+      uint64_t xp[2][4];  // the same values as fp32 pairs
+      float amax[2];
+      uint64_t ilp[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int row = warp * 16 + i * 4 + sub;  // row inside the tile
-        const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
-        float xh[8];
+      for (int t = 0; t < 4; ++t) ilp[t] = f2pack(il[2 * t], il[2 * t + 1]);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        row[i] = warp * 8 + i * 4 + sub;
+        cell[i] = reinterpret_cast<uint4*>(xt + swz128(row[i], kg * 16));
+        const uint4 xv = *cell[i];
+        const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          xh[2 * t] = __fmul_rn(__uint_as_float(w[t] << 16), il[2 * t]);
-          xh[2 * t + 1] = __fmul_rn(__uint_as_float(w[t] & 0xFFFF0000u), il[2 * t + 1]);
+          // bf16 -> fp32 is exact; x_hat = fp32(x) * (1/lambda), one rounding per element
+          xp[i][t] = f2mul(f2pack(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xFFFF0000u)), ilp[t]);
+          f2unpack(xp[i][t], xh[i][2 * t], xh[i][2 * t + 1]);
         }
-        uint32_t sbits;
-        const uint32_t codes = quantize8<PREC>(xh, sbits);
-        *reinterpret_cast<uint32_t*>(codes_chunk + swz128(row, cc * 32 + kg * 4)) = codes;
+        amax[i] = fmaxf(fmaxf(fmaxf(fabsf(xh[i][0]), fabsf(xh[i][1])), fmaxf(fabsf(xh[i][2]), fabsf(xh[i][3]))),
+                        fmaxf(fmaxf(fabsf(xh[i][4]), fabsf(xh[i][5])), fmaxf(fabsf(xh[i][6]), fabsf(xh[i][7]))));
+      }
+      uint32_t codes[2], sbits[2];
+      if (PREC == 0) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 1));
+        bool slow = false;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          // scale code: UE4M3_rne(RN(amax / 6)), bracketed the same way
+          const float s_est = __fmul_rn(amax[i], kInv6);
+          const uint32_t sc_lo = cvt_e4m3(__fmul_rn(s_est, kNudgeLo));
+          const uint32_t sc_hi = cvt_e4m3(__fmul_rn(s_est, kNudgeHi));
+          sbits[i] = sc_lo;
+          codes[i] = 0;
+          if (sc_lo == sc_hi) {
+            if (sc_lo != 0) {
+              const float rr = rcp_tbl[sc_lo];
+              const uint32_t lo = e2m1x8_scaled(xp[i], __fmul_rn(rr, kNudgeLo));
+              const uint32_t hi = e2m1x8_scaled(xp[i], __fmul_rn(rr, kNudgeHi));
+              codes[i] = lo;
+              slow |= lo != hi;
+            }
+          } else {
+            slow = true;
+          }
+        }
+        if (slow) {  // rare: recompute both rows exactly
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const uint32_t sc = cvt_e4m3(__fdiv_rn(amax[i], 6.0f));
+            const float sd = e4m3_to_f32(sc);
+            sbits[i] = sc;
+            codes[i] = sd != 0.0f ? e2m1x8_div(xh[i], sd) : 0u;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 1));
+          amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 2));
+          amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 4));
+        }
+        bool slow = false;
+        float sc[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          sc[i] = __fdiv_rn(amax[i], 7.0f);
+          sbits[i] = __float_as_uint(sc[i]);
+          codes[i] = 0;
+          if (sc[i] != 0.0f) {
+            const float rr = __frcp_rn(sc[i]);
+            if (rr < 1e30f) {
+              const uint32_t lo = int4x8(xh[i], __fmul_rn(rr, kNudgeLo));
+              const uint32_t hi = int4x8(xh[i], __fmul_rn(rr, kNudgeHi));
+              codes[i] = lo;
+              slow |= lo != hi;
+            } else {
+              slow = true;  // tiny scale: reciprocal out of range
+            }
+          }
+        }
+        if (slow) {
+#pragma unroll
+          for (int i = 0; i < 2; ++i) codes[i] = sc[i] != 0.0f ? int4x8_div(xh[i], sc[i]) : 0u;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        *reinterpret_cast<uint32_t*>(codes_chunk + swz128(row[i], cc * 32 + kg * 4)) = codes[i];
         if (PREC == 0) {
-          const uint32_t s1 = __shfl_down_sync(0xffffffffu, sbits, 2);
-          const uint32_t s2 = __shfl_down_sync(0xffffffffu, sbits, 4);
-          const uint32_t s3 = __shfl_down_sync(0xffffffffu, sbits, 6);
-          if (kg == 0)
-            *reinterpret_cast<uint32_t*>(sf_chunk + cc * 512 + (row & 31) * 16 + (row >> 5) * 4) =
-                sbits | (s1 << 8) | (s2 << 16) | (s3 << 24);
+          // the pair (kg, kg+1) shares one 16-group; the even lane stores its scale byte
+          if ((kg & 1) == 0)
+            sf_chunk[cc * 512 + (row[i] & 31) * 16 + (row[i] >> 5) * 4 + (kg >> 1)] = static_cast<uint8_t>(sbits[i]);
         } else {
-          if (kg == 0) reinterpret_cast<uint32_t*>(sf_chunk)[sf_int4_a_index(row, cc)] = sbits;
+          if (kg == 0) reinterpret_cast<uint32_t*>(sf_chunk)[sf_int4_a_index(row[i], cc)] = sbits[i];
         }
         if (has_lr) {
           uint4 hv;
-          hv.x = pack_bf16x2(xh[0], xh[1]);
-          hv.y = pack_bf16x2(xh[2], xh[3]);
-          hv.z = pack_bf16x2(xh[4], xh[5]);
-          hv.w = pack_bf16x2(xh[6], xh[7]);
-          *reinterpret_cast<uint4*>(xs + st * kXsBytes + swz128(row, kg * 16)) = hv;
+          hv.x = pack_bf16x2(xh[i][0], xh[i][1]);
+          hv.y = pack_bf16x2(xh[i][2], xh[i][3]);
+          hv.z = pack_bf16x2(xh[i][4], xh[i][5]);
+          hv.w = pack_bf16x2(xh[i][6], xh[i][7]);
+          *cell[i] = hv;  // bf16(x_hat) in place: the tile becomes the MMA's A operand
         }
       }
-      if (has_lr) {
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&xfull[st]);
+      if (has_lr) fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(has_lr ? &xready[st] : &empty[st]);
+    }
+  } else if (warp == kQdTmaWarp) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      int issued = 0;
+      for (int c = 0; c < nch; ++c) {
+        const int st = c % NS;
+        if (c >= NS && (*abort_flag || !wait_parity_bounded(&empty[st], ((c / NS) - 1) & 1, kErrWaitQuantDown))) {
+          *abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[st], kXsBytes + (has_lr ? l1_bytes : 0u));
+        tma_load_2d(xs + st * kXsBytes, &tmap_x, (c0 + c) * 64, mt * kBM, &full[st]);
+        if (has_lr)
+          bulk_g2s(l1s + st * l1_stride, p.l1 + static_cast<size_t>(c0 + c) * l1_bytes, l1_bytes, &full[st]);
+        ++issued;
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
+      if (*abort_flag) {
+        // Let every issued copy land before the CTA can retire.
+        for (int q = (issued > NS ? issued - NS : 0); q < issued; ++q)
+          wait_parity_bounded(&full[q % NS], (q / NS) & 1, kErrWaitQuantDown);
+      }
     }
   } else if (has_lr && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     const uint32_t idesc = idesc_bf16(128, r);
-    int pcount = 0;  // L1 chunks whose copy has been issued
-    bool ok = true;
-    for (int c = 0; c < nch && ok; ++c) {
-      while (pcount < nch && pcount < c + kQdStages) {
-        const int sp = pcount % kQdStages;
-        if (pcount >= kQdStages && !wait_parity_bounded(&empty[sp], ((pcount / kQdStages) - 1) & 1, kErrWaitQuantDown)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&l1full[sp], l1_stage_bytes);
-        bulk_g2s(l1s + sp * align_up(l1_stage_bytes, 1024), p.l1 + static_cast<size_t>(c0 + pcount) * l1_stage_bytes,
-                 l1_stage_bytes, &l1full[sp]);
-        ++pcount;
-      }
-      if (!ok) break;
-      const int st = c % kQdStages;
-      const uint32_t par = (c / kQdStages) & 1;
-      if (!wait_parity_bounded(&l1full[st], par, kErrWaitQuantDown) ||
-          !wait_parity_bounded(&xfull[st], par, kErrWaitQuantDown)) {
-        ok = false;
+    for (int c = 0; c < nch; ++c) {
+      const int st = c % NS;
+      const uint32_t par = (c / NS) & 1;
+      if (*abort_flag || !wait_parity_bounded(&full[st], par, kErrWaitQuantDown) ||
+          !wait_parity_bounded(&xready[st], par, kErrWaitQuantDown)) {
+        *abort_flag = 1;
         break;
       }
       tc_fence_after();
       const uint64_t ad = smem_desc(smem_u32(xs + st * kXsBytes), 16, 1024, kLayoutSw128);
-      const uint64_t bd = smem_desc(smem_u32(l1s + st * align_up(l1_stage_bytes, 1024)), 16, 1024, kLayoutSw128);
+      const uint64_t bd = smem_desc(smem_u32(l1s + st * l1_stride), 16, 1024, kLayoutSw128);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        mma_bf16(tmem_base, ad + 2 * ks, bd + 2 * ks, idesc, (c | ks) != 0 ? 1u : 0u);
+      for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem_base, ad + 2 * ks, bd + 2 * ks, idesc, (c | ks) != 0 ? 1u : 0u);
       tc_commit(&empty[st]);
     }
     tc_commit(done);
-    if (!ok) {
-      *abort_flag = 1;
-      // Let every issued L1 copy land before the CTA can retire.
-      for (int q = 0; q < pcount; ++q)
-        wait_parity_bounded(&l1full[q % kQdStages], (q / kQdStages) & 1, kErrWaitQuantDown);
-    }
   }
 
   // ---------------------------------------------------------------- T epilogue
   __syncthreads();
   const bool aborted = *abort_flag != 0;
-  float* part = reinterpret_cast<float*>(xs);  // 128 x r fp32 partial (reuses the x_hat stages)
+  float* part = reinterpret_cast<float*>(xs);  // 128 x r fp32 partial (reuses the X stages)
   if (has_lr && warp < 4) {
     bool ok = !aborted && wait_parity_bounded(done, 0, kErrWaitQuantDown);
     ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-collective
@@ -322,44 +422,119 @@ __global__ void __launch_bounds__(kQdThreads, 1) quant_down_kernel(const QdParam
   }
   tc_fence_before();
   __syncthreads();
-  if (has_lr && warp == kQdWorkerWarps) {
+  if (has_lr && warp == kQdMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
   }
 }
 
-int quant_down_splits(int M, int K, int num_sms) {
+// Largest number of co-resident clusters of `splits` CTAs for one launch configuration; the query
+// runs once per (kernel, splits, shared-memory size) and is cached.
+static int max_active_clusters(void (*kern)(const CUtensorMap, const QdParams), int splits, size_t smem) {
+  struct Entry { const void* k; int s; size_t smem; int n; };
+  static Entry cache[64];
+  static int used = 0;
+  for (int i = 0; i < used; ++i)
+    if (cache[i].k == reinterpret_cast<const void*>(kern) && cache[i].s == splits && cache[i].smem == smem)
+      return cache[i].n;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(splits));
+  cfg.blockDim = dim3(kQdThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 1;
+  }
+  if (used < 64) cache[used++] = Entry{reinterpret_cast<const void*>(kern), splits, smem, n};
+  return n;
+}
+
+// The K slices of one 128-row tile form one cluster (<= 8 CTAs).  The split count minimises
+// (waves of co-resident clusters) x (k-blocks per CTA): a second partial wave would double the
+// time, so the grid is kept to what fits on the GPU at once.
+static int choose_splits(void (*kern)(const CUtensorMap, const QdParams), int M, int K, size_t smem) {
   const int mt = (M + kBM - 1) / kBM;
   const int KB = K / kBK;
-  int s = 1;
-  // Enough CTAs to keep every SM streaming; the K slices of a tile form one cluster (<= 8).
-  while (s < 8 && s * 2 <= KB && mt * s < num_sms) s *= 2;
-  return s;
+  int best = 1;
+  long best_cost = -1;
+  for (int s = 1; s <= 8 && s <= KB; ++s) {
+    const int active = max_active_clusters(kern, s, smem);
+    const long waves = (mt + active - 1) / active;
+    const long cost = waves * ((KB + s - 1) / s);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+static int quant_down_stages(int r) {
+  const size_t per = kXsBytes + align_up(static_cast<size_t>(r) * 128, 1024);
+  const int ns = static_cast<int>((kQdSmemBudget - 2048) / per);
+  return ns < kQdMaxStages ? ns : kQdMaxStages;
 }
 
 static size_t quant_down_smem_bytes(int r) {
-  return 1024 + kQdStages * kXsBytes + kQdStages * align_up(static_cast<size_t>(r) * 128, 1024) + 256;
+  const int ns = quant_down_stages(r);
+  return 1024 + ns * (kXsBytes + align_up(static_cast<size_t>(r) * 128, 1024)) + 256;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link dependency).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
 }
 
 cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t stream) {
   QdParams p;
-  p.X = a.X;
   p.M = a.M;
   p.K = a.K;
-  p.ldx = a.ldx;
   p.rank = a.rank;
   p.KB = a.K / kBK;
-  p.splits = quant_down_splits(a.M, a.K, num_sms);
+  p.stages = quant_down_stages(a.rank);
   p.inv_lambda = a.inv_lambda;
   p.l1 = a.l1;
   p.codes = a.codes;
   p.sf = a.sf;
   p.t = a.t;
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tmap;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.ldx) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBM)};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.X), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   const int mt = (a.M + kBM - 1) / kBM;
   const size_t smem = quant_down_smem_bytes(a.rank);
-  void (*kern)(const QdParams) = a.precision == 0 ? quant_down_kernel<0> : quant_down_kernel<1>;
+  void (*kern)(const CUtensorMap, const QdParams) = a.precision == 0 ? quant_down_kernel<0> : quant_down_kernel<1>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  (void)num_sms;
+  p.splits = choose_splits(kern, a.M, a.K, smem);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(mt * p.splits));
   cfg.blockDim = dim3(kQdThreads);
@@ -372,7 +547,7 @@ cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  return cudaLaunchKernelEx(&cfg, kern, tmap, p);
 }
 
 // ============================================================================ kernel 2

@@ -34,7 +34,4 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream);
 cudaError_t launch_selftest_wait(int spin_limit, cudaStream_t stream);
 cudaError_t read_and_clear_device_error(unsigned int* value, cudaStream_t stream);
 
-// Split-K factor (cluster size) kernel 1 uses for a given shape.
-int quant_down_splits(int M, int K, int num_sms);
-
 }  // namespace svdq

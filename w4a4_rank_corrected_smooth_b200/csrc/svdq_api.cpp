@@ -303,6 +303,56 @@ svdq_status svdq_free_weights(svdq_weights* w) {
   return SVDQ_OK;
 }
 
+svdq_status svdq_clone_weights(const svdq_weights* src, void* stream, svdq_weights** out) {
+  if (!src || !out) return fail(SVDQ_ERR_INVALID_ARG, "NULL argument");
+  *out = nullptr;
+  DeviceGuard guard(src->device);
+  if (!guard.ok) return fail(SVDQ_ERR_CUDA, "cudaSetDevice(%d) failed", src->device);
+  svdq_weights* w = new (std::nothrow) svdq_weights();
+  if (!w) return fail(SVDQ_ERR_OOM, "host allocation of the handle failed");
+  try {
+    w->canon = src->canon;
+  } catch (const std::bad_alloc&) {
+    delete w;
+    return fail(SVDQ_ERR_OOM, "host allocation failed while cloning");
+  }
+  w->N = src->N;
+  w->K = src->K;
+  w->rank = src->rank;
+  w->precision = src->precision;
+  w->device = src->device;
+  w->num_sms = src->num_sms;
+  const size_t npad = static_cast<size_t>((src->N + svdq::kBN - 1) / svdq::kBN) * svdq::kBN;
+  const size_t K = static_cast<size_t>(src->K), r = static_cast<size_t>(src->rank);
+  struct Buf { void** dst; const void* src; size_t bytes; };
+  const Buf bufs[] = {
+      {reinterpret_cast<void**>(&w->d_inv_lambda), src->d_inv_lambda, K * sizeof(float)},
+      {reinterpret_cast<void**>(&w->d_codes), src->d_codes, npad * K / 2},
+      {reinterpret_cast<void**>(&w->d_sf), src->d_sf, npad * K / svdq::kBK * svdq::kSfBytesPerRowKb},
+      {reinterpret_cast<void**>(&w->d_l1), src->d_l1, K * r * 2},
+      {reinterpret_cast<void**>(&w->d_l2), src->d_l2, npad * r * 2},
+      {reinterpret_cast<void**>(&w->d_bias), src->d_bias, npad * sizeof(float)},
+  };
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (const Buf& b : bufs) {
+    cudaError_t e = cudaMalloc(b.dst, b.bytes > 0 ? b.bytes : 16);
+    if (e == cudaSuccess && b.bytes > 0) e = cudaMemcpyAsync(*b.dst, b.src, b.bytes, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) {
+      free_device(w);
+      delete w;
+      return cuda_fail(e, "cloning prepared weights");
+    }
+  }
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) {
+    free_device(w);
+    delete w;
+    return cuda_fail(e, "cloning prepared weights");
+  }
+  *out = w;
+  return SVDQ_OK;
+}
+
 svdq_status svdq_get_weights_info(const svdq_weights* w, svdq_weights_info* info) {
   if (!w || !info) return fail(SVDQ_ERR_INVALID_ARG, "NULL argument");
   info->N = w->N;
