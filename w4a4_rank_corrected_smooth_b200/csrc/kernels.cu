@@ -461,7 +461,7 @@ static int max_active_clusters(void (*kern)(const CUtensorMap, const QdParams), 
 // (waves of co-resident clusters) x (k-blocks per CTA): a second partial wave would double the
 // time, so the grid is kept to what fits on the GPU at once.
 static int choose_splits(void (*kern)(const CUtensorMap, const QdParams), int M, int K, size_t smem) {
-  const int mt = (M + kBM - 1) / kBM;
+  const int mt = 2 * ((M + 2 * kBM - 1) / (2 * kBM));
   const int KB = K / kBK;
   int best = 1;
   long best_cost = -1;
@@ -528,7 +528,7 @@ cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t 
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  const int mt = (a.M + kBM - 1) / kBM;
+  const int mt = 2 * ((a.M + 2 * kBM - 1) / (2 * kBM));  // pairs of 128-row tiles (kernel 2 works on 256 rows)
   const size_t smem = quant_down_smem_bytes(a.rank);
   void (*kern)(const CUtensorMap, const QdParams) = a.precision == 0 ? quant_down_kernel<0> : quant_down_kernel<1>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -550,45 +550,134 @@ cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t 
   return cudaLaunchKernelEx(&cfg, kern, tmap, p);
 }
 
+
+// A byte buffer seen as a 2-D tensor of 256-byte rows, copied in boxes of `box_rows` rows (the
+// operands are stored as shared-memory images, so a box is a contiguous chunk of the buffer).
+static cudaError_t make_rows_map(CUtensorMap* map, const void* base, uint64_t bytes, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {256, bytes / 256};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {256, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  return cudaSuccess;
+}
+
 // ============================================================================ kernel 2
+//
+// A cluster of two CTAs computes 256 x 256 output tiles with cta_group::2 MMAs: each CTA holds its
+// own 128 rows of A, half (128 rows) of B and the scale factors its half of the accumulator needs
+// (its SFA, all 256 rows of SFB); each CTA's TMEM accumulates its 128 rows x 256 columns.  Each
+// CTA copies its operands into its own shared memory and signals its own barrier; a lane of the
+// peer CTA relays the peer's stage completions to the leader, which alone issues the tensor-core
+// work and then commits to the empty/accumulator barriers of both CTAs by cluster address.
 
 constexpr int kGStages = 4;
 constexpr int kGEpiWarps = 8;
 constexpr int kGThreads = (2 + kGEpiWarps) * 32;
-constexpr uint32_t kGA = kBM * kRowBytes;                     // 16 KB
-constexpr uint32_t kGB = kBN * kRowBytes;                     // 32 KB
-constexpr uint32_t kGSfa = kBM * kSfBytesPerRowKb;            // 2 KB
-constexpr uint32_t kGSfb = kBN * kSfBytesPerRowKb;            // 4 KB
-constexpr uint32_t kGStage = kGA + kGB + kGSfa + kGSfb;       // 54 KB
+constexpr uint32_t kGA = kBM * kRowBytes;                   // 16 KB: own 128 rows of A
+constexpr uint32_t kGB = (kBN / 2) * kRowBytes;             // 16 KB: own half of B
+constexpr uint32_t kGSfa = kBM * kSfBytesPerRowKb;          // 2 KB
+constexpr uint32_t kGSfb = kBN * kSfBytesPerRowKb;          // 4 KB: all 256 rows of B's scales
+constexpr uint32_t kGStage = kGA + kGB + kGSfa + kGSfb;     // 38 KB
+constexpr uint32_t kGStagePitch = kBN * 2 + 16;             // bf16 output row + 16 B: conflict-free rows
+constexpr uint32_t kGStaging = kBM * kGStagePitch;          // 66 KB: bf16 output tile of this CTA
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemSfa = 256, kTmemSfb = 272;
 
 struct GemmParams {
-  int M, N, K, rank, KB, MT, NT, ldy;
-  const uint8_t* a_codes;
-  const uint8_t* a_sf;
-  const uint8_t* t;
-  const uint8_t* b_codes;
-  const uint8_t* b_sf;
-  const uint8_t* l2;
+  int M, N, K, rank, KB, MT2, NT, ldy;
   const float* bias;
   uint16_t* Y;
 };
 
-__global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const GemmParams p) {
-  extern __shared__ uint8_t smem_raw[];
+// Box heights (256-byte rows) of the operand maps.
+constexpr uint32_t kBoxA = kGA / 256, kBoxB = kGB / 256, kBoxSfa = kGSfa / 256, kBoxSfb = kGSfb / 256, kBoxLr = 16;
+
+struct alignas(64) GemmMaps {
+  CUtensorMap a, b, sfa, sfb, t, l2;
+};
+
+__device__ __forceinline__ void tmem_alloc2(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Arrive on the barrier at cluster address `bar` once all prior tcgen05 ops of this thread complete.
+__device__ __forceinline__ void tc_commit2(uint32_t bar_cluster_addr) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ void mma2_bf16(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(ad), "l"(bd), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma2_nvfp4(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t sfa,
+                                           uint32_t sfb, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d),
+      "l"(ad), "l"(bd), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_cp2_32x128(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// 2-D tensor copy of this CTA's box into its own shared memory; completion is counted on the
+// barrier at cluster address `bar` (the leader CTA's barrier for both CTAs of the pair).
+__device__ __forceinline__ void tma_rows_cg2(void* smem_dst, const CUtensorMap* map, int row, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
+__device__ __forceinline__ void bulk_s2g(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_constant__ GemmMaps maps,
+                                                                    const GemmParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGStages * kGStage);
-  uint64_t* empty = full + kGStages;
-  uint64_t* acc_full = empty + kGStages;
-  uint64_t* acc_empty = acc_full + 1;
+  uint8_t* staging = smem + kGStages * kGStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + kGStaging);  // (leader) both CTAs' copies landed
+  uint64_t* empty = full + kGStages;        // (both) MMAs done with the stage
+  uint64_t* acc_full = empty + kGStages;    // (both) accumulator ready
+  uint64_t* acc_empty = acc_full + 1;       // (leader) both CTAs drained the accumulator
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int r = p.rank;
   const int nlr = (r + kLrChunk - 1) / kLrChunk;
-  const int tiles = p.MT * p.NT;
+  const int tiles = p.MT2 * p.NT;
+  const int nstages_tile = nlr + p.KB;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGStages; ++s) {
@@ -596,83 +685,81 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const GemmPara
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kGEpiWarps);
+    mbar_init(acc_empty, 2 * kGEpiWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc2(tmem_slot, kTmemCols);
+    tmem_relinquish2();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------------------ producer
+      // ------------------------------------------------------------ producer (both CTAs)
+      // Each CTA copies its own boxes; all copies complete on the leader's full barrier, which the
+      // leader arms with the bytes of both CTAs.
+      const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
       int st = 0;
       uint32_t ph = 0;
-      int issued_phase[kGStages];
-      for (int s = 0; s < kGStages; ++s) issued_phase[s] = -1;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-        const int mt = tile / p.NT, nt = tile % p.NT;
-        const int nstages = nlr + p.KB;
-        for (int j = 0; j < nstages; ++j) {
+      for (int tile = pair; tile < tiles && ok; tile += npairs) {
+        const int m2 = tile / p.NT, nt = tile % p.NT;
+        const int mt = 2 * m2 + static_cast<int>(rank);  // this CTA's 128-row tile
+        for (int j = 0; j < nstages_tile; ++j) {
           if (*abort_flag || !wait_parity_bounded(&empty[st], ph ^ 1u, kErrWaitGemm)) {
             ok = false;
             break;
           }
-          uint8_t* sbase = smem + st * kGStage;
+          uint8_t* sb = smem + st * kGStage;
+          const uint32_t bar = full_leader + 8u * st;
           if (j < nlr) {
             const uint32_t cw = lr_chunk_width(r, j);
-            const uint32_t tb = kBM * cw * 2, lb = kBN * cw * 2;
-            mbar_arrive_expect_tx(&full[st], tb + lb);
-            bulk_g2s(sbase, p.t + static_cast<size_t>(mt) * kBM * r * 2 + static_cast<size_t>(kBM) * kLrChunk * 2 * j, tb,
-                     &full[st]);
-            bulk_g2s(sbase + kGA, p.l2 + static_cast<size_t>(nt) * kBN * r * 2 + static_cast<size_t>(kBN) * kLrChunk * 2 * j,
-                     lb, &full[st]);
+            const uint32_t tb = kBM * cw * 2, lb = (kBN / 2) * cw * 2;  // per CTA
+            if (leader) mbar_arrive_expect_tx(&full[st], 2 * (tb + lb));
+            const int trow = static_cast<int>((static_cast<size_t>(mt) * kBM * r * 2 + static_cast<size_t>(kBM) * kLrChunk * 2 * j) / 256);
+            const int lrow = static_cast<int>((static_cast<size_t>(nt) * kBN * r * 2 + static_cast<size_t>(kBN) * kLrChunk * 2 * j + rank * lb) / 256);
+            for (uint32_t q = 0; q < tb / 4096; ++q) tma_rows_cg2(sb + 4096 * q, &maps.t, trow + 16 * q, bar);
+            for (uint32_t q = 0; q < lb / 4096; ++q) tma_rows_cg2(sb + kGA + 4096 * q, &maps.l2, lrow + 16 * q, bar);
           } else {
             const int kb = j - nlr;
-            mbar_arrive_expect_tx(&full[st], kGStage);
-            bulk_g2s(sbase, p.a_codes + codes_chunk_offset(mt, kb, p.KB, kBM), kGA, &full[st]);
-            bulk_g2s(sbase + kGA, p.b_codes + codes_chunk_offset(nt, kb, p.KB, kBN), kGB, &full[st]);
-            bulk_g2s(sbase + kGA + kGB, p.a_sf + sf_chunk_offset(mt, kb, p.KB, kBM), kGSfa, &full[st]);
-            bulk_g2s(sbase + kGA + kGB + kGSfa, p.b_sf + sf_chunk_offset(nt, kb, p.KB, kBN), kGSfb, &full[st]);
+            if (leader) mbar_arrive_expect_tx(&full[st], 2 * kGStage);
+            tma_rows_cg2(sb, &maps.a, static_cast<int>(codes_chunk_offset(mt, kb, p.KB, kBM) / 256), bar);
+            tma_rows_cg2(sb + kGA, &maps.b, static_cast<int>((codes_chunk_offset(nt, kb, p.KB, kBN) + rank * kGB) / 256), bar);
+            tma_rows_cg2(sb + kGA + kGB, &maps.sfa, static_cast<int>(sf_chunk_offset(mt, kb, p.KB, kBM) / 256), bar);
+            tma_rows_cg2(sb + kGA + kGB + kGSfa, &maps.sfb, static_cast<int>(sf_chunk_offset(nt, kb, p.KB, kBN) / 256), bar);
           }
-          issued_phase[st] = static_cast<int>(ph);
           if (++st == kGStages) {
             st = 0;
             ph ^= 1u;
           }
         }
       }
-      if (!ok) {
-        *abort_flag = 1;
-        for (int s = 0; s < kGStages; ++s)
-          if (issued_phase[s] >= 0) wait_parity_bounded(&full[s], static_cast<uint32_t>(issued_phase[s]), kErrWaitGemm);
-      }
+      if (!ok) *abort_flag = 1;
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
-      const uint32_t id_lr = idesc_bf16(128, 256);
-      const uint32_t id_fp4 = idesc_nvfp4(128, 256);
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (leader CTA)
+      const uint32_t id_lr = idesc_bf16(256, 256);
+      const uint32_t id_fp4 = idesc_nvfp4(256, 256);
+      const uint32_t empty_local = smem_u32(empty), empty_peer = mapa_shared(smem_u32(empty), 1);
+      const uint32_t accf_local = smem_u32(acc_full), accf_peer = mapa_shared(smem_u32(acc_full), 1);
       int st = 0;
       uint32_t ph = 0;
       bool ok = true;
       int local = 0;
-      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++local) {
+      for (int tile = pair; tile < tiles && ok; tile += npairs, ++local) {
         if (*abort_flag || !wait_parity_bounded(acc_empty, (static_cast<uint32_t>(local) & 1u) ^ 1u, kErrWaitGemm)) {
           ok = false;
           break;
         }
         tc_fence_after();
         uint32_t accum = 0;
-        const int nstages = nlr + p.KB;
-        for (int j = 0; j < nstages; ++j) {
+        for (int j = 0; j < nstages_tile; ++j) {
           if (*abort_flag || !wait_parity_bounded(&full[st], ph, kErrWaitGemm)) {
             ok = false;
             break;
@@ -684,53 +771,60 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const GemmPara
             const uint64_t ad = smem_desc(sb, 128, cw * 16, kLayoutNone);
             const uint64_t bd = smem_desc(sb + kGA, 128, cw * 16, kLayoutNone);
             for (uint32_t ks = 0; ks < cw / 16; ++ks) {
-              mma_bf16(tmem, ad + 16 * ks, bd + 16 * ks, id_lr, accum);
+              mma2_bf16(tmem, ad + 16 * ks, bd + 16 * ks, id_lr, accum);
               accum = 1;
             }
           } else {
             const uint32_t sfa = sb + kGA + kGB, sfb = sfa + kGSfa;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              tmem_cp_32x128_warpx4(tmem + kTmemSfa + 4 * kk, smem_desc(sfa + 512 * kk, 0, 128, kLayoutNone));
-              tmem_cp_32x128_warpx4(tmem + kTmemSfb + 8 * kk, smem_desc(sfb + 1024 * kk, 0, 128, kLayoutNone));
-              tmem_cp_32x128_warpx4(tmem + kTmemSfb + 8 * kk + 4, smem_desc(sfb + 1024 * kk + 512, 0, 128, kLayoutNone));
+              tmem_cp2_32x128(tmem + kTmemSfa + 4 * kk, smem_desc(sfa + 512 * kk, 0, 128, kLayoutNone));
+              tmem_cp2_32x128(tmem + kTmemSfb + 8 * kk, smem_desc(sfb + 1024 * kk, 0, 128, kLayoutNone));
+              tmem_cp2_32x128(tmem + kTmemSfb + 8 * kk + 4, smem_desc(sfb + 1024 * kk + 512, 0, 128, kLayoutNone));
             }
             const uint64_t ad = smem_desc(sb, 16, 1024, kLayoutSw128);
             const uint64_t bd = smem_desc(sb + kGA, 16, 1024, kLayoutSw128);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              mma_nvfp4(tmem, ad + 2 * kk, bd + 2 * kk, id_fp4, tmem + kTmemSfa + 4 * kk, tmem + kTmemSfb + 8 * kk,
-                        accum);
+              mma2_nvfp4(tmem, ad + 2 * kk, bd + 2 * kk, id_fp4, tmem + kTmemSfa + 4 * kk, tmem + kTmemSfb + 8 * kk,
+                         accum);
               accum = 1;
             }
           }
-          tc_commit(&empty[st]);
+          tc_commit2(empty_local + 8u * st);
+          tc_commit2(empty_peer + 8u * st);
           if (++st == kGStages) {
             st = 0;
             ph ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        tc_commit2(accf_local);
+        tc_commit2(accf_peer);
       }
       if (!ok) {
         *abort_flag = 1;
-        // Make sure no issued tcgen05 operation is still running when TMEM is released.
-        tc_commit(acc_full);
+        tc_commit2(accf_local);  // completes once every issued tcgen05 op has
+        tc_commit2(accf_peer);
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (8 warps)
+    // ------------------------------------------------------------ epilogue (8 warps per CTA)
     const int q = warp & 3, h = (warp - 2) >> 2;
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+    const int rloc = q * 32 + lane;                       // row inside this CTA's 128 rows
+    uint8_t* srow = staging + rloc * kGStagePitch + h * 256;  // this thread's 128 bf16 of the row
     int local = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++local) {
-      bool ok = !*abort_flag && wait_parity_bounded(acc_full, static_cast<uint32_t>(local) & 1u, kErrWaitGemm);
-      if (!__all_sync(0xffffffffu, ok)) {  // the TMEM loads below are warp-collective
+    for (int tile = pair; tile < tiles; tile += npairs, ++local) {
+      bool ok = true;
+      if (lane == 0) ok = !*abort_flag && wait_parity_bounded(acc_full, static_cast<uint32_t>(local) & 1u, kErrWaitGemm);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const int mt = tile / p.NT, nt = tile % p.NT;
+      const int m2 = tile / p.NT, nt = tile % p.NT;
       uint32_t v[4][32];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -738,48 +832,50 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const GemmPara
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-      const int row = mt * kBM + q * 32 + lane;
+      if (lane == 0) mbar_arrive_remote(acc_empty_leader);  // the accumulator may be overwritten now
+      const int row = (2 * m2 + static_cast<int>(rank)) * kBM + rloc;
       const int n0 = nt * kBN + h * 128;
-      if (row < p.M) {
-        uint16_t* yrow = p.Y + static_cast<size_t>(row) * p.ldy;
+      bulk_wait_read0();  // the previous tile's stores have finished reading the staging rows
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 4; ++i) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int n = n0 + i * 32 + g * 8;
-            if (n < p.N) {
-              const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n));
-              const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n + 4));
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(v[i][g * 8 + 0]) + b0.x, __uint_as_float(v[i][g * 8 + 1]) + b0.y);
-              o.y = pack_bf16x2(__uint_as_float(v[i][g * 8 + 2]) + b0.z, __uint_as_float(v[i][g * 8 + 3]) + b0.w);
-              o.z = pack_bf16x2(__uint_as_float(v[i][g * 8 + 4]) + b1.x, __uint_as_float(v[i][g * 8 + 5]) + b1.y);
-              o.w = pack_bf16x2(__uint_as_float(v[i][g * 8 + 6]) + b1.z, __uint_as_float(v[i][g * 8 + 7]) + b1.w);
-              *reinterpret_cast<uint4*>(yrow + n) = o;
-            }
-          }
+        for (int g = 0; g < 4; ++g) {
+          const int u = i * 4 + g;  // 16-byte unit of the row segment
+          const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8));
+          const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8 + 4));
+          uint4 o;
+          o.x = pack_bf16x2(__uint_as_float(v[i][g * 8 + 0]) + b0.x, __uint_as_float(v[i][g * 8 + 1]) + b0.y);
+          o.y = pack_bf16x2(__uint_as_float(v[i][g * 8 + 2]) + b0.z, __uint_as_float(v[i][g * 8 + 3]) + b0.w);
+          o.z = pack_bf16x2(__uint_as_float(v[i][g * 8 + 4]) + b1.x, __uint_as_float(v[i][g * 8 + 5]) + b1.y);
+          o.w = pack_bf16x2(__uint_as_float(v[i][g * 8 + 6]) + b1.z, __uint_as_float(v[i][g * 8 + 7]) + b1.w);
+          *reinterpret_cast<uint4*>(srow + 16 * u) = o;  // row pitch 528 B: 8 lanes, 8 bank groups
         }
       }
+      fence_proxy_async_smem();
+      if (row < p.M && n0 < p.N) {
+        const int ncols = (p.N - n0) < 128 ? (p.N - n0) : 128;
+        bulk_s2g(p.Y + static_cast<size_t>(row) * p.ldy + n0, smem_u32(srow), static_cast<uint32_t>(ncols) * 2u);
+      }
+      bulk_commit();
     }
+    bulk_wait0();
   }
 
-  // The MMA issuer's last commit (normal or abort) tells when no tcgen05 op is in flight.
   __syncthreads();
-  if (warp == 1) {
-    if (*abort_flag && lane == 0) {
-      // acc_full received one extra commit in the abort path; wait for all of them to land.
-      const unsigned long long t0 = globaltimer_ns();
-      while (globaltimer_ns() - t0 < 2000000ull) {
-      }
+  if (warp == 1 && leader && *abort_flag && lane == 0) {
+    const unsigned long long t0 = globaltimer_ns();  // the abort-path commits land within microseconds
+    while (globaltimer_ns() - t0 < 2000000ull) {
     }
-    __syncwarp();
+  }
+  tc_fence_before();
+  cluster_sync();  // neither CTA releases TMEM or exits while its peer may still address it
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc2(tmem, kTmemCols);
   }
 }
 
-static size_t gemm_smem_bytes() { return 1024 + kGStages * kGStage + 256; }
+static size_t gemm_smem_bytes() { return 1024 + kGStages * kGStage + kGStaging + 256; }
 
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   GemmParams p;
@@ -788,26 +884,43 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   p.K = a.K;
   p.rank = a.rank;
   p.KB = a.K / kBK;
-  p.MT = (a.M + kBM - 1) / kBM;
+  p.MT2 = (a.M + 2 * kBM - 1) / (2 * kBM);
   p.NT = (a.N + kBN - 1) / kBN;
   p.ldy = a.ldy;
-  p.a_codes = a.a_codes;
-  p.a_sf = a.a_sf;
-  p.t = a.t;
-  p.b_codes = a.b_codes;
-  p.b_sf = a.b_sf;
-  p.l2 = a.l2;
   p.bias = a.bias;
   p.Y = a.Y;
   if (a.precision != 0) return cudaErrorNotSupported;
+  const size_t mt = static_cast<size_t>(p.MT2) * 2, nt = static_cast<size_t>(p.NT), KB = static_cast<size_t>(p.KB);
+  const size_t rr = static_cast<size_t>(a.rank);
+  GemmMaps maps;
+  cudaError_t me;
+  if ((me = make_rows_map(&maps.a, a.a_codes, mt * KB * kGA, kBoxA)) != cudaSuccess ||
+      (me = make_rows_map(&maps.b, a.b_codes, nt * KB * kBN * kRowBytes, kBoxB)) != cudaSuccess ||
+      (me = make_rows_map(&maps.sfa, a.a_sf, mt * KB * kGSfa, kBoxSfa)) != cudaSuccess ||
+      (me = make_rows_map(&maps.sfb, a.b_sf, nt * KB * kGSfb, kBoxSfb)) != cudaSuccess ||
+      (me = make_rows_map(&maps.t, a.t, rr ? mt * kBM * rr * 2 : 4096, kBoxLr)) != cudaSuccess ||
+      (me = make_rows_map(&maps.l2, a.l2, rr ? nt * kBN * rr * 2 : 4096, kBoxLr)) != cudaSuccess)
+    return me;
   const size_t smem = gemm_smem_bytes();
   cudaError_t e =
       cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int tiles = p.MT * p.NT;
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  gemm_nvfp4_kernel<<<grid, kGThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  const int tiles = p.MT2 * p.NT;
+  int pairs = num_sms / 2;
+  if (pairs > tiles) pairs = tiles;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(kGThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, maps, p);
 }
 
 // ============================================================================ failure detection

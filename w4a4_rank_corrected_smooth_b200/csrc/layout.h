@@ -79,7 +79,7 @@ struct WorkspaceLayout {
 
 inline WorkspaceLayout workspace_layout(int M, int K, int r) {
   WorkspaceLayout w;
-  w.m_tiles = (M + kBM - 1) / kBM;
+  w.m_tiles = 2 * ((M + 2 * kBM - 1) / (2 * kBM));  // kernel 2 consumes rows in pairs of 128-row tiles
   const size_t mpad = static_cast<size_t>(w.m_tiles) * kBM;
   w.codes = 0;
   size_t end = mpad * static_cast<size_t>(K) / 2;
