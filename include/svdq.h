@@ -147,6 +147,23 @@ svdq_status svdq_workspace_size(const svdq_weights* w, int M, size_t* bytes);
 svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* The forward without a caller workspace and without any device allocation.  The pages have no
+ * counterpart to this call: it exists for callers that cannot allocate device memory while they
+ * run, for instance code inside a host framework that owns all device memory and hands its
+ * plugins no allocator, or a latency-critical path where cudaMalloc (which may synchronise the
+ * device) is not acceptable.  The scratch between the two kernels is a fixed 16 MiB array in the
+ * library's own device module, which every GPU that loads the library keeps until the process
+ * exits.  The first call on a device looks up that array's device address (cudaGetSymbolAddress,
+ * with the device current) and caches it; make that first call before any stream capture.
+ * All calls on a device share the one array and it keeps the contents of the last call: calls
+ * whose kernels overlap on the GPU (different streams, no ordering between them) race and give
+ * wrong results, so order them on one stream or use svdq_linear_forward with separate
+ * workspaces.  Nothing in the array has to start at zero.  Shapes whose workspace
+ * (svdq_workspace_size) exceeds 16 MiB are rejected with SVDQ_ERR_INVALID_ARG; at K = 3072 and
+ * rank 32 that allows M up to 9216.  Other arguments and errors as svdq_linear_forward. */
+svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
+                                        void* stream);
+
 /* Kernel 1 alone (same arguments as the forward minus Y): fills the workspace. */
 svdq_status svdq_quant_down(const svdq_weights* w, const void* X, int M, int ldx, void* workspace,
                             size_t workspace_bytes, void* stream);

@@ -58,6 +58,7 @@ def _load() -> ctypes.CDLL:
         "svdq_export_weights": ([vp, vp, vp, vp, vp, vp, vp, vp], i),
         "svdq_workspace_size": ([vp, i, ctypes.POINTER(sz)], i),
         "svdq_linear_forward": ([vp, vp, i, i, vp, i, vp, sz, vp], i),
+        "svdq_linear_forward_noalloc": ([vp, vp, i, i, vp, i, vp], i),
         "svdq_quant_down": ([vp, vp, i, i, vp, sz, vp], i),
         "svdq_gemm_up": ([vp, i, vp, i, vp, sz, vp], i),
         "svdq_export_activations": ([vp, vp, sz, i, vp, vp, vp, vp], i),
@@ -75,7 +76,7 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 DECLARED_SYMBOLS = tuple(sorted([
     "svdq_status_string", "svdq_last_error", "svdq_check_device", "svdq_get_device_error", "svdq_prepare_weights",
-    "svdq_free_weights", "svdq_clone_weights", "svdq_get_weights_info", "svdq_export_weights", "svdq_workspace_size", "svdq_linear_forward",
+    "svdq_free_weights", "svdq_clone_weights", "svdq_get_weights_info", "svdq_export_weights", "svdq_workspace_size", "svdq_linear_forward", "svdq_linear_forward_noalloc",
     "svdq_quant_down", "svdq_gemm_up", "svdq_export_activations", "svdq_quantize_rows_host", "svdq_prepare_host",
     "svdq_selftest_wait_timeout"]))
 
@@ -237,6 +238,11 @@ class SVDQLinear:
     def svdq_linear_forward(self, X, M: int, ldx: int, Y, ldy: int, workspace, workspace_bytes: int, stream=None):
         _check(_lib.svdq_linear_forward(self._h, _ptr(X), M, ldx, _ptr(Y), ldy, _ptr(workspace), workspace_bytes,
                                         _stream(stream)))
+
+    def svdq_linear_forward_noalloc(self, X, M: int, ldx: int, Y, ldy: int, stream=None):
+        """The forward using the library's fixed device scratch instead of a caller workspace
+        (for callers that cannot allocate device memory; see include/svdq.h)."""
+        _check(_lib.svdq_linear_forward_noalloc(self._h, _ptr(X), M, ldx, _ptr(Y), ldy, _stream(stream)))
 
     def svdq_quant_down(self, X, M: int, ldx: int, workspace, workspace_bytes: int, stream=None):
         _check(_lib.svdq_quant_down(self._h, _ptr(X), M, ldx, _ptr(workspace), workspace_bytes, _stream(stream)))

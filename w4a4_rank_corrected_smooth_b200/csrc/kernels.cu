@@ -17,6 +17,7 @@
 // accumulator in tensor memory; eight epilogue warps drain the accumulator, add the bias and
 // write bf16 Y once.
 #include <cuda.h>
+#include <mutex>
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -921,6 +922,37 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, maps, p);
+}
+
+// ============================================================================ fixed scratch
+
+// Scratch of svdq_linear_forward_noalloc: a fixed array in the module's global memory, so that
+// the forward can run without any device allocation.  Every device that loads the library holds
+// it until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// Device address of the fixed scratch on the current device.  The host-side name of the array is
+// only a stand-in, so the address is looked up once per device (with that device current) and
+// cached.
+cudaError_t noalloc_scratch_address(void** ptr) {
+  static std::mutex mu;
+  static void* addr[128] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return cudaSuccess;
 }
 
 // ============================================================================ failure detection

@@ -34,4 +34,8 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream);
 cudaError_t launch_selftest_wait(int spin_limit, cudaStream_t stream);
 cudaError_t read_and_clear_device_error(unsigned int* value, cudaStream_t stream);
 
+// Fixed-size scratch in the library's device module (for the allocation-free forward).
+size_t noalloc_scratch_bytes();
+cudaError_t noalloc_scratch_address(void** ptr);
+
 }  // namespace svdq

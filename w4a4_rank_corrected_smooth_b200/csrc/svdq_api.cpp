@@ -389,6 +389,26 @@ svdq_status svdq_workspace_size(const svdq_weights* w, int M, size_t* bytes) {
   return SVDQ_OK;
 }
 
+svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
+                                        void* stream) {
+  if (!w) return fail(SVDQ_ERR_INVALID_ARG, "weights handle is NULL");
+  if (M < 0) return fail(SVDQ_ERR_INVALID_ARG, "M=%d is negative", M);
+  if (M == 0) return SVDQ_OK;
+  const size_t need = svdq::workspace_layout(M, w->K, w->rank).total;
+  const size_t have = svdq::noalloc_scratch_bytes();
+  if (need > have)
+    return fail(SVDQ_ERR_INVALID_ARG,
+                "svdq_linear_forward_noalloc: M=%d (K=%d, rank=%d) needs %zu bytes of scratch, more than the %zu bytes "
+                "of the library's fixed scratch; use svdq_linear_forward with a caller workspace",
+                M, w->K, w->rank, need, have);
+  DeviceGuard guard(w->device);
+  if (!guard.ok) return fail(SVDQ_ERR_CUDA, "cudaSetDevice(%d) failed", w->device);
+  void* scratch = nullptr;
+  cudaError_t e = svdq::noalloc_scratch_address(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "looking up the fixed scratch (cudaGetSymbolAddress)");
+  return svdq_linear_forward(w, X, M, ldx, Y, ldy, scratch, have, stream);
+}
+
 svdq_status svdq_quant_down(const svdq_weights* w, const void* X, int M, int ldx, void* workspace,
                             size_t workspace_bytes, void* stream) {
   svdq_status s = check_forward_common(w, M, workspace, workspace_bytes);
