@@ -175,6 +175,13 @@ def max_over_ranks(value: float, world: int) -> float:
     return float(t.item())
 
 
+def weak_scaling_value(flops_per_step: float, steps: int, local_ms: float, world: int):
+    """Whole-job throughput (TFLOP/s) of `world` replicas that each ran `steps` steps: the work of
+    all ranks over the slowest rank's time.  Returns (value, slowest_ms)."""
+    slowest = max_over_ranks(local_ms, world)
+    return world * flops_per_step * steps / (slowest / 1e3) / 1e12, slowest
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -360,10 +367,8 @@ def run_ours(args):
     barrier(world)
     clocks = sampler.stop() if not args.no_clocks else None
     S.svdq_get_device_error(stream)
-    total_ms = max_over_ranks(total_ms, world)
-
     flops = spec.flops
-    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    value, total_ms = weak_scaling_value(flops, args.steps, total_ms, world)
     k2_flops = spec.flops_4bit + 2 * spec.M * spec.rank * spec.N
     k2_tflops = k2_flops / (k2_ms / 1e3) / 1e12
     fp4_peak_sustained = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
