@@ -154,7 +154,7 @@ def test_quant_down_codec_boundaries_bitexact(prec):
     check_activations(lin, X, prec, ops)
 
 
-@pytest.mark.parametrize("prec", ["nvfp4"])
+@pytest.mark.parametrize("prec", ["nvfp4", "int4"])
 def test_forward_tiny(prec):
     spec = synth.get("tiny_256x512x512_r16")
     X, W, b, lin = make_layer(spec, prec)
@@ -164,17 +164,18 @@ def test_forward_tiny(prec):
     check_y(Y, ref)
 
 
+@pytest.mark.parametrize("prec", ["nvfp4", "int4"])
 @pytest.mark.parametrize("M,K,N,r", [(1, 256, 256, 16), (17, 512, 264, 0), (255, 768, 512, 48), (129, 256, 512, 128),
                                      (300, 1024, 768, 64), (128, 512, 1024, 32)])
-def test_forward_edge_shapes(M, K, N, r):
+def test_forward_edge_shapes(M, K, N, r, prec):
     spec = synth.custom(f"edge_{M}_{K}_{N}_{r}", M=M, K=K, N=N, rank=r, seed=M + K + N + r)
-    X, W, b, lin = make_layer(spec, "nvfp4")
+    X, W, b, lin = make_layer(spec, prec)
     ops = lin.export_weights()
-    check_activations(lin, X, "nvfp4", ops)
+    check_activations(lin, X, prec, ops)
     Yd = run_forward(lin, X, ldy_pad=8)
     assert torch.isnan(Yd[:, N:].float()).all()  # nothing written past column N
     Y = y_to_f64(Yd[:, :N].contiguous())
-    check_y(Y, O.linear(X, ops, "nvfp4")["Y"])
+    check_y(Y, O.linear(X, ops, prec)["Y"])
 
 
 def test_forward_m_zero_is_noop():
@@ -191,18 +192,19 @@ def test_forward_deterministic():
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
 
-def test_forward_flux_qkv_full_size_sampled_rows():
-    """4608 x 3072 -> 9216, rank 32, NVFP4, in the launch configuration the benchmark times:
+@pytest.mark.parametrize("prec", ["nvfp4", "int4"])
+def test_forward_flux_qkv_full_size_sampled_rows(prec):
+    """4608 x 3072 -> 9216, rank 32, in the launch configuration the benchmark times:
     all codes and scales bit-exact; Y checked on a seeded sample of 192 full rows."""
     spec = synth.get("flux_qkv_4608x3072x9216_r32")
-    X, W, b, lin = make_layer(spec, "nvfp4")
+    X, W, b, lin = make_layer(spec, prec)
     ops = lin.export_weights()
-    act = check_activations(lin, X, "nvfp4", ops)
+    act = check_activations(lin, X, prec, ops)
     Yd = run_forward(lin, X)
     rows = np.sort(np.random.default_rng(5).choice(spec.M, 192, replace=False))
     Y = y_to_f64(Yd[torch.from_numpy(rows).cuda()])
-    xh, cx, sx = O.quantize_activations(X[rows], ops["inv_lambda"], "nvfp4")
+    xh, cx, sx = O.quantize_activations(X[rows], ops["inv_lambda"], prec)
     T = O.lowrank_down(xh, ops["L1"])
-    ref = O.forward(cx, sx, T, ops["codes_w"], ops["scales_w"], ops["L2"], ops["bias"], "nvfp4")
+    ref = O.forward(cx, sx, T, ops["codes_w"], ops["scales_w"], ops["L2"], ops["bias"], prec)
     check_y(Y, ref)
     assert act["codes_x"].shape == (spec.M, spec.K // 2)

@@ -137,8 +137,6 @@ svdq_status do_gemm(const svdq_weights* w, int M, void* Y, int ldy, const void* 
   if (!Y) return fail(SVDQ_ERR_INVALID_ARG, "Y is NULL");
   if (ldy < w->N || ldy % 8 != 0) return fail(SVDQ_ERR_INVALID_ARG, "ldy=%d must be >= N=%d and a multiple of 8", ldy, w->N);
   if (!aligned(Y, 16)) return fail(SVDQ_ERR_INVALID_ARG, "Y must be 16-byte aligned");
-  if (w->precision != SVDQ_NVFP4)
-    return fail(SVDQ_ERR_INVALID_ARG, "the INT4 4-bit GEMM kernel is not available in this build");
   const svdq::WorkspaceLayout L = svdq::workspace_layout(M, w->K, w->rank);
   const uint8_t* base = static_cast<const uint8_t*>(ws);
   svdq::GemmArgs a;
@@ -432,8 +430,6 @@ svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int
   if (!Y) return fail(SVDQ_ERR_INVALID_ARG, "Y is NULL");
   if (ldy < w->N || ldy % 8 != 0 || !aligned(Y, 16))
     return fail(SVDQ_ERR_INVALID_ARG, "Y must be 16-byte aligned with ldy >= N and a multiple of 8");
-  if (w->precision != SVDQ_NVFP4)
-    return fail(SVDQ_ERR_INVALID_ARG, "the INT4 4-bit GEMM kernel is not available in this build");
   DeviceGuard guard(w->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   s = do_quant_down(w, X, M, ldx, workspace, st);
