@@ -571,36 +571,51 @@ static cudaError_t make_rows_map(CUtensorMap* map, const void* base, uint64_t by
 // ============================================================================ kernel 2
 //
 // A cluster of two CTAs computes 256 x 256 output tiles with cta_group::2 MMAs: each CTA holds its
-// own 128 rows of A, half (128 rows) of B and the scale factors its half of the accumulator needs
-// (its SFA, all 256 rows of SFB); each CTA's TMEM accumulates its 128 rows x 256 columns.  Each
-// CTA copies its operands into its own shared memory and signals its own barrier; a lane of the
-// peer CTA relays the peer's stage completions to the leader, which alone issues the tensor-core
-// work and then commits to the empty/accumulator barriers of both CTAs by cluster address.
+// own 128 rows of A and half (128 rows) of B in shared memory, the scale factors its half of the
+// accumulator needs (its SFA, all 256 rows of SFB) in TMEM, and accumulates its 128 rows x 256
+// columns in TMEM.  The leader CTA alone issues the MMAs.
+//
+// Every per-stage chain is kept short because each runs on one thread (or warp) whose
+// synchronisation and issue instructions have long latencies:
+//   producer (1 thread per CTA): wait empty[s]; A, B and scale tiles of this CTA by TMA onto its
+//     full[s];
+//   scale warps (4 per CTA, one per TMEM lane quadrant): wait full[s], copy the stage's scale
+//     bytes from shared memory into the stage's TMEM scale buffer with tcgen05.st (instead of
+//     tcgen05.cp in the MMA issuer's instruction stream), then arrive on the leader's ready[s] --
+//     which thereby also tells the leader that this CTA's operand tiles have landed;
+//   MMA issuer (leader, 1 thread): wait ready[s] (8 arrivals: both CTAs' scale warps); 4 MMAs;
+//     one commit multicast to empty[s] of both CTAs;
+//   epilogue (8 warps per CTA): drain the accumulator, add the bias, round to bf16 into a 128-byte
+//     swizzled staging tile and write it with two TMA tensor stores per warp.
 
 constexpr int kGStages = 4;
+constexpr int kGSfWarps = 4;
 constexpr int kGEpiWarps = 8;
-constexpr int kGThreads = (2 + kGEpiWarps) * 32;
+constexpr int kGFirstEpiWarp = 2 + kGSfWarps;
+constexpr int kGThreads = (2 + kGSfWarps + kGEpiWarps) * 32;
 constexpr uint32_t kGA = kBM * kRowBytes;                   // 16 KB: own 128 rows of A
 constexpr uint32_t kGB = (kBN / 2) * kRowBytes;             // 16 KB: own half of B
-constexpr uint32_t kGSfa = kBM * kSfBytesPerRowKb;          // 2 KB
-constexpr uint32_t kGSfb = kBN * kSfBytesPerRowKb;          // 4 KB: all 256 rows of B's scales
+constexpr uint32_t kGSfa = kBM * kSfBytesPerRowKb;          // 2 KB of A scales per (m-tile, k-block)
+constexpr uint32_t kGSfb = kBN * kSfBytesPerRowKb;          // 4 KB of B scales per (n-tile, k-block)
 constexpr uint32_t kGStage = kGA + kGB + kGSfa + kGSfb;     // 38 KB
-constexpr uint32_t kGStagePitch = kBN * 2 + 16;             // bf16 output row + 16 B: conflict-free rows
-constexpr uint32_t kGStaging = kBM * kGStagePitch;          // 66 KB: bf16 output tile of this CTA
+constexpr uint32_t kGOutBox = 32 * 128;                     // staging box: 32 rows x 64 bf16, 128-byte swizzle
+constexpr uint32_t kGStaging = kGEpiWarps * 2 * kGOutBox;   // 64 KB: two boxes per epilogue warp
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemSfa = 256, kTmemSfb = 272;
+// Per-stage scale buffer: 12 blocks of 4 columns (SFA k-steps 0..3, then SFB k-steps 0..3 with
+// two 128-row blocks each), in the order of the 12 blocks of 512 B of the global scale layout.
+constexpr uint32_t kTmemSf = 256, kTmemSfCols = 48;
+static_assert(kTmemSf + kGStages * kTmemSfCols <= kTmemCols, "TMEM columns");
 
 struct GemmParams {
   int M, N, K, rank, KB, MT2, NT, ldy;
   const float* bias;
-  uint16_t* Y;
 };
 
 // Box heights (256-byte rows) of the operand maps.
 constexpr uint32_t kBoxA = kGA / 256, kBoxB = kGB / 256, kBoxSfa = kGSfa / 256, kBoxSfb = kGSfb / 256, kBoxLr = 16;
 
 struct alignas(64) GemmMaps {
-  CUtensorMap a, b, sfa, sfb, t, l2;
+  CUtensorMap a, b, sfa, sfb, t, l2, y;
 };
 
 __device__ __forceinline__ void tmem_alloc2(uint32_t* slot, uint32_t ncols) {
@@ -613,10 +628,13 @@ __device__ __forceinline__ void tmem_relinquish2() {
 __device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
-// Arrive on the barrier at cluster address `bar` once all prior tcgen05 ops of this thread complete.
-__device__ __forceinline__ void tc_commit2(uint32_t bar_cluster_addr) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster_addr)
-               : "memory");
+// Arrive on the barrier at offset `bar` of both CTAs of the pair once all prior tcgen05 ops of
+// this thread complete.
+__device__ __forceinline__ void tc_commit2_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
 }
 __device__ __forceinline__ void mma2_bf16(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -635,21 +653,19 @@ __device__ __forceinline__ void mma2_nvfp4(uint32_t d, uint64_t ad, uint64_t bd,
       "l"(ad), "l"(bd), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
       : "memory");
 }
-__device__ __forceinline__ void tmem_cp2_32x128(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-// 2-D tensor copy of this CTA's box into its own shared memory; completion is counted on the
-// barrier at cluster address `bar` (the leader CTA's barrier for both CTAs of the pair).
-__device__ __forceinline__ void tma_rows_cg2(void* smem_dst, const CUtensorMap* map, int row, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-          "r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row), "r"(bar)
-      : "memory");
-}
-
+// Arrive on a barrier given by cluster address (possibly the peer CTA's).  Default (CTA-scope
+// release) semantics: what the arrival publishes is TMEM state, ordered by the tcgen05 wait and
+// fence that precede it, so no cluster-scope memory fence is needed (and it would stall the
+// warp behind every memory operation the SM has in flight).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
+// 2-D tensor store of a box from this CTA's shared memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t ssrc, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(ssrc)
+               : "memory");
 }
 __device__ __forceinline__ void bulk_s2g(void* gdst, uint32_t ssrc, uint32_t bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
@@ -659,14 +675,36 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Lane 0 waits (bounded) and the warp agrees on the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = !*abort_flag && wait_parity_bounded(bar, parity, kErrWaitGemm);
+  return __shfl_sync(0xffffffffu, ok, 0);
+}
+
+// Read-only 16-byte load kept in program order (volatile asm), so the compiler does not hoist
+// the epilogue's bias loads above the accumulator loads and run out of registers.
+__device__ __forceinline__ float4 ldg_f4_in_order(const float* ptr) {
+  float4 r;
+  asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(ptr));
+  return r;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+// Staging box layout: 32 rows of 128 bytes (64 bf16); 16-byte unit u of row l sits at
+// u ^ (l % 8), the tensor map's 128-byte swizzle, so lanes 8i..8i+7 hit distinct bank groups.
 __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_constant__ GemmMaps maps,
                                                                     const GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + kGStages * kGStage;
-  uint64_t* full = reinterpret_cast<uint64_t*>(staging + kGStaging);  // (leader) both CTAs' copies landed
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + kGStaging);  // (both) this CTA's tiles landed
   uint64_t* empty = full + kGStages;        // (both) MMAs done with the stage
-  uint64_t* acc_full = empty + kGStages;    // (both) accumulator ready
+  uint64_t* ready = empty + kGStages;       // (leader) both CTAs' tiles landed and scales written
+  uint64_t* acc_full = ready + kGStages;    // (both) accumulator ready
   uint64_t* acc_empty = acc_full + 1;       // (leader) both CTAs drained the accumulator
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -684,6 +722,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
     for (int s = 0; s < kGStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&ready[s], 2 * kGSfWarps);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kGEpiWarps);
@@ -702,9 +741,6 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer (both CTAs)
-      // Each CTA copies its own boxes; all copies complete on the leader's full barrier, which the
-      // leader arms with the bytes of both CTAs.
-      const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
       int st = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -717,22 +753,23 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
             break;
           }
           uint8_t* sb = smem + st * kGStage;
-          const uint32_t bar = full_leader + 8u * st;
           if (j < nlr) {
             const uint32_t cw = lr_chunk_width(r, j);
-            const uint32_t tb = kBM * cw * 2, lb = (kBN / 2) * cw * 2;  // per CTA
-            if (leader) mbar_arrive_expect_tx(&full[st], 2 * (tb + lb));
+            const uint32_t tb = kBM * cw * 2, lb = (kBN / 2) * cw * 2;
+            mbar_arrive_expect_tx(&full[st], tb + lb);
             const int trow = static_cast<int>((static_cast<size_t>(mt) * kBM * r * 2 + static_cast<size_t>(kBM) * kLrChunk * 2 * j) / 256);
             const int lrow = static_cast<int>((static_cast<size_t>(nt) * kBN * r * 2 + static_cast<size_t>(kBN) * kLrChunk * 2 * j + rank * lb) / 256);
-            for (uint32_t q = 0; q < tb / 4096; ++q) tma_rows_cg2(sb + 4096 * q, &maps.t, trow + 16 * q, bar);
-            for (uint32_t q = 0; q < lb / 4096; ++q) tma_rows_cg2(sb + kGA + 4096 * q, &maps.l2, lrow + 16 * q, bar);
+            for (uint32_t q = 0; q < tb / 4096; ++q) tma_load_2d(sb + 4096 * q, &maps.t, 0, trow + 16 * q, &full[st]);
+            for (uint32_t q = 0; q < lb / 4096; ++q) tma_load_2d(sb + kGA + 4096 * q, &maps.l2, 0, lrow + 16 * q, &full[st]);
           } else {
             const int kb = j - nlr;
-            if (leader) mbar_arrive_expect_tx(&full[st], 2 * kGStage);
-            tma_rows_cg2(sb, &maps.a, static_cast<int>(codes_chunk_offset(mt, kb, p.KB, kBM) / 256), bar);
-            tma_rows_cg2(sb + kGA, &maps.b, static_cast<int>((codes_chunk_offset(nt, kb, p.KB, kBN) + rank * kGB) / 256), bar);
-            tma_rows_cg2(sb + kGA + kGB, &maps.sfa, static_cast<int>(sf_chunk_offset(mt, kb, p.KB, kBM) / 256), bar);
-            tma_rows_cg2(sb + kGA + kGB + kGSfa, &maps.sfb, static_cast<int>(sf_chunk_offset(nt, kb, p.KB, kBN) / 256), bar);
+            mbar_arrive_expect_tx(&full[st], kGStage);
+            tma_load_2d(sb, &maps.a, 0, static_cast<int>(codes_chunk_offset(mt, kb, p.KB, kBM) / 256), &full[st]);
+            tma_load_2d(sb + kGA, &maps.b, 0, static_cast<int>((codes_chunk_offset(nt, kb, p.KB, kBN) + rank * kGB) / 256),
+                        &full[st]);
+            tma_load_2d(sb + kGA + kGB, &maps.sfa, 0, static_cast<int>(sf_chunk_offset(mt, kb, p.KB, kBM) / 256), &full[st]);
+            tma_load_2d(sb + kGA + kGB + kGSfa, &maps.sfb, 0, static_cast<int>(sf_chunk_offset(nt, kb, p.KB, kBN) / 256),
+                        &full[st]);
           }
           if (++st == kGStages) {
             st = 0;
@@ -747,8 +784,6 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
       // ------------------------------------------------------------ MMA issuer (leader CTA)
       const uint32_t id_lr = idesc_bf16(256, 256);
       const uint32_t id_fp4 = idesc_nvfp4(256, 256);
-      const uint32_t empty_local = smem_u32(empty), empty_peer = mapa_shared(smem_u32(empty), 1);
-      const uint32_t accf_local = smem_u32(acc_full), accf_peer = mapa_shared(smem_u32(acc_full), 1);
       int st = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -761,7 +796,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
         tc_fence_after();
         uint32_t accum = 0;
         for (int j = 0; j < nstages_tile; ++j) {
-          if (*abort_flag || !wait_parity_bounded(&full[st], ph, kErrWaitGemm)) {
+          if (*abort_flag || !wait_parity_bounded(&ready[st], ph, kErrWaitGemm)) {
             ok = false;
             break;
           }
@@ -776,90 +811,136 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
               accum = 1;
             }
           } else {
-            const uint32_t sfa = sb + kGA + kGB, sfb = sfa + kGSfa;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              tmem_cp2_32x128(tmem + kTmemSfa + 4 * kk, smem_desc(sfa + 512 * kk, 0, 128, kLayoutNone));
-              tmem_cp2_32x128(tmem + kTmemSfb + 8 * kk, smem_desc(sfb + 1024 * kk, 0, 128, kLayoutNone));
-              tmem_cp2_32x128(tmem + kTmemSfb + 8 * kk + 4, smem_desc(sfb + 1024 * kk + 512, 0, 128, kLayoutNone));
-            }
+            const uint32_t sf = tmem + kTmemSf + kTmemSfCols * static_cast<uint32_t>(st);
             const uint64_t ad = smem_desc(sb, 16, 1024, kLayoutSw128);
             const uint64_t bd = smem_desc(sb + kGA, 16, 1024, kLayoutSw128);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              mma2_nvfp4(tmem, ad + 2 * kk, bd + 2 * kk, id_fp4, tmem + kTmemSfa + 4 * kk, tmem + kTmemSfb + 8 * kk,
-                         accum);
+              mma2_nvfp4(tmem, ad + 2 * kk, bd + 2 * kk, id_fp4, sf + 4 * kk, sf + 16 + 8 * kk, accum);
               accum = 1;
             }
           }
-          tc_commit2(empty_local + 8u * st);
-          tc_commit2(empty_peer + 8u * st);
+          tc_commit2_both(smem_u32(&empty[st]));
           if (++st == kGStages) {
             st = 0;
             ph ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit2(accf_local);
-        tc_commit2(accf_peer);
+        tc_commit2_both(smem_u32(acc_full));
       }
       if (!ok) {
         *abort_flag = 1;
-        tc_commit2(accf_local);  // completes once every issued tcgen05 op has
-        tc_commit2(accf_peer);
+        tc_commit2_both(smem_u32(acc_full));  // completes once every issued tcgen05 op has
       }
     }
+  } else if (warp < kGFirstEpiWarp) {
+    // ------------------------------------------------------------ scale warps (both CTAs)
+    // Warp of lane quadrant q: lane l copies, for each of the stage's 12 scale blocks of 512 B in
+    // shared memory, bytes [16 l, 16 l + 16) into TMEM lane 32 q + l, four columns per block (the
+    // same contents in every quadrant, as the MMA's scale layout wants).
+    const int q = warp & 3;
+    const uint32_t ready_leader = mapa_shared(smem_u32(ready), 0);
+    const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16) + kTmemSf;
+    int st = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int tile = pair; tile < tiles && ok; tile += npairs) {
+      for (int j = 0; j < nstages_tile; ++j) {
+        if (!warp_wait(&full[st], ph, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (j >= nlr) {
+          tc_fence_after();  // the MMAs that last read this buffer completed before the stage refilled
+          const uint8_t* src = smem + st * kGStage + kGA + kGB + 16 * lane;
+          uint32_t v[3][16];
+#pragma unroll
+          for (int b = 0; b < 12; ++b) {
+            const uint4 w = *reinterpret_cast<const uint4*>(src + 512 * b);
+            v[b >> 2][4 * (b & 3) + 0] = w.x;
+            v[b >> 2][4 * (b & 3) + 1] = w.y;
+            v[b >> 2][4 * (b & 3) + 2] = w.z;
+            v[b >> 2][4 * (b & 3) + 3] = w.w;
+          }
+          const uint32_t dst = tq + kTmemSfCols * static_cast<uint32_t>(st);
+          tmem_st16(dst, v[0]);
+          tmem_st16(dst + 16, v[1]);
+          tmem_st16(dst + 32, v[2]);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(ready_leader + 8u * st);
+        if (++st == kGStages) {
+          st = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    if (!ok) *abort_flag = 1;
   } else {
     // ------------------------------------------------------------ epilogue (8 warps per CTA)
-    const int q = warp & 3, h = (warp - 2) >> 2;
+    // Warp (q, h): rows 32 q .. 32 q + 31 of this CTA's 128, columns 128 h .. 128 h + 127 of the
+    // tile; lane l holds row 32 q + l.  Two staging boxes of 32 rows x 64 columns (128-byte rows,
+    // 16-byte units swizzled by row % 8), stored by TMA.
+    const int q = warp & 3, h = (warp - kGFirstEpiWarp) >> 2;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
-    const int rloc = q * 32 + lane;                       // row inside this CTA's 128 rows
-    uint8_t* srow = staging + rloc * kGStagePitch + h * 256;  // this thread's 128 bf16 of the row
+    uint8_t* box0 = staging + (warp - kGFirstEpiWarp) * 2 * kGOutBox;
+    const uint32_t lrow = static_cast<uint32_t>(lane) * 128u;
     int local = 0;
     for (int tile = pair; tile < tiles; tile += npairs, ++local) {
-      bool ok = true;
-      if (lane == 0) ok = !*abort_flag && wait_parity_bounded(acc_full, static_cast<uint32_t>(local) & 1u, kErrWaitGemm);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
+      if (!warp_wait(acc_full, static_cast<uint32_t>(local) & 1u, abort_flag)) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
       const int m2 = tile / p.NT, nt = tile % p.NT;
-      uint32_t v[4][32];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * 128 + i * 32), v[i]);
+      const int row0 = (2 * m2 + static_cast<int>(rank)) * kBM + q * 32;
+      const int n0 = nt * kBN + h * 128;
+      const uint32_t tacc = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * 128);
+      // All 128 columns are read before the accumulator is released (the next tile's MMAs wait
+      // for it), then biased, rounded and staged.
+      uint32_t v[2][2][32];
+      tmem_ld32(tacc, v[0][0]);
+      tmem_ld32(tacc + 32, v[0][1]);
+      tmem_ld32(tacc + 64, v[1][0]);
+      tmem_ld32(tacc + 96, v[1][1]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(acc_empty_leader);  // the accumulator may be overwritten now
-      const int row = (2 * m2 + static_cast<int>(rank)) * kBM + rloc;
-      const int n0 = nt * kBN + h * 128;
-      bulk_wait_read0();  // the previous tile's stores have finished reading the staging rows
+      bulk_wait_read0();  // (lane 0's groups) the previous tile's stores have finished reading the staging boxes
+      __syncwarp();
+      // Row l of a box starts at a multiple of 128 B, so unit u's address (row + ((u ^ l % 8) << 4))
+      // is (row ^ ((l % 8) << 4)) ^ (u << 4): one XOR per store.
+      const uint32_t srow_swz[2] = {smem_u32(box0) + lrow ^ ((static_cast<uint32_t>(lane) & 7u) << 4),
+                                    smem_u32(box0 + kGOutBox) + lrow ^ ((static_cast<uint32_t>(lane) & 7u) << 4)};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int bx = 0; bx < 2; ++bx)
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int u = i * 4 + g;  // 16-byte unit of the row segment
-          const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8));
-          const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8 + 4));
+        for (int u = 0; u < 8; ++u) {  // 16-byte unit u: columns 8u .. 8u + 7 of the box
+          const int hh = u >> 2, c = 8 * (u & 3);
+          const float4 b0 = ldg_f4_in_order(p.bias + n0 + 64 * bx + 8 * u);
+          const float4 b1 = ldg_f4_in_order(p.bias + n0 + 64 * bx + 8 * u + 4);
           uint4 o;
-          o.x = pack_bf16x2(__uint_as_float(v[i][g * 8 + 0]) + b0.x, __uint_as_float(v[i][g * 8 + 1]) + b0.y);
-          o.y = pack_bf16x2(__uint_as_float(v[i][g * 8 + 2]) + b0.z, __uint_as_float(v[i][g * 8 + 3]) + b0.w);
-          o.z = pack_bf16x2(__uint_as_float(v[i][g * 8 + 4]) + b1.x, __uint_as_float(v[i][g * 8 + 5]) + b1.y);
-          o.w = pack_bf16x2(__uint_as_float(v[i][g * 8 + 6]) + b1.z, __uint_as_float(v[i][g * 8 + 7]) + b1.w);
-          *reinterpret_cast<uint4*>(srow + 16 * u) = o;  // row pitch 528 B: 8 lanes, 8 bank groups
+          o.x = pack_bf16x2(__uint_as_float(v[bx][hh][c + 0]) + b0.x, __uint_as_float(v[bx][hh][c + 1]) + b0.y);
+          o.y = pack_bf16x2(__uint_as_float(v[bx][hh][c + 2]) + b0.z, __uint_as_float(v[bx][hh][c + 3]) + b0.w);
+          o.z = pack_bf16x2(__uint_as_float(v[bx][hh][c + 4]) + b1.x, __uint_as_float(v[bx][hh][c + 5]) + b1.y);
+          o.w = pack_bf16x2(__uint_as_float(v[bx][hh][c + 6]) + b1.z, __uint_as_float(v[bx][hh][c + 7]) + b1.w);
+          st_shared_v4(srow_swz[bx] ^ (static_cast<uint32_t>(u) << 4), o);
         }
-      }
       fence_proxy_async_smem();
-      if (row < p.M && n0 < p.N) {
-        const int ncols = (p.N - n0) < 128 ? (p.N - n0) : 128;
-        bulk_s2g(p.Y + static_cast<size_t>(row) * p.ldy + n0, smem_u32(srow), static_cast<uint32_t>(ncols) * 2u);
+      __syncwarp();
+      if (lane == 0) {
+        if (row0 < p.M) {
+          if (n0 < p.N) tma_store_2d(&maps.y, smem_u32(box0), n0, row0);
+          if (n0 + 64 < p.N) tma_store_2d(&maps.y, smem_u32(box0 + kGOutBox), n0 + 64, row0);
+        }
+        bulk_commit();
       }
-      bulk_commit();
     }
-    bulk_wait0();
+    if (lane == 0) bulk_wait0();
   }
 
   __syncthreads();
@@ -1270,6 +1351,7 @@ static cudaError_t launch_gemm_int4(const GemmArgs& a, int num_sms, cudaStream_t
 static size_t gemm_smem_bytes() { return 1024 + kGStages * kGStage + kGStaging + 256; }
 
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
+  if (a.precision != 0) return launch_gemm_int4(a, num_sms, stream);
   GemmParams p;
   p.M = a.M;
   p.N = a.N;
@@ -1280,8 +1362,6 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   p.NT = (a.N + kBN - 1) / kBN;
   p.ldy = a.ldy;
   p.bias = a.bias;
-  p.Y = a.Y;
-  if (a.precision != 0) return launch_gemm_int4(a, num_sms, stream);
   const size_t mt = static_cast<size_t>(p.MT2) * 2, nt = static_cast<size_t>(p.NT), KB = static_cast<size_t>(p.KB);
   const size_t rr = static_cast<size_t>(a.rank);
   GemmMaps maps;
@@ -1293,6 +1373,18 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
       (me = make_rows_map(&maps.t, a.t, rr ? mt * kBM * rr * 2 : 4096, kBoxLr)) != cudaSuccess ||
       (me = make_rows_map(&maps.l2, a.l2, rr ? nt * kBN * rr * 2 : 4096, kBoxLr)) != cudaSuccess)
     return me;
+  {
+    // Y: M rows of N bf16 (row stride ldy), written in boxes of 32 rows x 64 columns, 128-byte swizzle.
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return cudaErrorInitializationError;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.N), static_cast<cuuint64_t>(a.M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.ldy) * 2};
+    const cuuint32_t box[2] = {64, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   const size_t smem = gemm_smem_bytes();
   cudaError_t e =
       cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
