@@ -577,8 +577,8 @@ static cudaError_t make_rows_map(CUtensorMap* map, const void* base, uint64_t by
 //
 // Every per-stage chain is kept short because each runs on one thread (or warp) whose
 // synchronisation and issue instructions have long latencies:
-//   producer (1 thread per CTA): wait empty[s]; A, B and scale tiles of this CTA by TMA onto its
-//     full[s];
+//   producers (2 threads per CTA): wait empty[s]; one copies the A and B tiles of this CTA by
+//     TMA onto its full[s] (arming it with the stage's bytes), the other the two scale tiles;
 //   scale warps (4 per CTA, one per TMEM lane quadrant): wait full[s], copy the stage's scale
 //     bytes from shared memory into the stage's TMEM scale buffer with tcgen05.st (instead of
 //     tcgen05.cp in the MMA issuer's instruction stream), then arrive on the leader's ready[s] --
@@ -586,20 +586,21 @@ static cudaError_t make_rows_map(CUtensorMap* map, const void* base, uint64_t by
 //   MMA issuer (leader, 1 thread): wait ready[s] (8 arrivals: both CTAs' scale warps); 4 MMAs;
 //     one commit multicast to empty[s] of both CTAs;
 //   epilogue (8 warps per CTA): drain the accumulator, add the bias, round to bf16 into a 128-byte
-//     swizzled staging tile and write it with two TMA tensor stores per warp.
+//     swizzled staging box and write it with a TMA tensor store, twice per warp.
 
-constexpr int kGStages = 4;
+constexpr int kGStages = 5;
 constexpr int kGSfWarps = 4;
 constexpr int kGEpiWarps = 8;
 constexpr int kGFirstEpiWarp = 2 + kGSfWarps;
-constexpr int kGThreads = (2 + kGSfWarps + kGEpiWarps) * 32;
+constexpr int kGScaleProducerWarp = kGFirstEpiWarp + kGEpiWarps;
+constexpr int kGThreads = (kGScaleProducerWarp + 1) * 32;
 constexpr uint32_t kGA = kBM * kRowBytes;                   // 16 KB: own 128 rows of A
 constexpr uint32_t kGB = (kBN / 2) * kRowBytes;             // 16 KB: own half of B
 constexpr uint32_t kGSfa = kBM * kSfBytesPerRowKb;          // 2 KB of A scales per (m-tile, k-block)
 constexpr uint32_t kGSfb = kBN * kSfBytesPerRowKb;          // 4 KB of B scales per (n-tile, k-block)
 constexpr uint32_t kGStage = kGA + kGB + kGSfa + kGSfb;     // 38 KB
 constexpr uint32_t kGOutBox = 32 * 128;                     // staging box: 32 rows x 64 bf16, 128-byte swizzle
-constexpr uint32_t kGStaging = kGEpiWarps * 2 * kGOutBox;   // 64 KB: two boxes per epilogue warp
+constexpr uint32_t kGStaging = kGEpiWarps * kGOutBox;       // 32 KB: one box per epilogue warp
 constexpr uint32_t kTmemCols = 512;
 // Per-stage scale buffer: 12 blocks of 4 columns (SFA k-steps 0..3, then SFB k-steps 0..3 with
 // two 128-row blocks each), in the order of the 12 blocks of 512 B of the global scale layout.
@@ -767,6 +768,34 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
             tma_load_2d(sb, &maps.a, 0, static_cast<int>(codes_chunk_offset(mt, kb, p.KB, kBM) / 256), &full[st]);
             tma_load_2d(sb + kGA, &maps.b, 0, static_cast<int>((codes_chunk_offset(nt, kb, p.KB, kBN) + rank * kGB) / 256),
                         &full[st]);
+          }
+          if (++st == kGStages) {
+            st = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) *abort_flag = 1;
+    }
+  } else if (warp == kGScaleProducerWarp) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ scale producer (both CTAs)
+      // Copies each k-block stage's two scale tiles onto full[s], which the operand producer arms
+      // with the whole stage's bytes (a copy may complete before that arrival; the phase cannot).
+      int st = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = pair; tile < tiles && ok; tile += npairs) {
+        const int m2 = tile / p.NT, nt = tile % p.NT;
+        const int mt = 2 * m2 + static_cast<int>(rank);
+        for (int j = 0; j < nstages_tile; ++j) {
+          if (j >= nlr) {
+            if (*abort_flag || !wait_parity_bounded(&empty[st], ph ^ 1u, kErrWaitGemm)) {
+              ok = false;
+              break;
+            }
+            const int kb = j - nlr;
+            uint8_t* sb = smem + st * kGStage;
             tma_load_2d(sb + kGA + kGB, &maps.sfa, 0, static_cast<int>(sf_chunk_offset(mt, kb, p.KB, kBM) / 256), &full[st]);
             tma_load_2d(sb + kGA + kGB + kGSfa, &maps.sfb, 0, static_cast<int>(sf_chunk_offset(nt, kb, p.KB, kBN) / 256),
                         &full[st]);
@@ -882,11 +911,11 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
   } else {
     // ------------------------------------------------------------ epilogue (8 warps per CTA)
     // Warp (q, h): rows 32 q .. 32 q + 31 of this CTA's 128, columns 128 h .. 128 h + 127 of the
-    // tile; lane l holds row 32 q + l.  Two staging boxes of 32 rows x 64 columns (128-byte rows,
-    // 16-byte units swizzled by row % 8), stored by TMA.
+    // tile; lane l holds row 32 q + l.  One staging box of 32 rows x 64 columns (128-byte rows,
+    // 16-byte units swizzled by row % 8), filled and stored by TMA twice per tile.
     const int q = warp & 3, h = (warp - kGFirstEpiWarp) >> 2;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
-    uint8_t* box0 = staging + (warp - kGFirstEpiWarp) * 2 * kGOutBox;
+    uint8_t* box = staging + (warp - kGFirstEpiWarp) * kGOutBox;
     const uint32_t lrow = static_cast<uint32_t>(lane) * 128u;
     int local = 0;
     for (int tile = pair; tile < tiles; tile += npairs, ++local) {
@@ -910,14 +939,13 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(acc_empty_leader);  // the accumulator may be overwritten now
-      bulk_wait_read0();  // (lane 0's groups) the previous tile's stores have finished reading the staging boxes
-      __syncwarp();
-      // Row l of a box starts at a multiple of 128 B, so unit u's address (row + ((u ^ l % 8) << 4))
+      // Row l of the box starts at a multiple of 128 B, so unit u's address (row + ((u ^ l % 8) << 4))
       // is (row ^ ((l % 8) << 4)) ^ (u << 4): one XOR per store.
-      const uint32_t srow_swz[2] = {smem_u32(box0) + lrow ^ ((static_cast<uint32_t>(lane) & 7u) << 4),
-                                    smem_u32(box0 + kGOutBox) + lrow ^ ((static_cast<uint32_t>(lane) & 7u) << 4)};
+      const uint32_t srow_swz = smem_u32(box) + lrow ^ ((static_cast<uint32_t>(lane) & 7u) << 4);
 #pragma unroll
-      for (int bx = 0; bx < 2; ++bx)
+      for (int bx = 0; bx < 2; ++bx) {
+        bulk_wait_read0();  // (lane 0's groups) the box's previous store has finished reading it
+        __syncwarp();
 #pragma unroll
         for (int u = 0; u < 8; ++u) {  // 16-byte unit u: columns 8u .. 8u + 7 of the box
           const int hh = u >> 2, c = 8 * (u & 3);
@@ -928,16 +956,14 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
           o.y = pack_bf16x2(__uint_as_float(v[bx][hh][c + 2]) + b0.z, __uint_as_float(v[bx][hh][c + 3]) + b0.w);
           o.z = pack_bf16x2(__uint_as_float(v[bx][hh][c + 4]) + b1.x, __uint_as_float(v[bx][hh][c + 5]) + b1.y);
           o.w = pack_bf16x2(__uint_as_float(v[bx][hh][c + 6]) + b1.z, __uint_as_float(v[bx][hh][c + 7]) + b1.w);
-          st_shared_v4(srow_swz[bx] ^ (static_cast<uint32_t>(u) << 4), o);
+          st_shared_v4(srow_swz ^ (static_cast<uint32_t>(u) << 4), o);
         }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        if (row0 < p.M) {
-          if (n0 < p.N) tma_store_2d(&maps.y, smem_u32(box0), n0, row0);
-          if (n0 + 64 < p.N) tma_store_2d(&maps.y, smem_u32(box0 + kGOutBox), n0 + 64, row0);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (row0 < p.M && n0 + 64 * bx < p.N) tma_store_2d(&maps.y, smem_u32(box), n0 + 64 * bx, row0);
+          bulk_commit();
         }
-        bulk_commit();
       }
     }
     if (lane == 0) bulk_wait0();
