@@ -181,93 +181,136 @@ __global__ void __launch_bounds__(kQdThreads, 1)
 
   if (warp < kQdWorkerWarps) {
     // ------------------------------------------------------------ workers
-    // Lane (sub, kg) of warp w handles 8 consecutive columns (16-byte unit kg) of rows
-    // 8w + sub and 8w + 4 + sub.  Quantization is exact (codes = E2M1_rne(RN(x / s)), resp.
-    // rint): the quotient is bracketed between x * RN(RN(1/s)(1 -+ 2^-20)); both roundings are
-    // monotonic, so when the two bracketing codes agree they are the exact codes, and
-    // otherwise (x/s within ~2^-20 of a threshold) the IEEE division decides.
-    const int sub = lane >> 3, kg = lane & 7;
-    const float kInv6 = __frcp_rn(6.0f);
-    for (int c = 0; c < nch; ++c) {
-      const int st = c % NS;
-      const bool ok = !*abort_flag && wait_parity_bounded(&full[st], (c / NS) & 1, kErrWaitQuantDown);
-      if (!__all_sync(0xffffffffu, ok)) {
-        *abort_flag = 1;
-        break;
-      }
-      const int gc = c0 + c;
-      const int col = gc * 64 + kg * 8;
-      const float4 il0 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + col));
-      const float4 il1 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + col + 4));
-      const float il[8] = {il0.x, il0.y, il0.z, il0.w, il1.x, il1.y, il1.z, il1.w};
-      const int kb = gc >> 2, cc = gc & 3;
-      uint8_t* codes_chunk = p.codes + codes_chunk_offset(mt, kb, p.KB, kBM);
-      uint8_t* sf_chunk = p.sf + sf_chunk_offset(mt, kb, p.KB, kBM);
-      uint8_t* xt = xs + st * kXsBytes;
-      int row[2];
-      uint4* cell[2];
-      float xh[2][8];
-      uint64_t xp[2][4];  // the same values as fp32 pairs
-      float amax[2];
-      uint64_t ilp[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) ilp[t] = f2pack(il[2 * t], il[2 * t + 1]);
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        row[i] = warp * 8 + i * 4 + sub;
-        cell[i] = reinterpret_cast<uint4*>(xt + swz128(row[i], kg * 16));
-        const uint4 xv = *cell[i];
-        const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          // bf16 -> fp32 is exact; x_hat = fp32(x) * (1/lambda), one rounding per element
-          xp[i][t] = f2mul(f2pack(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xFFFF0000u)), ilp[t]);
-          f2unpack(xp[i][t], xh[i][2 * t], xh[i][2 * t + 1]);
+    // Quantization is exact (codes = E2M1_rne(RN(x / s)), resp. rint(RN(x / s)) for INT4): the
+    // quotient is bracketed between x * RN(RN(1/s)(1 -+ 2^-20)); both roundings are monotonic, so
+    // when the two bracketing codes agree they are the exact codes, and otherwise (x/s within
+    // ~2^-20 of a threshold) the IEEE division decides.
+    if (PREC == 0) {
+      // NVFP4: thread t of the 512 handles one 16-element group per 64-column chunk: row t / 4,
+      // group t % 4 (two swizzled 16-byte units; the quarter-warps' loads hit distinct banks).
+      const int row = warp * 8 + (lane >> 2), g = lane & 3;
+      const float kInv6 = __frcp_rn(6.0f);
+      for (int c = 0; c < nch; ++c) {
+        const int st = c % NS;
+        const bool ok = !*abort_flag && wait_parity_bounded(&full[st], (c / NS) & 1, kErrWaitQuantDown);
+        if (!__all_sync(0xffffffffu, ok)) {
+          *abort_flag = 1;
+          break;
         }
-        amax[i] = fmaxf(fmaxf(fmaxf(fabsf(xh[i][0]), fabsf(xh[i][1])), fmaxf(fabsf(xh[i][2]), fabsf(xh[i][3]))),
-                        fmaxf(fmaxf(fabsf(xh[i][4]), fabsf(xh[i][5])), fmaxf(fabsf(xh[i][6]), fabsf(xh[i][7]))));
-      }
-      uint32_t codes[2], sbits[2];
-      if (PREC == 0) {
+        const int gc = c0 + c;
+        const int kb = gc >> 2, cc = gc & 3;
+        const float4* ilv = reinterpret_cast<const float4*>(p.inv_lambda + gc * 64 + g * 16);
+        uint8_t* xt = xs + st * kXsBytes;
+        uint4* cell0 = reinterpret_cast<uint4*>(xt + swz128(row, g * 32));
+        uint4* cell1 = reinterpret_cast<uint4*>(xt + swz128(row, g * 32 + 16));
+        const uint4 xa = *cell0, xb = *cell1;
+        const uint32_t w[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+        uint64_t xp[2][4];  // x_hat as fp32 pairs: element 2t, 2t + 1 of half h in xp[h][t]
+        float amax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 1));
-        bool slow = false;
+        for (int h = 0; h < 2; ++h) {
+          const float4 i0 = __ldg(ilv + 2 * h), i1 = __ldg(ilv + 2 * h + 1);
+          const float il[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          // scale code: UE4M3_rne(RN(amax / 6)), bracketed the same way
-          const float s_est = __fmul_rn(amax[i], kInv6);
-          const uint32_t sc_lo = cvt_e4m3(__fmul_rn(s_est, kNudgeLo));
-          const uint32_t sc_hi = cvt_e4m3(__fmul_rn(s_est, kNudgeHi));
-          sbits[i] = sc_lo;
-          codes[i] = 0;
-          if (sc_lo == sc_hi) {
-            if (sc_lo != 0) {
-              const float rr = rcp_tbl[sc_lo];
-              const uint32_t lo = e2m1x8_scaled(xp[i], __fmul_rn(rr, kNudgeLo));
-              const uint32_t hi = e2m1x8_scaled(xp[i], __fmul_rn(rr, kNudgeHi));
-              codes[i] = lo;
-              slow |= lo != hi;
+          for (int t = 0; t < 4; ++t) {
+            // bf16 -> fp32 is exact; x_hat = fp32(x) * (1/lambda), one rounding per element
+            const uint32_t ww = w[4 * h + t];
+            xp[h][t] = f2mul(f2pack(__uint_as_float(ww << 16), __uint_as_float(ww & 0xFFFF0000u)),
+                             f2pack(il[2 * t], il[2 * t + 1]));
+            float lo, hi;
+            f2unpack(xp[h][t], lo, hi);
+            amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+          }
+        }
+        // scale code: UE4M3_rne(RN(amax / 6)), bracketed the same way
+        const float s_est = __fmul_rn(amax, kInv6);
+        uint32_t sbits = cvt_e4m3(__fmul_rn(s_est, kNudgeLo));
+        const uint32_t sc_hi = cvt_e4m3(__fmul_rn(s_est, kNudgeHi));
+        uint2 code = make_uint2(0u, 0u);
+        bool slow = sbits != sc_hi;
+        if (!slow && sbits != 0) {
+          const float rr = rcp_tbl[sbits];
+          const float mlo = __fmul_rn(rr, kNudgeLo), mhi = __fmul_rn(rr, kNudgeHi);
+          code.x = e2m1x8_scaled(xp[0], mlo);
+          code.y = e2m1x8_scaled(xp[1], mlo);
+          slow = (code.x != e2m1x8_scaled(xp[0], mhi)) | (code.y != e2m1x8_scaled(xp[1], mhi));
+        }
+        if (slow) {  // rare: the exact quotients decide
+          float xh[2][8];
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int t = 0; t < 4; ++t) f2unpack(xp[h][t], xh[h][2 * t], xh[h][2 * t + 1]);
+          sbits = cvt_e4m3(__fdiv_rn(amax, 6.0f));
+          const float sd = e4m3_to_f32(sbits);
+          code.x = sd != 0.0f ? e2m1x8_div(xh[0], sd) : 0u;
+          code.y = sd != 0.0f ? e2m1x8_div(xh[1], sd) : 0u;
+        }
+        *reinterpret_cast<uint2*>(p.codes + codes_chunk_offset(mt, kb, p.KB, kBM) + swz128(row, cc * 32 + g * 8)) = code;
+        p.sf[sf_chunk_offset(mt, kb, p.KB, kBM) + cc * 512 + (row & 31) * 16 + (row >> 5) * 4 + g] =
+            static_cast<uint8_t>(sbits);
+        if (has_lr) {
+          uint32_t hv[8];
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              float lo, hi;
+              f2unpack(xp[h][t], lo, hi);
+              hv[4 * h + t] = pack_bf16x2(lo, hi);
             }
-          } else {
-            slow = true;
-          }
+          *cell0 = make_uint4(hv[0], hv[1], hv[2], hv[3]);  // bf16(x_hat) in place: the MMA's A operand
+          *cell1 = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+          fence_proxy_async_smem();
         }
-        if (slow) {  // rare: recompute both rows exactly
+        __syncwarp();
+        if (lane == 0) mbar_arrive(has_lr ? &xready[st] : &empty[st]);
+      }
+    } else {
+      // INT4: lane (sub, kg) of warp w handles 8 consecutive columns (16-byte unit kg) of rows
+      // 8w + sub and 8w + 4 + sub; the 64-element group spans the 8 lanes of a row.
+      const int sub = lane >> 3, kg = lane & 7;
+      for (int c = 0; c < nch; ++c) {
+        const int st = c % NS;
+        const bool ok = !*abort_flag && wait_parity_bounded(&full[st], (c / NS) & 1, kErrWaitQuantDown);
+        if (!__all_sync(0xffffffffu, ok)) {
+          *abort_flag = 1;
+          break;
+        }
+        const int gc = c0 + c;
+        const int col = gc * 64 + kg * 8;
+        const float4 il0 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + col));
+        const float4 il1 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + col + 4));
+        const float il[8] = {il0.x, il0.y, il0.z, il0.w, il1.x, il1.y, il1.z, il1.w};
+        const int kb = gc >> 2, cc = gc & 3;
+        uint8_t* codes_chunk = p.codes + codes_chunk_offset(mt, kb, p.KB, kBM);
+        uint8_t* sf_chunk = p.sf + sf_chunk_offset(mt, kb, p.KB, kBM);
+        uint8_t* xt = xs + st * kXsBytes;
+        int row[2];
+        uint4* cell[2];
+        float xh[2][8];
+        float amax[2];
+        uint64_t ilp[4];
 #pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const uint32_t sc = cvt_e4m3(__fdiv_rn(amax[i], 6.0f));
-            const float sd = e4m3_to_f32(sc);
-            sbits[i] = sc;
-            codes[i] = sd != 0.0f ? e2m1x8_div(xh[i], sd) : 0u;
-          }
-        }
-      } else {
+        for (int t = 0; t < 4; ++t) ilp[t] = f2pack(il[2 * t], il[2 * t + 1]);
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
+          row[i] = warp * 8 + i * 4 + sub;
+          cell[i] = reinterpret_cast<uint4*>(xt + swz128(row[i], kg * 16));
+          const uint4 xv = *cell[i];
+          const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const uint64_t xp = f2mul(f2pack(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xFFFF0000u)), ilp[t]);
+            f2unpack(xp, xh[i][2 * t], xh[i][2 * t + 1]);
+          }
+          amax[i] = fmaxf(fmaxf(fmaxf(fabsf(xh[i][0]), fabsf(xh[i][1])), fmaxf(fabsf(xh[i][2]), fabsf(xh[i][3]))),
+                          fmaxf(fmaxf(fabsf(xh[i][4]), fabsf(xh[i][5])), fmaxf(fabsf(xh[i][6]), fabsf(xh[i][7]))));
           amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 1));
           amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 2));
           amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 4));
         }
+        uint32_t codes[2], sbits[2];
         bool slow = false;
         float sc[2];
 #pragma unroll
@@ -291,29 +334,23 @@ __global__ void __launch_bounds__(kQdThreads, 1)
 #pragma unroll
           for (int i = 0; i < 2; ++i) codes[i] = sc[i] != 0.0f ? int4x8_div(xh[i], sc[i]) : 0u;
         }
-      }
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        *reinterpret_cast<uint32_t*>(codes_chunk + swz128(row[i], cc * 32 + kg * 4)) = codes[i];
-        if (PREC == 0) {
-          // the pair (kg, kg+1) shares one 16-group; the even lane stores its scale byte
-          if ((kg & 1) == 0)
-            sf_chunk[cc * 512 + (row[i] & 31) * 16 + (row[i] >> 5) * 4 + (kg >> 1)] = static_cast<uint8_t>(sbits[i]);
-        } else {
+        for (int i = 0; i < 2; ++i) {
+          *reinterpret_cast<uint32_t*>(codes_chunk + swz128(row[i], cc * 32 + kg * 4)) = codes[i];
           if (kg == 0) reinterpret_cast<uint32_t*>(sf_chunk)[sf_int4_a_index(row[i], cc)] = sbits[i];
+          if (has_lr) {
+            uint4 hv;
+            hv.x = pack_bf16x2(xh[i][0], xh[i][1]);
+            hv.y = pack_bf16x2(xh[i][2], xh[i][3]);
+            hv.z = pack_bf16x2(xh[i][4], xh[i][5]);
+            hv.w = pack_bf16x2(xh[i][6], xh[i][7]);
+            *cell[i] = hv;  // bf16(x_hat) in place: the tile becomes the MMA's A operand
+          }
         }
-        if (has_lr) {
-          uint4 hv;
-          hv.x = pack_bf16x2(xh[i][0], xh[i][1]);
-          hv.y = pack_bf16x2(xh[i][2], xh[i][3]);
-          hv.z = pack_bf16x2(xh[i][4], xh[i][5]);
-          hv.w = pack_bf16x2(xh[i][6], xh[i][7]);
-          *cell[i] = hv;  // bf16(x_hat) in place: the tile becomes the MMA's A operand
-        }
+        if (has_lr) fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(has_lr ? &xready[st] : &empty[st]);
       }
-      if (has_lr) fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(has_lr ? &xready[st] : &empty[st]);
     }
   } else if (warp == kQdTmaWarp) {
     if (lane == 0) {
