@@ -142,7 +142,10 @@ svdq_status svdq_workspace_size(const svdq_weights* w, int M, size_t* bytes);
  *     writes Y = bf16_rn(acc) once.
  * X:  device, M rows of K bf16, row stride ldx elements.   Y: device, M x N bf16, stride ldy.
  * workspace: device, >= svdq_workspace_size(w, M) bytes, 256-byte aligned; holds the codes,
- *   scales and T between the two kernels; contents are scratch.
+ *   scales and T between the two kernels and, when kernel 1 splits K, the fp32 partials of T and
+ *   one arrival counter per 128-row tile; contents are scratch and need no initialisation (a
+ *   counter tagged with another launch restarts; the last slice resets it).  One workspace must
+ *   not be used by two forwards whose kernels overlap on the GPU.
  * No allocation, no synchronisation.  Errors: INVALID_ARG, CUDA (launch failure). */
 svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
                                 void* workspace, size_t workspace_bytes, void* stream);
@@ -151,7 +154,7 @@ svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int
  * counterpart to this call: it exists for callers that cannot allocate device memory while they
  * run, for instance code inside a host framework that owns all device memory and hands its
  * plugins no allocator, or a latency-critical path where cudaMalloc (which may synchronise the
- * device) is not acceptable.  The scratch between the two kernels is a fixed 16 MiB array in the
+ * device) is not acceptable.  The scratch between the two kernels is a fixed 20 MiB array in the
  * library's own device module, which every GPU that loads the library keeps until the process
  * exits.  The first call on a device looks up that array's device address (cudaGetSymbolAddress,
  * with the device current) and caches it; make that first call before any stream capture.
@@ -159,8 +162,8 @@ svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int
  * whose kernels overlap on the GPU (different streams, no ordering between them) race and give
  * wrong results, so order them on one stream or use svdq_linear_forward with separate
  * workspaces.  Nothing in the array has to start at zero.  Shapes whose workspace
- * (svdq_workspace_size) exceeds 16 MiB are rejected with SVDQ_ERR_INVALID_ARG; at K = 3072 and
- * rank 32 that allows M up to 9216.  Other arguments and errors as svdq_linear_forward. */
+ * (svdq_workspace_size) exceeds 20 MiB are rejected with SVDQ_ERR_INVALID_ARG; at K = 3072 and
+ * rank 32 that allows every M up to 9984.  Other arguments and errors as svdq_linear_forward. */
 svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
                                         void* stream);
 

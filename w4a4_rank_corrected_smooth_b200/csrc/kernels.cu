@@ -17,6 +17,7 @@
 // accumulator in tensor memory; eight epilogue warps drain the accumulator, add the bias and
 // write bf16 Y once.
 #include <cuda.h>
+#include <atomic>
 #include <mutex>
 #include <cuda_bf16.h>
 
@@ -34,6 +35,7 @@ constexpr int kQdMmaWarp = kQdWorkerWarps;        // tcgen05 MMA issuer (+ TMEM 
 constexpr int kQdTmaWarp = kQdWorkerWarps + 1;    // TMA producer
 constexpr int kQdThreads = (kQdWorkerWarps + 2) * 32;
 constexpr uint32_t kXsBytes = kBM * 128;  // one stage of X: 128 rows x 64 bf16, 128-byte swizzle
+constexpr uint32_t kIlBytes = 64 * 4;     // the stage's 64 values of 1/lambda
 constexpr size_t kQdSmemBudget = 220 * 1024;
 // Relative nudges that bracket a correctly rounded quotient (see the worker loop).
 constexpr float kNudgeLo = 1.0f - 0x1p-20f;
@@ -46,7 +48,28 @@ struct QdParams {
   uint8_t* codes;
   uint8_t* sf;
   uint8_t* t;
+  float* part;              // [m-tile][split][128][rank] fp32 partials of T (splits > 1)
+  unsigned long long* cnt;  // per m-tile: (launch epoch << 8) | slices arrived
+  unsigned long long epoch; // distinct per launch, never 0
 };
+
+// Counts this CTA's slice in the tile's counter and returns whether it was the last of `splits`.
+// The counter holds (epoch << 8) | count; a value from another launch (or uninitialised memory)
+// restarts the count, and the last CTA resets it to 0, so a replay of the same launch also starts
+// from 0.  Lock-free (a failed CAS means another slice succeeded); bounded all the same.
+__device__ __forceinline__ bool arrive_slice_counter(unsigned long long* cnt, unsigned long long epoch, int splits,
+                                                     bool* ok) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(cnt);
+  for (int it = 0; it < (1 << 20); ++it) {
+    const unsigned long long nxt = (cur >> 8) == epoch ? cur + 1 : ((epoch << 8) | 1ull);
+    const unsigned long long prev = atomicCAS(cnt, cur, nxt);
+    if (prev == cur) return static_cast<int>(nxt & 0xFFull) == splits;
+    cur = prev;
+  }
+  atomicOr(&g_device_error, kErrWaitQuantDown);
+  *ok = false;
+  return false;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -144,7 +167,8 @@ __global__ void __launch_bounds__(kQdThreads, 1)
   const uint32_t l1_stride = static_cast<uint32_t>(align_up(l1_bytes, 1024));
   uint8_t* xs = smem;                       // NS x 16 KB (X, then bf16 x_hat in place)
   uint8_t* l1s = smem + NS * kXsBytes;      // NS x r*128 (L1 chunk)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(l1s + NS * l1_stride);
+  const float* ils = reinterpret_cast<const float*>(l1s + NS * l1_stride);  // NS x 64 fp32 (1/lambda chunk)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(l1s + NS * l1_stride + NS * kIlBytes);
   uint64_t* full = bars;                    // TMA landed: X tile (+ L1 chunk)
   uint64_t* xready = bars + NS;             // workers wrote x_hat (one arrive per worker warp)
   uint64_t* empty = bars + 2 * NS;          // stage free again
@@ -154,7 +178,7 @@ __global__ void __launch_bounds__(kQdThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int mt = blockIdx.x / p.splits;
-  const int split = blockIdx.x % p.splits;  // == rank in the cluster (clusters are consecutive blocks)
+  const int split = blockIdx.x % p.splits;
   const int kb0 = split * p.KB / p.splits, kb1 = (split + 1) * p.KB / p.splits;
   const int c0 = kb0 * 4, nch = (kb1 - kb0) * 4;
   const uint32_t tmem_cols = r <= 32 ? 32u : (r <= 64 ? 64u : 128u);
@@ -199,7 +223,7 @@ __global__ void __launch_bounds__(kQdThreads, 1)
         }
         const int gc = c0 + c;
         const int kb = gc >> 2, cc = gc & 3;
-        const float4* ilv = reinterpret_cast<const float4*>(p.inv_lambda + gc * 64 + g * 16);
+        const float4* ilv = reinterpret_cast<const float4*>(ils + st * 64 + g * 16);
         uint8_t* xt = xs + st * kXsBytes;
         uint4* cell0 = reinterpret_cast<uint4*>(xt + swz128(row, g * 32));
         uint4* cell1 = reinterpret_cast<uint4*>(xt + swz128(row, g * 32 + 16));
@@ -209,7 +233,7 @@ __global__ void __launch_bounds__(kQdThreads, 1)
         float amax = 0.0f;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const float4 i0 = __ldg(ilv + 2 * h), i1 = __ldg(ilv + 2 * h + 1);
+          const float4 i0 = ilv[2 * h], i1 = ilv[2 * h + 1];
           const float il[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
@@ -278,9 +302,8 @@ __global__ void __launch_bounds__(kQdThreads, 1)
           break;
         }
         const int gc = c0 + c;
-        const int col = gc * 64 + kg * 8;
-        const float4 il0 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + col));
-        const float4 il1 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + col + 4));
+        const float4 il0 = *reinterpret_cast<const float4*>(ils + st * 64 + kg * 8);
+        const float4 il1 = *reinterpret_cast<const float4*>(ils + st * 64 + kg * 8 + 4);
         const float il[8] = {il0.x, il0.y, il0.z, il0.w, il1.x, il1.y, il1.z, il1.w};
         const int kb = gc >> 2, cc = gc & 3;
         uint8_t* codes_chunk = p.codes + codes_chunk_offset(mt, kb, p.KB, kBM);
@@ -362,8 +385,9 @@ __global__ void __launch_bounds__(kQdThreads, 1)
           *abort_flag = 1;
           break;
         }
-        mbar_arrive_expect_tx(&full[st], kXsBytes + (has_lr ? l1_bytes : 0u));
+        mbar_arrive_expect_tx(&full[st], kXsBytes + kIlBytes + (has_lr ? l1_bytes : 0u));
         tma_load_2d(xs + st * kXsBytes, &tmap_x, (c0 + c) * 64, mt * kBM, &full[st]);
+        bulk_g2s(const_cast<float*>(ils) + st * 64, p.inv_lambda + static_cast<size_t>(c0 + c) * 64, kIlBytes, &full[st]);
         if (has_lr)
           bulk_g2s(l1s + st * l1_stride, p.l1 + static_cast<size_t>(c0 + c) * l1_bytes, l1_bytes, &full[st]);
         ++issued;
@@ -398,13 +422,13 @@ __global__ void __launch_bounds__(kQdThreads, 1)
   // ---------------------------------------------------------------- T epilogue
   __syncthreads();
   const bool aborted = *abort_flag != 0;
-  float* part = reinterpret_cast<float*>(xs);  // 128 x r fp32 partial (reuses the X stages)
   if (has_lr && warp < 4) {
     bool ok = !aborted && wait_parity_bounded(done, 0, kErrWaitQuantDown);
     ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-collective
     tc_fence_after();
     if (ok) {
       const int row = warp * 32 + lane;
+      float* prow = p.splits > 1 ? p.part + ((static_cast<size_t>(mt) * p.splits + split) * kBM + row) * r : nullptr;
       for (int j = 0; j < r; j += 16) {
         uint32_t v[16];
         tmem_ld16(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + j, v);
@@ -423,28 +447,36 @@ __global__ void __launch_bounds__(kQdThreads, 1)
         } else {
 #pragma unroll
           for (int q = 0; q < 16; q += 4)
-            *reinterpret_cast<float4*>(part + row * r + j + q) =
-                make_float4(__uint_as_float(v[q]), __uint_as_float(v[q + 1]), __uint_as_float(v[q + 2]),
-                            __uint_as_float(v[q + 3]));
+            *reinterpret_cast<float4*>(prow + j + q) = make_float4(__uint_as_float(v[q]), __uint_as_float(v[q + 1]),
+                                                                   __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]));
         }
       }
+      if (p.splits > 1) __threadfence();  // each writer publishes its partial row at GPU scope
     }
   }
   if (has_lr && p.splits > 1) {
-    // Fixed-order reduction of the cluster's partials: rank s sums rows [s*128/S, (s+1)*128/S).
-    // Every thread of every CTA passes both cluster barriers, whatever happened before.
-    cluster_sync();
-    if (warp < kQdWorkerWarps && !aborted) {
-      const int rlo = split * kBM / p.splits, rhi = (split + 1) * kBM / p.splits;
-      const int units = (rhi - rlo) * r / 4;
-      const uint32_t part_addr = smem_u32(part);
+    // The last slice of the tile to finish sums all slices' partials in slice order
+    // (deterministic) and writes bf16 T.
+    __shared__ int s_last;
+    __syncthreads();  // this CTA's partial rows are written
+    if (threadIdx.x == 0) {
+      bool ok = !aborted;
+      __threadfence();  // publish the partials before counting this slice
+      const bool last = ok && arrive_slice_counter(p.cnt + mt, p.epoch, p.splits, &ok);
+      if (!ok) *abort_flag = 1;
+      s_last = last ? 1 : 0;
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
       uint8_t* tt = p.t + static_cast<size_t>(mt) * kBM * r * 2;
-      for (int u = threadIdx.x; u < units; u += kQdWorkerWarps * 32) {
-        const int row = rlo + (u * 4) / r, col = (u * 4) % r;
-        const uint32_t off = static_cast<uint32_t>((row * r + col) * 4);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q = 0; q < p.splits; ++q) {
-          const float4 x = ld_shared_cluster_f4(mapa_shared(part_addr + off, static_cast<uint32_t>(q)));
+      const float* pt = p.part + static_cast<size_t>(mt) * p.splits * kBM * r;
+      const int units = kBM * r / 4;
+      for (int u = threadIdx.x; u < units; u += blockDim.x) {
+        const int row = (u * 4) / r, col = (u * 4) % r;
+        float4 acc = __ldcg(reinterpret_cast<const float4*>(pt + row * r + col));
+        for (int q = 1; q < p.splits; ++q) {
+          const float4 x = __ldcg(reinterpret_cast<const float4*>(pt + (static_cast<size_t>(q) * kBM + row) * r + col));
           acc.x += x.x;
           acc.y += x.y;
           acc.z += x.z;
@@ -455,8 +487,8 @@ __global__ void __launch_bounds__(kQdThreads, 1)
         o.y = pack_bf16x2(acc.z, acc.w);
         *reinterpret_cast<uint2*>(tt + lr_offset(row, col, kBM, r)) = o;
       }
+      if (threadIdx.x == 0) atomicExch(p.cnt + mt, 0ull);
     }
-    cluster_sync();
   }
   tc_fence_before();
   __syncthreads();
@@ -466,64 +498,15 @@ __global__ void __launch_bounds__(kQdThreads, 1)
   }
 }
 
-// Largest number of co-resident clusters of `splits` CTAs for one launch configuration; the query
-// runs once per (kernel, splits, shared-memory size) and is cached.
-static int max_active_clusters(void (*kern)(const CUtensorMap, const QdParams), int splits, size_t smem) {
-  struct Entry { const void* k; int s; size_t smem; int n; };
-  static Entry cache[64];
-  static int used = 0;
-  for (int i = 0; i < used; ++i)
-    if (cache[i].k == reinterpret_cast<const void*>(kern) && cache[i].s == splits && cache[i].smem == smem)
-      return cache[i].n;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(splits));
-  cfg.blockDim = dim3(kQdThreads);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
-    cudaGetLastError();
-    n = 1;
-  }
-  if (used < 64) cache[used++] = Entry{reinterpret_cast<const void*>(kern), splits, smem, n};
-  return n;
-}
-
-// The K slices of one 128-row tile form one cluster (<= 8 CTAs).  The split count minimises
-// (waves of co-resident clusters) x (k-blocks per CTA): a second partial wave would double the
-// time, so the grid is kept to what fits on the GPU at once.
-static int choose_splits(void (*kern)(const CUtensorMap, const QdParams), int M, int K, size_t smem) {
-  const int mt = 2 * ((M + 2 * kBM - 1) / (2 * kBM));
-  const int KB = K / kBK;
-  int best = 1;
-  long best_cost = -1;
-  for (int s = 1; s <= 8 && s <= KB; ++s) {
-    const int active = max_active_clusters(kern, s, smem);
-    const long waves = (mt + active - 1) / active;
-    const long cost = waves * ((KB + s - 1) / s);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = s;
-    }
-  }
-  return best;
-}
-
 static int quant_down_stages(int r) {
-  const size_t per = kXsBytes + align_up(static_cast<size_t>(r) * 128, 1024);
+  const size_t per = kXsBytes + align_up(static_cast<size_t>(r) * 128, 1024) + kIlBytes;
   const int ns = static_cast<int>((kQdSmemBudget - 2048) / per);
   return ns < kQdMaxStages ? ns : kQdMaxStages;
 }
 
 static size_t quant_down_smem_bytes(int r) {
   const int ns = quant_down_stages(r);
-  return 1024 + ns * (kXsBytes + align_up(static_cast<size_t>(r) * 128, 1024)) + 256;
+  return 1024 + ns * (kXsBytes + align_up(static_cast<size_t>(r) * 128, 1024) + kIlBytes) + 256;
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link dependency).
@@ -571,21 +554,23 @@ cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t 
   void (*kern)(const CUtensorMap, const QdParams) = a.precision == 0 ? quant_down_kernel<0> : quant_down_kernel<1>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  (void)num_sms;
-  p.splits = choose_splits(kern, a.M, a.K, smem);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(mt * p.splits));
-  cfg.blockDim = dim3(kQdThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(p.splits);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tmap, p);
+  // One CTA per SM (shared memory), one wave: as many K slices per tile as the SMs allow, within
+  // what the workspace's partials have room for.
+  int splits = num_sms / mt;
+  if (splits > a.split_cap) splits = a.split_cap;
+  if (splits < 1) splits = 1;
+  if (a.rank > 0 && splits > 1 && (!a.part || !a.cnt)) splits = 1;
+  p.splits = splits;
+  p.part = a.part;
+  p.cnt = a.cnt;
+  static std::atomic<unsigned long long> epoch_counter{0};
+  p.epoch = (epoch_counter.fetch_add(1) + 1) & ((1ull << 56) - 1);
+  if (p.epoch == 0) p.epoch = 1;
+  if (a.precision == 0)
+    quant_down_kernel<0><<<mt * splits, kQdThreads, smem, stream>>>(tmap, p);
+  else
+    quant_down_kernel<1><<<mt * splits, kQdThreads, smem, stream>>>(tmap, p);
+  return cudaGetLastError();
 }
 
 
@@ -1475,7 +1460,7 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
 // Scratch of svdq_linear_forward_noalloc: a fixed array in the module's global memory, so that
 // the forward can run without any device allocation.  Every device that loads the library holds
 // it until the process exits.
-constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(20) << 20;  // 20 MiB
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
