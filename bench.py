@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--sets", type=int, default=3, help="rotating copies of the layer")
     ap.add_argument("--no-extras", action="store_true", help="skip overhead, e2e and CPU-baseline legs")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one JSON line per FLUX-shaped layer and per point of the M x rank sweep (not the driver's line)")
     return ap.parse_args()
 
 
@@ -295,25 +297,98 @@ def run_reference(args):
 # ---------------------------------------------------------------- our arm
 
 
-def time_loop(layers, sets, steps, stream):
-    """Runs `steps` steps rotating over `sets`; returns (total_ms, mean k1 ms, mean k2 ms)."""
+def time_loop(layers, sets, steps, stream, sample_every: int = 8):
+    """Runs `steps` steps rotating over `sets`; returns (total_ms, mean k1 ms, mean k2 ms).
+
+    The total comes from events before the first and after the last step.  The per-kernel
+    durations come from events around the two kernels of every `sample_every`-th step only: an
+    event between the kernels would keep kernel 2's prologue from overlapping kernel 1's tail
+    (programmatic dependent launch), so most steps run without one."""
     import torch
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    samples = []
+    start.record(stream)
     for i in range(steps):
         lin = layers[i % len(layers)]
         X, Y, ws = sets[i % len(sets)]
         M = X.shape[0]
-        ev[i][0].record(stream)
+        sampled = i % sample_every == sample_every // 2 or steps < sample_every
+        if sampled:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            ev[0].record(stream)
         lin.svdq_quant_down(X, M, X.stride(0), ws, ws.numel(), stream)
-        ev[i][1].record(stream)
+        if sampled:
+            ev[1].record(stream)
         lin.svdq_gemm_up(M, Y, Y.stride(0), ws, ws.numel(), stream)
-        ev[i][2].record(stream)
+        if sampled:
+            ev[2].record(stream)
+            samples.append(ev)
+    end.record(stream)
     torch.cuda.synchronize()
-    total = ev[0][0].elapsed_time(ev[-1][2])
-    k1 = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
-    k2 = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+    total = start.elapsed_time(end)
+    k1 = sum(e[0].elapsed_time(e[1]) for e in samples) / len(samples)
+    k2 = sum(e[1].elapsed_time(e[2]) for e in samples) / len(samples)
     return total, k1, k2
+
+
+def unfused_comparator(lin, layers, sets, layers0, sets0, steps, stream, k2_bare_ms):
+    """The same layer with the low-rank branch unfused (the pages' naive version, for context):
+    kernel 1 and kernel 2 of the rank-0 layer, plus a separate down projection that reads X again
+    (one cuBLAS GEMM with the smoothing folded into L1: X (diag(1/lambda) L1)) and a separate up
+    projection that reads and rewrites Y (Y += T L2, one cuBLAS GEMM with beta = 1).  Not the
+    product: a timing comparator only.  All three variants are timed as whole steps."""
+    import numpy as np
+    import torch
+
+    dev = sets[0][0].device
+    ops = lin.export_weights()
+    il = torch.from_numpy(ops["inv_lambda"].astype(np.float32)).to(dev)
+    L1 = bf16_device(ops["L1"], dev).float()
+    L1s = (il[:, None] * L1).to(torch.bfloat16).contiguous()
+    L2 = bf16_device(ops["L2"], dev).contiguous()
+    Ts = [torch.empty((x.shape[0], L1s.shape[1]), dtype=torch.bfloat16, device=dev) for (x, _, _) in sets]
+
+    def unfused_steps(n):
+        for i in range(n):
+            l0 = layers0[i % len(layers0)]
+            X, Y, ws = sets0[i % len(sets0)]
+            T = Ts[i % len(Ts)]
+            M = X.shape[0]
+            l0.svdq_quant_down(X, M, X.stride(0), ws, ws.numel(), stream)
+            torch.mm(X, L1s, out=T)
+            l0.svdq_gemm_up(M, Y, Y.stride(0), ws, ws.numel(), stream)
+            Y.addmm_(T, L2)
+
+    def fused_steps(lays, sts, n):
+        for i in range(n):
+            l = lays[i % len(lays)]
+            X, Y, ws = sts[i % len(sts)]
+            M = X.shape[0]
+            l.svdq_quant_down(X, M, X.stride(0), ws, ws.numel(), stream)
+            l.svdq_gemm_up(M, Y, Y.stride(0), ws, ws.numel(), stream)
+
+    def timed(fn):
+        fn(3)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn(steps)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    t_unfused = timed(unfused_steps)
+    t_fused = timed(lambda n: fused_steps(layers, sets, n))
+    t_bare = timed(lambda n: fused_steps(layers0, sets0, n))
+    return {"ms_step": {"fused_rank": t_fused, "unfused_rank": t_unfused, "rank0": t_bare},
+            "fused_pct_of_bare_gemm": 100.0 * (t_fused - t_bare) / k2_bare_ms,
+            "unfused_pct_of_bare_gemm": 100.0 * (t_unfused - t_bare) / k2_bare_ms,
+            "fused_pct_of_bare_layer": 100.0 * (t_fused - t_bare) / t_bare,
+            "unfused_pct_of_bare_layer": 100.0 * (t_unfused - t_bare) / t_bare,
+            "comparator": "down projection X (diag(1/lambda) L1) and up projection Y += T L2 as separate cuBLAS GEMMs"}
 
 
 def run_ours(args):
@@ -418,6 +493,7 @@ def run_ours(args):
             "rank": spec.rank, "ms_rank": {"quant_down": k1_r, "gemm": k2_r},
             "ms_rank0": {"quant_down": k1_0, "gemm": k2_0},
             "pct_of_bare_gemm": 100.0 * over / k2_0, "pct_of_bare_layer": 100.0 * over / (k1_0 + k2_0)}
+        line["lowrank_overhead_unfused"] = unfused_comparator(lin, layers, sets, layers0, sets0, n_over, stream, k2_0)
         for l0 in layers0:
             l0.close()
         # End to end through the public API: pinned host X -> device, forward, Y -> pinned host.
@@ -455,6 +531,79 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """Times every FLUX-shaped layer (QKV, MLP pair, DiT block) and the M x rank sweep at K = N =
+    3072 on one GPU: one JSON line each, with the step time (both kernels, whole steps), the
+    per-kernel times, TFLOP/s over the algorithmic flops, and the low-rank overhead against the
+    same layer prepared with rank 0.  Two rotating copies of X/Y/workspace per point."""
+    import numpy as np
+    import torch
+
+    import synth
+    import w4a4_rank_corrected_smooth_b200 as S
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    S.svdq_check_device(0)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
+    names = ["flux_qkv_4608x3072x9216_r32", "flux_mlp_up_4608x3072x12288_r32", "flux_mlp_down_4608x12288x3072_r32",
+             "dit_qkv_mlp_in_16896x3072x21504_r32", "dit_out_16896x15360x3072_r32"]
+    names += [f"sweep_{M}x3072x3072_r{r}" for r in (0, 16, 32, 64, 128) for M in (256, 1024, 4096, 16384)]
+    prepared = {}
+    xcache = {}
+    for name in names:
+        if not name.startswith("sweep"):
+            xcache.clear()
+        spec = synth.get(name)
+        key = (spec.K, spec.N, spec.rank, name.split("_")[0] if name.startswith("sweep") else name)
+        if key not in prepared:
+            calib = synth.activations_bf16(spec.with_rows(min(spec.M, 4096)))
+            W = synth.weight_bf16(spec)
+            b = synth.bias_bf16(spec)
+            a = synth.act_absmax(calib)
+            for l_, l0_ in prepared.values():
+                l_.close()
+                l0_.close()
+            prepared.clear()
+            prepared[key] = (S.SVDQLinear(W, b, a, args.precision, spec.rank, device=0),
+                             S.SVDQLinear(W, b, a, args.precision, 0, device=0))
+        lin, lin0 = prepared[key]
+        xkey = spec.name.rsplit("_r", 1)[0]  # the sweep's points of one M share X
+        if xkey not in xcache:
+            xcache[xkey] = bf16_device(synth.activations_bf16(spec), dev)
+        Xd = xcache[xkey]
+        sets = []
+        for s_ in range(2):
+            Xs = Xd if s_ == 0 else Xd.roll(1, 0).contiguous()
+            sets.append((Xs, torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=dev), lin.new_workspace(spec.M)))
+        steps = max(20, min(400, int(2e12 / max(spec.flops, 1))))
+        time_loop([lin], sets, 5, stream)
+        t, k1, k2 = time_loop([lin], sets, steps, stream)
+        ms = t / steps
+        sets0 = [(x, y, lin0.new_workspace(spec.M)) for (x, y, _) in sets]
+        time_loop([lin0], sets0, 5, stream)
+        t0, k10, k20 = time_loop([lin0], sets0, steps, stream)
+        ms0 = t0 / steps
+        S.svdq_get_device_error(stream)
+        k2_flops = spec.flops_4bit + 2 * spec.M * spec.rank * spec.N
+        out = {"sweep": True, "workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "rank": spec.rank,
+               "precision": args.precision, "steps": steps, "ms_per_step": ms,
+               "tflops": spec.flops / (ms / 1e3) / 1e12,
+               "kernel_ms": {"quant_down": k1, "gemm": k2},
+               "gemm_tflops": k2_flops / (k2 / 1e3) / 1e12,
+               "gemm_frac_fp4_peak": k2_flops / (k2 / 1e3) / 1e12 / fp4_peak,
+               "ms_per_step_rank0": ms0, "kernel_ms_rank0": {"quant_down": k10, "gemm": k20},
+               "lowrank_overhead_pct_of_bare_gemm": 100.0 * (k1 + k2 - k10 - k20) / k20,
+               "peak": {"fp4_tflops": fp4_peak, "source": f"{peak_src} bf16 sustained x {FP4_PER_BF16:g}"}}
+        print(json.dumps(out), flush=True)
+        del sets, sets0
+    for l, l0 in prepared.values():
+        l.close()
+        l0.close()
+
+
 def main():
     args = parse_args()
     world, _, _ = dist_info()
@@ -462,6 +611,8 @@ def main():
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_ours(args)
 

@@ -92,6 +92,18 @@ __device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
   return r;
 }
 
+// Element-wise round-to-nearest a - b and a * b + c of fp32 pairs.
+__device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 // E2M1 codes (RNE, saturating) of the 8 values held as 4 fp32 pairs; element 2i in the low nibble.
 __device__ __forceinline__ uint32_t e2m1x8_pairs(const uint64_t (&v)[4]) {
   float a[8];
@@ -202,6 +214,9 @@ __global__ void __launch_bounds__(kQdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = has_lr ? *tmem_slot : 0u;
+  // Kernel 2 may be scheduled once every block of this grid has got here (it waits for this
+  // grid's completion before reading anything this kernel writes).
+  pdl_launch_dependents();
 
   if (warp < kQdWorkerWarps) {
     // ------------------------------------------------------------ workers
@@ -451,41 +466,54 @@ __global__ void __launch_bounds__(kQdThreads, 1)
                                                                    __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]));
         }
       }
-      if (p.splits > 1) __threadfence();  // each writer publishes its partial row at GPU scope
     }
   }
   if (has_lr && p.splits > 1) {
     // The last slice of the tile to finish sums all slices' partials in slice order
-    // (deterministic) and writes bf16 T.
+    // (deterministic) and writes bf16 T.  Publication: the CTA barrier orders every thread's
+    // partial stores before thread 0's GPU-scope fence, which is cumulative, and that fence
+    // before the counter update; the last slice fences again before reading.
     __shared__ int s_last;
-    __syncthreads();  // this CTA's partial rows are written
+    __syncthreads();
     if (threadIdx.x == 0) {
       bool ok = !aborted;
-      __threadfence();  // publish the partials before counting this slice
+      __threadfence();
       const bool last = ok && arrive_slice_counter(p.cnt + mt, p.epoch, p.splits, &ok);
+      if (last) __threadfence();
       if (!ok) *abort_flag = 1;
       s_last = last ? 1 : 0;
     }
     __syncthreads();
     if (s_last) {
-      __threadfence();
       uint8_t* tt = p.t + static_cast<size_t>(mt) * kBM * r * 2;
       const float* pt = p.part + static_cast<size_t>(mt) * p.splits * kBM * r;
+      const size_t slice = static_cast<size_t>(kBM) * r;
       const int units = kBM * r / 4;
-      for (int u = threadIdx.x; u < units; u += blockDim.x) {
-        const int row = (u * 4) / r, col = (u * 4) % r;
-        float4 acc = __ldcg(reinterpret_cast<const float4*>(pt + row * r + col));
-        for (int q = 1; q < p.splits; ++q) {
-          const float4 x = __ldcg(reinterpret_cast<const float4*>(pt + (static_cast<size_t>(q) * kBM + row) * r + col));
-          acc.x += x.x;
-          acc.y += x.y;
-          acc.z += x.z;
-          acc.w += x.w;
-        }
-        uint2 o;
-        o.x = pack_bf16x2(acc.x, acc.y);
-        o.y = pack_bf16x2(acc.z, acc.w);
-        *reinterpret_cast<uint2*>(tt + lr_offset(row, col, kBM, r)) = o;
+      // Two 4-column units per thread per round, all of a round's loads issued before the sums.
+      for (int u0 = threadIdx.x; u0 < units; u0 += 2 * blockDim.x) {
+        const int u1 = u0 + blockDim.x;
+        const bool has1 = u1 < units;
+        const int o0 = u0 * 4, o1 = (has1 ? u1 : u0) * 4;
+        float4 a0 = __ldcg(reinterpret_cast<const float4*>(pt + o0));
+        float4 a1 = __ldcg(reinterpret_cast<const float4*>(pt + o1));
+        float4 x0[7], x1[7];
+#pragma unroll
+        for (int q = 1; q < 8; ++q)
+          if (q < p.splits) {
+            x0[q - 1] = __ldcg(reinterpret_cast<const float4*>(pt + q * slice + o0));
+            x1[q - 1] = __ldcg(reinterpret_cast<const float4*>(pt + q * slice + o1));
+          }
+#pragma unroll
+        for (int q = 1; q < 8; ++q)
+          if (q < p.splits) {
+            a0.x += x0[q - 1].x; a0.y += x0[q - 1].y; a0.z += x0[q - 1].z; a0.w += x0[q - 1].w;
+            a1.x += x1[q - 1].x; a1.y += x1[q - 1].y; a1.z += x1[q - 1].z; a1.w += x1[q - 1].w;
+          }
+        *reinterpret_cast<uint2*>(tt + lr_offset(o0 / r, o0 % r, kBM, r)) =
+            make_uint2(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w));
+        if (has1)
+          *reinterpret_cast<uint2*>(tt + lr_offset(o1 / r, o1 % r, kBM, r)) =
+              make_uint2(pack_bf16x2(a1.x, a1.y), pack_bf16x2(a1.z, a1.w));
       }
       if (threadIdx.x == 0) atomicExch(p.cnt + mt, 0ull);
     }
@@ -760,6 +788,9 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
   cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Launched as a programmatic dependent of kernel 1: everything above overlapped its tail; the
+  // activation codes, scales and T are read only after it has completed.
+  pdl_wait_primary();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -1009,12 +1040,18 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
 //
 // INT4 codes with one fp32 scale per 64 elements cannot use block-scaled MMAs, so the 4-bit GEMM
 // runs on kind::i8: converter warps sign-extend the packed nibbles into int8 tiles, one 64-element
-// group at a time; the MMA warp accumulates each group's int32 partial in one of two TMEM buffers
+// group at a time; the MMA warp accumulates each group's int32 partial in one of four TMEM buffers
 // (the bf16 up projection T L2 first, as fp32); the epilogue warps keep the fp32 accumulator in
-// registers and add each partial converted exactly to fp32 and multiplied by s_x[m,g] s_w[n,g].
+// registers and add each partial converted exactly to fp32 and multiplied by s_x[m,g] s_w[n,g]
+// (packed f32x2 arithmetic).  The k-block's scales arrive by bulk copy in a ring of their own,
+// released by the epilogue once it has applied them.
 
 constexpr int kIStages = 3;                                   // packed stages
 constexpr int kIGroups = 4;                                   // int8 group buffers
+constexpr int kISlots = 4;                                    // TMEM partial buffers (128 columns each)
+constexpr int kISfStages = 4;                                 // scale stages (one k-block each)
+constexpr uint32_t kISfA = kBM * 4 * 4;                       // 2 KB: fp32 [128 rows][4 groups]
+constexpr uint32_t kISfB = 4 * kBN * 4;                       // 4 KB: fp32 [4 groups][256 rows]
 constexpr int kIBN = 128;                                     // output columns per tile
 constexpr int kIConvWarps = 4;
 constexpr int kIEpiWarps = 8;
@@ -1056,14 +1093,17 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* packed = smem;                                  // kIStages x 32 KB
   uint8_t* groups = packed + kIStages * kIPack;            // kIGroups x 16 KB
-  uint8_t* staging = groups + kIGroups * kIGrp;
+  uint8_t* sfring = groups + kIGroups * kIGrp;              // kISfStages x 6 KB
+  uint8_t* staging = sfring + kISfStages * (kISfA + kISfB);
   uint64_t* pfull = reinterpret_cast<uint64_t*>(staging + kIStaging);
   uint64_t* pempty = pfull + kIStages;
   uint64_t* gfull = pempty + kIStages;
   uint64_t* gempty = gfull + kIGroups;
   uint64_t* tfull = gempty + kIGroups;
-  uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* tempty = tfull + kISlots;
+  uint64_t* sfull = tempty + kISlots;
+  uint64_t* sempty = sfull + kISfStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + kISfStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1082,15 +1122,19 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
       mbar_init(&gfull[s], kIConvWarps);
       mbar_init(&gempty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kISlots; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], kIEpiWarps);
+    }
+    for (int b = 0; b < kISfStages; ++b) {
+      mbar_init(&sfull[b], 1);
+      mbar_init(&sempty[b], kIEpiWarps);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, kISlots * kIBN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -1103,8 +1147,11 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
       // ------------------------------------------------------------ producer
       int st = 0;
       uint32_t ph = 0;
-      int issued_phase[kIStages];
+      int issued_phase[kIStages], sf_issued_phase[kISfStages];
       for (int s = 0; s < kIStages; ++s) issued_phase[s] = -1;
+      for (int s = 0; s < kISfStages; ++s) sf_issued_phase[s] = -1;
+      int ss = 0;
+      uint32_t sph = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
         const int mt = tile / p.NT, n128 = tile % p.NT, n256 = n128 >> 1, nh = n128 & 1;
@@ -1125,6 +1172,20 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
                      bytes, &pfull[st]);
           } else {
             const int kb = j - nlr;
+            // the k-block's scales: A [128 rows][4 groups], B [4 groups][256 rows] (both halves)
+            if (*abort_flag || !wait_parity_bounded(&sempty[ss], sph ^ 1u, kErrWaitGemm)) {
+              ok = false;
+              break;
+            }
+            uint8_t* sfb = sfring + ss * (kISfA + kISfB);
+            mbar_arrive_expect_tx(&sfull[ss], kISfA + kISfB);
+            bulk_g2s(sfb, p.a_sf + (static_cast<size_t>(mt) * p.KB + kb) * (kBM * 4), kISfA, &sfull[ss]);
+            bulk_g2s(sfb + kISfA, p.b_sf + (static_cast<size_t>(n256) * p.KB + kb) * (kBN * 4), kISfB, &sfull[ss]);
+            sf_issued_phase[ss] = static_cast<int>(sph);
+            if (++ss == kISfStages) {
+              ss = 0;
+              sph ^= 1u;
+            }
             mbar_arrive_expect_tx(&pfull[st], kIPack);
             bulk_g2s(sb, p.a_codes + codes_chunk_offset(mt, kb, p.KB, kBM), kIPackA, &pfull[st]);
             bulk_g2s(sb + kIPackA, p.b_codes + codes_chunk_offset(n256, kb, p.KB, kBN) + nh * kIPackB, kIPackB, &pfull[st]);
@@ -1140,6 +1201,9 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
         *abort_flag = 1;
         for (int s = 0; s < kIStages; ++s)
           if (issued_phase[s] >= 0) wait_parity_bounded(&pfull[s], static_cast<uint32_t>(issued_phase[s]), kErrWaitGemm);
+        for (int s = 0; s < kISfStages; ++s)
+          if (sf_issued_phase[s] >= 0)
+            wait_parity_bounded(&sfull[s], static_cast<uint32_t>(sf_issued_phase[s]), kErrWaitGemm);
       }
     }
   } else if (warp == 1) {
@@ -1151,10 +1215,10 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
       uint32_t ph = 0, gph = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-        // low-rank slot: T L2 in fp32 into TMEM buffer (slot & 1)
+        // low-rank slot: T L2 in fp32 into TMEM buffer (slot % kISlots)
         for (int j = 0; j < nlr && ok; ++j) {
-          const uint32_t b = slot & 1;
-          if (j == 0 && (*abort_flag || !wait_parity_bounded(&tempty[b], ((slot >> 1) & 1) ^ 1u, kErrWaitGemm))) {
+          const uint32_t b = slot % kISlots;
+          if (j == 0 && (*abort_flag || !wait_parity_bounded(&tempty[b], ((slot / kISlots) & 1) ^ 1u, kErrWaitGemm))) {
             ok = false;
             break;
           }
@@ -1181,8 +1245,8 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
         }
         // one slot per 64-element group
         for (int g = 0; g < ngrp && ok; ++g) {
-          const uint32_t b = slot & 1;
-          if (*abort_flag || !wait_parity_bounded(&tempty[b], ((slot >> 1) & 1) ^ 1u, kErrWaitGemm) ||
+          const uint32_t b = slot % kISlots;
+          if (*abort_flag || !wait_parity_bounded(&tempty[b], ((slot / kISlots) & 1) ^ 1u, kErrWaitGemm) ||
               !wait_parity_bounded(&gfull[gs], gph, kErrWaitGemm)) {
             ok = false;
             break;
@@ -1272,32 +1336,36 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
     const int q = warp & 3, h = ew >> 2;  // TMEM lane quadrant this warp may access (warp % 4), column half
     const int rloc = q * 32 + lane;
     uint8_t* srow = staging + rloc * kIStagePitch + h * 128;
-    int slot = 0;
+    // |partial| <= 64*8*8: adding 1.5*2^23 as an integer and subtracting it as a float is exact
+    const uint64_t magic2 = f2pack(12582912.0f, 12582912.0f);
+    int slot = 0, ss = 0;
+    uint32_t sph = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-      const int mt = tile / p.NT, n128 = tile % p.NT, n256 = n128 >> 1, nh = n128 & 1;
-      float acc[64];
+      const int mt = tile / p.NT, n128 = tile % p.NT, nh = n128 & 1;
+      uint64_t acc[32];  // this thread's 64 fp32 accumulators as pairs
 #pragma unroll
-      for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
+      for (int c = 0; c < 32; ++c) acc[c] = 0ull;
       const int nslots = (nlr > 0 ? 1 : 0) + ngrp;
       for (int si = 0; si < nslots; ++si) {
-        const uint32_t b = slot & 1;
+        const uint32_t b = slot % kISlots;
+        const bool lr = nlr > 0 && si == 0;
+        const int g = lr ? 0 : si - (nlr > 0 ? 1 : 0);
+        const int gi = g & 3;
         bool w = true;
-        if (lane == 0) w = !*abort_flag && wait_parity_bounded(&tfull[b], (slot >> 1) & 1, kErrWaitGemm);
+        if (lane == 0) {
+          w = !*abort_flag && wait_parity_bounded(&tfull[b], (slot / kISlots) & 1, kErrWaitGemm);
+          if (w && !lr && gi == 0) w = wait_parity_bounded(&sfull[ss], sph, kErrWaitGemm);
+        }
         if (!__shfl_sync(0xffffffffu, w, 0)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const bool lr = nlr > 0 && si == 0;
-        const int g = lr ? 0 : si - (nlr > 0 ? 1 : 0);
-        float sx = 0.0f;
-        const float* swp = nullptr;
-        if (!lr) {
-          const int kb = g >> 2, gi = g & 3;
-          sx = p.a_sf[(static_cast<size_t>(mt) * p.KB + kb) * (kBM * 4) + rloc * 4 + gi];
-          swp = p.b_sf + (static_cast<size_t>(n256) * p.KB + kb) * (kBN * 4) + gi * kBN + nh * kIBN + h * 64;
-        }
+        const uint8_t* sfb = sfring + ss * (kISfA + kISfB);
+        const float sx = lr ? 0.0f : reinterpret_cast<const float*>(sfb)[rloc * 4 + gi];
+        const float* swp = reinterpret_cast<const float*>(sfb + kISfA) + gi * kBN + nh * kIBN + h * 64;
+        const uint64_t sx2 = f2pack(sx, sx);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t v[32];
@@ -1305,24 +1373,29 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
           tmem_wait_ld();
           if (lr) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) acc[half * 32 + c] = __uint_as_float(v[c]);
+            for (int c = 0; c < 16; ++c) acc[half * 16 + c] = f2pack(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1]));
           } else {
 #pragma unroll
             for (int c = 0; c < 32; c += 4) {
-              const float4 sw = __ldg(reinterpret_cast<const float4*>(swp + half * 32 + c));
-              const float swv[4] = {sw.x, sw.y, sw.z, sw.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                // |partial| <= 64*8*8: adding 1.5*2^23 as an integer and subtracting it as a float is exact
-                const float f = __uint_as_float(v[c + e] + 0x4B400000u) - 12582912.0f;
-                acc[half * 32 + c + e] = fmaf(f, sx * swv[e], acc[half * 32 + c + e]);
-              }
+              const float4 sw = *reinterpret_cast<const float4*>(swp + half * 32 + c);  // same for all lanes
+              const uint64_t c01 = f2mul(sx2, f2pack(sw.x, sw.y)), c23 = f2mul(sx2, f2pack(sw.z, sw.w));
+              const uint64_t f01 = f2sub(f2pack(__uint_as_float(v[c] + 0x4B400000u), __uint_as_float(v[c + 1] + 0x4B400000u)), magic2);
+              const uint64_t f23 = f2sub(f2pack(__uint_as_float(v[c + 2] + 0x4B400000u), __uint_as_float(v[c + 3] + 0x4B400000u)), magic2);
+              acc[half * 16 + c / 2] = f2fma(f01, c01, acc[half * 16 + c / 2]);
+              acc[half * 16 + c / 2 + 1] = f2fma(f23, c23, acc[half * 16 + c / 2 + 1]);
             }
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[b]);
+        if (lane == 0) {
+          mbar_arrive(&tempty[b]);
+          if (!lr && gi == 3) mbar_arrive(&sempty[ss]);  // the k-block's scales are applied
+        }
+        if (!lr && gi == 3 && ++ss == kISfStages) {
+          ss = 0;
+          sph ^= 1u;
+        }
         ++slot;
       }
       if (!ok) break;
@@ -1335,10 +1408,13 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
         const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8));
         const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8 + 4));
         uint4 o;
-        o.x = pack_bf16x2(acc[u * 8 + 0] + b0.x, acc[u * 8 + 1] + b0.y);
-        o.y = pack_bf16x2(acc[u * 8 + 2] + b0.z, acc[u * 8 + 3] + b0.w);
-        o.z = pack_bf16x2(acc[u * 8 + 4] + b1.x, acc[u * 8 + 5] + b1.y);
-        o.w = pack_bf16x2(acc[u * 8 + 6] + b1.z, acc[u * 8 + 7] + b1.w);
+        float a[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) f2unpack(acc[u * 4 + k], a[2 * k], a[2 * k + 1]);
+        o.x = pack_bf16x2(a[0] + b0.x, a[1] + b0.y);
+        o.y = pack_bf16x2(a[2] + b0.z, a[3] + b0.w);
+        o.z = pack_bf16x2(a[4] + b1.x, a[5] + b1.y);
+        o.w = pack_bf16x2(a[6] + b1.z, a[7] + b1.w);
         *reinterpret_cast<uint4*>(srow + 16 * u) = o;
       }
       fence_proxy_async_smem();
@@ -1361,12 +1437,12 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
     }
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, kISlots * kIBN);
   }
 }
 
 static size_t gemm_int4_smem_bytes() {
-  return 1024 + kIStages * kIPack + kIGroups * kIGrp + kIStaging + 256;
+  return 1024 + kIStages * kIPack + kIGroups * kIGrp + kISfStages * (kISfA + kISfB) + kIStaging + 256;
 }
 
 static cudaError_t launch_gemm_int4(const GemmArgs& a, int num_sms, cudaStream_t stream) {
@@ -1445,13 +1521,15 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   cfg.blockDim = dim3(kGThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, maps, p);
 }
 

@@ -83,6 +83,15 @@ __device__ __forceinline__ bool wait_parity_bounded(uint64_t* bar, uint32_t pari
   }
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Lets the next kernel in the stream (launched with programmatic stream serialization) start its
+// prologue once every block of this grid has executed this or exited.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Blocks until the grid this one depends on has completed and its memory is visible (no-op
+// without such a dependency).
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ async proxy / bulk copies
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
