@@ -1055,6 +1055,7 @@ constexpr uint32_t kISfB = 4 * kBN * 4;                       // 4 KB: fp32 [4 g
 constexpr int kIBN = 128;                                     // output columns per tile
 constexpr int kIConvWarps = 4;
 constexpr int kIEpiWarps = 8;
+constexpr int kIEpiCols = kIBN / (kIEpiWarps / 4);             // 64 accumulator columns per epilogue thread
 constexpr int kIThreads = (2 + kIConvWarps + kIEpiWarps) * 32;
 constexpr uint32_t kIPackA = kBM * kRowBytes;                 // 16 KB
 constexpr uint32_t kIPackB = kIBN * kRowBytes;                // 16 KB
@@ -1081,10 +1082,15 @@ __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Four 4-bit two's-complement values, one per byte (0..15), sign-extended to int8 in place: a byte
+// with bit 3 set gets 0xF0 ORed in; (x & 0x08080808) * 0x1E puts exactly 0xF0 in those bytes (8 *
+// 0x1E = 0xF0 < 0x100, so no carry crosses a byte).
+__device__ __forceinline__ uint32_t sext_nibbles4(uint32_t x) { return x | ((x & 0x08080808u) * 0x1Eu); }
+
 // 8 packed int4 codes (4 bytes, element 2i in the low nibble) -> 8 int8 in element order.
 __device__ __forceinline__ uint2 unpack_int4x8(uint32_t w) {
-  const uint32_t lo = __vsub4((w & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);         // elements 0,2,4,6
-  const uint32_t hi = __vsub4(((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);  // elements 1,3,5,7
+  const uint32_t lo = sext_nibbles4(w & 0x0F0F0F0Fu);          // elements 0,2,4,6
+  const uint32_t hi = sext_nibbles4((w >> 4) & 0x0F0F0F0Fu);   // elements 1,3,5,7
   return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
 }
 
@@ -1333,9 +1339,9 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
   } else {
     // ------------------------------------------------------------ rescale + epilogue (8 warps)
     const int ew = warp - 2 - kIConvWarps;
-    const int q = warp & 3, h = ew >> 2;  // TMEM lane quadrant this warp may access (warp % 4), column half
+    const int q = warp & 3, cg = ew >> 2;  // TMEM lane quadrant this warp may access (warp % 4), column group
     const int rloc = q * 32 + lane;
-    uint8_t* srow = staging + rloc * kIStagePitch + h * 128;
+    uint8_t* srow = staging + rloc * kIStagePitch + cg * kIEpiCols * 2;
     // |partial| <= 64*8*8: adding 1.5*2^23 as an integer and subtracting it as a float is exact
     const uint64_t magic2 = f2pack(12582912.0f, 12582912.0f);
     int slot = 0, ss = 0;
@@ -1343,9 +1349,9 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
     bool ok = true;
     for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
       const int mt = tile / p.NT, n128 = tile % p.NT, nh = n128 & 1;
-      uint64_t acc[32];  // this thread's 64 fp32 accumulators as pairs
+      uint64_t acc[kIEpiCols / 2];  // this thread's fp32 accumulators as pairs
 #pragma unroll
-      for (int c = 0; c < 32; ++c) acc[c] = 0ull;
+      for (int c = 0; c < kIEpiCols / 2; ++c) acc[c] = 0ull;
       const int nslots = (nlr > 0 ? 1 : 0) + ngrp;
       for (int si = 0; si < nslots; ++si) {
         const uint32_t b = slot % kISlots;
@@ -1364,12 +1370,12 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
         tc_fence_after();
         const uint8_t* sfb = sfring + ss * (kISfA + kISfB);
         const float sx = lr ? 0.0f : reinterpret_cast<const float*>(sfb)[rloc * 4 + gi];
-        const float* swp = reinterpret_cast<const float*>(sfb + kISfA) + gi * kBN + nh * kIBN + h * 64;
+        const float* swp = reinterpret_cast<const float*>(sfb + kISfA) + gi * kBN + nh * kIBN + cg * kIEpiCols;
         const uint64_t sx2 = f2pack(sx, sx);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int half = 0; half < kIEpiCols / 32; ++half) {
           uint32_t v[32];
-          tmem_ld32(tmem + b * kIBN + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * 64 + half * 32), v);
+          tmem_ld32(tmem + b * kIBN + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(cg * kIEpiCols + half * 32), v);
           tmem_wait_ld();
           if (lr) {
 #pragma unroll
@@ -1401,10 +1407,10 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
       if (!ok) break;
       // bias, bf16, stage, one bulk store per row segment
       const int row = mt * kBM + rloc;
-      const int n0 = n128 * kIBN + h * 64;
+      const int n0 = n128 * kIBN + cg * kIEpiCols;
       bulk_wait_read0();
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < kIEpiCols / 8; ++u) {
         const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8));
         const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8 + 4));
         uint4 o;
@@ -1419,7 +1425,7 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
       }
       fence_proxy_async_smem();
       if (row < p.M && n0 < p.N) {
-        const int ncols = (p.N - n0) < 64 ? (p.N - n0) : 64;
+        const int ncols = (p.N - n0) < kIEpiCols ? (p.N - n0) : kIEpiCols;
         bulk_s2g(p.Y + static_cast<size_t>(row) * p.ldy + n0, smem_u32(srow), static_cast<uint32_t>(ncols) * 2u);
       }
       bulk_commit();
