@@ -1,0 +1,90 @@
+"""Kernel 1's K split: the per-tile arrival counters and the last-slice reduction of T.
+
+When kernel 1 splits K, every slice writes an fp32 partial of T into the workspace and counts
+itself in a per-tile counter tagged with the launch; the last slice sums the partials in slice
+order.  These tests check that the result needs no initialised workspace (garbage counters),
+that reusing a workspace gives bit-identical results, and that a CUDA-graph replay of the same
+launches (the same launch tag every time) does too.
+"""
+import numpy as np
+import pytest
+
+import synth
+from oracle import svdq_oracle as O
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import w4a4_rank_corrected_smooth_b200 as S  # noqa: E402
+
+
+def _bf16_dev(x_bits):
+    return torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _layer(M=512, K=3072, N=512, r=32, seed=41):
+    # M = 512 rows -> 4 row tiles, K = 3072 -> 12 k-blocks: the split is 8 slices per tile on a B200
+    spec = synth.custom("ksplit", M=M, K=K, N=N, rank=r, seed=seed)
+    X = synth.activations_bf16(spec)
+    lin = S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(X), "nvfp4", r)
+    return spec, X, lin
+
+
+def _check_T(lin, X, act):
+    ops = lin.export_weights()
+    xh, cx, sx = O.quantize_activations(X, ops["inv_lambda"], "nvfp4")
+    assert np.array_equal(act["codes_x"], cx) and np.array_equal(act["scales_x"], sx)
+    T_ref = O.bf16_to_f32(O.lowrank_down(xh, ops["L1"])).astype(np.float64)
+    T_gpu = O.bf16_to_f32(act["T"]).astype(np.float64)
+    # fp32 accumulation in slice order vs the exact sum, both rounded to bf16: within 1 bf16 ulp
+    assert np.max(np.abs(T_gpu - T_ref)) <= 2 ** -7 * np.max(np.abs(T_ref))
+    assert O.rel_fro(T_gpu, T_ref) < 4e-3
+
+
+def test_split_reduction_needs_no_initialised_workspace_and_repeats_bit_exactly():
+    spec, X, lin = _layer()
+    Xd = _bf16_dev(X)
+    ws = lin.new_workspace(spec.M)
+    ws.fill_(0xFF)  # every counter starts as garbage
+    lin.svdq_quant_down(Xd, spec.M, spec.K, ws, ws.numel())
+    S.svdq_get_device_error()
+    first = lin.svdq_export_activations(ws, spec.M)
+    _check_T(lin, X, first)
+    for _ in range(2):  # the counters were reset by the last slice; the next launches start clean
+        lin.svdq_quant_down(Xd, spec.M, spec.K, ws, ws.numel())
+        S.svdq_get_device_error()
+        again = lin.svdq_export_activations(ws, spec.M)
+        for k in first:
+            assert np.array_equal(first[k], again[k]), k
+    lin.close()
+
+
+def test_graph_replay_of_the_forward_is_bit_identical_to_eager():
+    spec, X, lin = _layer(M=1000, seed=43)
+    Xd = _bf16_dev(X)
+    ws = lin.new_workspace(spec.M)
+    Y_eager = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device="cuda")
+    lin.svdq_linear_forward(Xd, spec.M, spec.K, Y_eager, spec.N, ws, ws.numel())
+    torch.cuda.synchronize()
+    S.svdq_get_device_error()
+    Y = torch.full((spec.M, spec.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm the launch path once outside the capture
+        lin.svdq_linear_forward(Xd, spec.M, spec.K, Y, spec.N, ws, ws.numel(), side)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        lin.svdq_linear_forward(Xd, spec.M, spec.K, Y, spec.N, ws, ws.numel())
+    for _ in range(3):  # the same launch tag on every replay
+        Y.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        S.svdq_get_device_error()
+        assert torch.equal(Y.view(torch.int16), Y_eager.view(torch.int16))
+    del g
+    lin.close()
