@@ -229,9 +229,15 @@ __global__ void __launch_bounds__(kQdThreads, 1)
       // group t % 4 (two swizzled 16-byte units; the quarter-warps' loads hit distinct banks).
       const int row = warp * 8 + (lane >> 2), g = lane & 3;
       const float kInv6 = __frcp_rn(6.0f);
+      // Per-thread constants: the two swizzled 16-byte units of the group inside a stage, and
+      // this row's code/scale positions inside a (tile, k-block) chunk.
+      const uint32_t off0 = swz128(row, g * 32), off1 = swz128(row, g * 32 + 16);
+      uint8_t* const codes_tile = p.codes + codes_chunk_offset(mt, 0, p.KB, kBM);
+      uint8_t* const sf_tile = p.sf + sf_chunk_offset(mt, 0, p.KB, kBM) + (row & 31) * 16 + (row >> 5) * 4 + g;
+      int st = 0;
+      uint32_t ph = 0;
       for (int c = 0; c < nch; ++c) {
-        const int st = c % NS;
-        const bool ok = !*abort_flag && wait_parity_bounded(&full[st], (c / NS) & 1, kErrWaitQuantDown);
+        const bool ok = !*abort_flag && wait_parity_bounded(&full[st], ph, kErrWaitQuantDown);
         if (!__all_sync(0xffffffffu, ok)) {
           *abort_flag = 1;
           break;
@@ -240,12 +246,12 @@ __global__ void __launch_bounds__(kQdThreads, 1)
         const int kb = gc >> 2, cc = gc & 3;
         const float4* ilv = reinterpret_cast<const float4*>(ils + st * 64 + g * 16);
         uint8_t* xt = xs + st * kXsBytes;
-        uint4* cell0 = reinterpret_cast<uint4*>(xt + swz128(row, g * 32));
-        uint4* cell1 = reinterpret_cast<uint4*>(xt + swz128(row, g * 32 + 16));
+        uint4* cell0 = reinterpret_cast<uint4*>(xt + off0);
+        uint4* cell1 = reinterpret_cast<uint4*>(xt + off1);
         const uint4 xa = *cell0, xb = *cell1;
         const uint32_t w[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
         uint64_t xp[2][4];  // x_hat as fp32 pairs: element 2t, 2t + 1 of half h in xp[h][t]
-        float amax = 0.0f;
+        float pm[8];        // per-pair maxima of |x_hat|, reduced as a tree (max is exact)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const float4 i0 = ilv[2 * h], i1 = ilv[2 * h + 1];
@@ -258,9 +264,11 @@ __global__ void __launch_bounds__(kQdThreads, 1)
                              f2pack(il[2 * t], il[2 * t + 1]));
             float lo, hi;
             f2unpack(xp[h][t], lo, hi);
-            amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+            pm[4 * h + t] = fmaxf(fabsf(lo), fabsf(hi));
           }
         }
+        const float amax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
         // scale code: UE4M3_rne(RN(amax / 6)), bracketed the same way
         const float s_est = __fmul_rn(amax, kInv6);
         uint32_t sbits = cvt_e4m3(__fmul_rn(s_est, kNudgeLo));
@@ -285,9 +293,8 @@ __global__ void __launch_bounds__(kQdThreads, 1)
           code.x = sd != 0.0f ? e2m1x8_div(xh[0], sd) : 0u;
           code.y = sd != 0.0f ? e2m1x8_div(xh[1], sd) : 0u;
         }
-        *reinterpret_cast<uint2*>(p.codes + codes_chunk_offset(mt, kb, p.KB, kBM) + swz128(row, cc * 32 + g * 8)) = code;
-        p.sf[sf_chunk_offset(mt, kb, p.KB, kBM) + cc * 512 + (row & 31) * 16 + (row >> 5) * 4 + g] =
-            static_cast<uint8_t>(sbits);
+        *reinterpret_cast<uint2*>(codes_tile + static_cast<size_t>(kb) * (kBM * kRowBytes) + swz128(row, cc * 32 + g * 8)) = code;
+        sf_tile[static_cast<size_t>(kb) * (kBM * kSfBytesPerRowKb) + cc * 512] = static_cast<uint8_t>(sbits);
         if (has_lr) {
           uint32_t hv[8];
 #pragma unroll
@@ -304,6 +311,10 @@ __global__ void __launch_bounds__(kQdThreads, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(has_lr ? &xready[st] : &empty[st]);
+        if (++st == NS) {
+          st = 0;
+          ph ^= 1u;
+        }
       }
     } else {
       // INT4: lane (sub, kg) of warp w handles 8 consecutive columns (16-byte unit kg) of rows
@@ -651,6 +662,7 @@ constexpr uint32_t kGSfb = kBN * kSfBytesPerRowKb;          // 4 KB of B scales 
 constexpr uint32_t kGStage = kGA + kGB + kGSfa + kGSfb;     // 38 KB
 constexpr uint32_t kGOutBox = 32 * 128;                     // staging box: 32 rows x 64 bf16, 128-byte swizzle
 constexpr uint32_t kGStaging = kGEpiWarps * kGOutBox;       // 32 KB: one box per epilogue warp
+constexpr uint32_t kGLrL2Offset = 16384;                    // L2 half in staging (T before it; rank <= 64)
 constexpr uint32_t kTmemCols = 512;
 // Per-stage scale buffer: 12 blocks of 4 columns (SFA k-steps 0..3, then SFB k-steps 0..3 with
 // two 128-row blocks each), in the order of the 12 blocks of 512 B of the global scale layout.
@@ -704,6 +716,16 @@ __device__ __forceinline__ void mma2_nvfp4(uint32_t d, uint64_t ad, uint64_t bd,
       "l"(ad), "l"(bd), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
       : "memory");
 }
+// 2-D tensor copy of this CTA's box into its own shared memory; completion is counted on the
+// barrier at cluster address `bar` (the leader CTA's barrier for both CTAs of the pair).
+__device__ __forceinline__ void tma_rows_cg2(void* smem_dst, const CUtensorMap* map, int row, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row), "r"(bar)
+      : "memory");
+}
+
 // Arrive on a barrier given by cluster address (possibly the peer CTA's).  Default (CTA-scope
 // release) semantics: what the arrival publishes is TMEM state, ordered by the tcgen05 wait and
 // fence that precede it, so no cluster-scope memory fence is needed (and it would stall the
@@ -757,7 +779,9 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
   uint64_t* ready = empty + kGStages;       // (leader) both CTAs' tiles landed and scales written
   uint64_t* acc_full = ready + kGStages;    // (both) accumulator ready
   uint64_t* acc_empty = acc_full + 1;       // (leader) both CTAs drained the accumulator
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  uint64_t* lr_full = acc_empty + 1;        // (leader) both CTAs' low-rank operands landed in staging
+  uint64_t* stg_free = lr_full + 1;         // (both) the epilogue's stores finished reading staging
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stg_free + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -767,7 +791,13 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
   const int r = p.rank;
   const int nlr = (r + kLrChunk - 1) / kLrChunk;
   const int tiles = p.MT2 * p.NT;
-  const int nstages_tile = nlr + p.KB;
+  // Up to rank 64 the low-rank operands (T and this CTA's half of L2: 512 r bytes) fit in the
+  // epilogue's staging, which is idle during a tile's k-loop: they are loaded there once the
+  // previous tile's stores have read it, and their MMAs close the tile.  Larger ranks take
+  // ring stages before the k-blocks.
+  const bool lr_in_staging = r > 0 && r <= 64;
+  const int nlr_ring = lr_in_staging ? 0 : nlr;
+  const int nstages_tile = nlr_ring + p.KB;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGStages; ++s) {
@@ -777,6 +807,8 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kGEpiWarps);
+    mbar_init(lr_full, 1);
+    mbar_init(stg_free, kGEpiWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -807,7 +839,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
             break;
           }
           uint8_t* sb = smem + st * kGStage;
-          if (j < nlr) {
+          if (j < nlr_ring) {
             const uint32_t cw = lr_chunk_width(r, j);
             const uint32_t tb = kBM * cw * 2, lb = (kBN / 2) * cw * 2;
             mbar_arrive_expect_tx(&full[st], tb + lb);
@@ -816,7 +848,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
             for (uint32_t q = 0; q < tb / 4096; ++q) tma_load_2d(sb + 4096 * q, &maps.t, 0, trow + 16 * q, &full[st]);
             for (uint32_t q = 0; q < lb / 4096; ++q) tma_load_2d(sb + kGA + 4096 * q, &maps.l2, 0, lrow + 16 * q, &full[st]);
           } else {
-            const int kb = j - nlr;
+            const int kb = j - nlr_ring;
             mbar_arrive_expect_tx(&full[st], kGStage);
             tma_load_2d(sb, &maps.a, 0, static_cast<int>(codes_chunk_offset(mt, kb, p.KB, kBM) / 256), &full[st]);
             tma_load_2d(sb + kGA, &maps.b, 0, static_cast<int>((codes_chunk_offset(nt, kb, p.KB, kBN) + rank * kGB) / 256),
@@ -842,12 +874,12 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
         const int m2 = tile / p.NT, nt = tile % p.NT;
         const int mt = 2 * m2 + static_cast<int>(rank);
         for (int j = 0; j < nstages_tile; ++j) {
-          if (j >= nlr) {
+          if (j >= nlr_ring) {
             if (*abort_flag || !wait_parity_bounded(&empty[st], ph ^ 1u, kErrWaitGemm)) {
               ok = false;
               break;
             }
-            const int kb = j - nlr;
+            const int kb = j - nlr_ring;
             uint8_t* sb = smem + st * kGStage;
             tma_load_2d(sb + kGA + kGB, &maps.sfa, 0, static_cast<int>(sf_chunk_offset(mt, kb, p.KB, kBM) / 256), &full[st]);
             tma_load_2d(sb + kGA + kGB + kGSfa, &maps.sfb, 0, static_cast<int>(sf_chunk_offset(nt, kb, p.KB, kBN) / 256),
@@ -884,7 +916,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
           }
           tc_fence_after();
           const uint32_t sb = smem_u32(smem + st * kGStage);
-          if (j < nlr) {
+          if (j < nlr_ring) {
             const uint32_t cw = lr_chunk_width(r, j);
             const uint64_t ad = smem_desc(sb, 128, cw * 16, kLayoutNone);
             const uint64_t bd = smem_desc(sb + kGA, 128, cw * 16, kLayoutNone);
@@ -909,6 +941,17 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
           }
         }
         if (!ok) break;
+        if (lr_in_staging) {
+          if (*abort_flag || !wait_parity_bounded(lr_full, static_cast<uint32_t>(local) & 1u, kErrWaitGemm)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sg = smem_u32(staging);
+          const uint64_t ad = smem_desc(sg, 128, static_cast<uint32_t>(r) * 16, kLayoutNone);
+          const uint64_t bd = smem_desc(sg + kGLrL2Offset, 128, static_cast<uint32_t>(r) * 16, kLayoutNone);
+          for (int ks = 0; ks < r / 16; ++ks) mma2_bf16(tmem, ad + 16 * ks, bd + 16 * ks, id_lr, 1u);
+        }
         tc_commit2_both(smem_u32(acc_full));
       }
       if (!ok) {
@@ -933,7 +976,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
           ok = false;
           break;
         }
-        if (j >= nlr) {
+        if (j >= nlr_ring) {
           tc_fence_after();  // the MMAs that last read this buffer completed before the stage refilled
           const uint8_t* src = smem + st * kGStage + kGA + kGB + 16 * lane;
           uint32_t v[3][16];
@@ -970,6 +1013,22 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
     uint8_t* box = staging + (warp - kGFirstEpiWarp) * kGOutBox;
     const uint32_t lrow = static_cast<uint32_t>(lane) * 128u;
+    const bool lr_issuer = lr_in_staging && warp == kGFirstEpiWarp && lane == 0;
+    const uint32_t lr_full_leader = mapa_shared(smem_u32(lr_full), 0);
+    // This CTA's T rows and half of L2 for `tile`, into staging (T at 0, L2 at kGLrL2Offset),
+    // completing on the leader's lr_full, which the leader arms with both CTAs' bytes.
+    auto issue_lr = [&](int tile) {
+      const int m2 = tile / p.NT, nt = tile % p.NT;
+      const int mt = 2 * m2 + static_cast<int>(rank);
+      const uint32_t tb = kBM * static_cast<uint32_t>(r) * 2, lb = (kBN / 2) * static_cast<uint32_t>(r) * 2;
+      if (leader) mbar_arrive_expect_tx(lr_full, 2 * (tb + lb));
+      const int trow = static_cast<int>(static_cast<size_t>(mt) * kBM * r * 2 / 256);
+      const int lrow = static_cast<int>((static_cast<size_t>(nt) * kBN * r * 2 + rank * lb) / 256);
+      for (uint32_t q = 0; q < tb / 4096; ++q) tma_rows_cg2(staging + 4096 * q, &maps.t, trow + 16 * q, lr_full_leader);
+      for (uint32_t q = 0; q < lb / 4096; ++q)
+        tma_rows_cg2(staging + kGLrL2Offset + 4096 * q, &maps.l2, lrow + 16 * q, lr_full_leader);
+    };
+    if (lr_issuer && pair < tiles) issue_lr(pair);
     int local = 0;
     for (int tile = pair; tile < tiles; tile += npairs, ++local) {
       if (!warp_wait(acc_full, static_cast<uint32_t>(local) & 1u, abort_flag)) {
@@ -1016,6 +1075,19 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
         if (lane == 0) {
           if (row0 < p.M && n0 + 64 * bx < p.N) tma_store_2d(&maps.y, smem_u32(box), n0 + 64 * bx, row0);
           bulk_commit();
+        }
+      }
+      if (lr_in_staging && tile + npairs < tiles) {
+        // staging is about to receive the next tile's low-rank operands
+        bulk_wait_read0();  // (lane 0's groups)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(stg_free);
+        if (lr_issuer) {
+          if (*abort_flag || !wait_parity_bounded(stg_free, static_cast<uint32_t>(local) & 1u, kErrWaitGemm)) {
+            *abort_flag = 1;
+            break;
+          }
+          issue_lr(tile + npairs);
         }
       }
     }
