@@ -62,8 +62,20 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    with open(KERNEL_SOURCE, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+    """sha256 of the kernel source's code: comments, trailing blanks and blank lines removed, so a
+    comment edit does not orphan the ncu counters while any change to the code does."""
+    import re
+
+    with open(KERNEL_SOURCE, encoding="utf-8") as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = []
+    for line in text.splitlines():
+        code = re.sub(r"//.*$", "", line) if '"' not in line else line  # keep lines with strings intact
+        code = code.rstrip()
+        if code:
+            lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
 
 
 def stored_traffic(kernel: str, workload: str):

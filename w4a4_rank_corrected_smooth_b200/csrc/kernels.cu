@@ -648,6 +648,10 @@ static cudaError_t make_rows_map(CUtensorMap* map, const void* base, uint64_t by
 //     one commit multicast to empty[s] of both CTAs;
 //   epilogue (8 warps per CTA): drain the accumulator, add the bias, round to bf16 into a 128-byte
 //     swizzled staging box and write it with a TMA tensor store, twice per warp.
+// The up projection T L2 (r/16 bf16 MMAs into the same accumulator): up to rank 64 its operands are
+// loaded into the staging buffer, which the epilogue does not use during a tile's k-loop, once the
+// previous tile's stores have read it, and their MMAs close the tile; larger ranks take ring
+// stages before the k-blocks.  Kernel 2 is launched as a programmatic dependent of kernel 1.
 
 constexpr int kGStages = 5;
 constexpr int kGSfWarps = 4;
