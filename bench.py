@@ -345,6 +345,62 @@ def time_loop(layers, sets, steps, stream, sample_every: int = 8):
     return total, k1, k2
 
 
+def e2e_pipelined(lin, X, spec, sets, stream, steps: int = 30):
+    """Per-step time of host X -> forward -> host Y through svdq_linear_forward, pipelined over a
+    copy-in stream, the compute stream and a copy-out stream with two device buffer sets (events
+    order the reuse of each buffer).  Returns (ms per step, steps, H2D bytes, D2H bytes)."""
+    import numpy as np
+    import torch
+
+    Xh = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Yh = [torch.empty((spec.M, spec.N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    bufs = [sets[0]]
+    if len(sets) > 1:
+        bufs.append(sets[1])
+    else:
+        X0, Y0, w0 = sets[0]
+        bufs.append((torch.empty_like(X0), torch.empty_like(Y0), torch.empty_like(w0)))
+    s_in = torch.cuda.Stream(device=stream.device)
+    s_out = torch.cuda.Stream(device=stream.device)
+
+    def run(n):
+        ev_in = [None] * n
+        ev_fw = [None] * n
+        ev_out = [None] * n
+        for i in range(n):
+            Xd, Yd, ws = bufs[i % 2]
+            if i >= 2:
+                s_in.wait_event(ev_fw[i - 2])  # Xd of step i-2 has been consumed
+            with torch.cuda.stream(s_in):
+                Xd.copy_(Xh, non_blocking=True)
+            ev_in[i] = torch.cuda.Event()
+            ev_in[i].record(s_in)
+            stream.wait_event(ev_in[i])
+            if i >= 2:
+                stream.wait_event(ev_out[i - 2])  # Yd of step i-2 has been copied out
+            lin.svdq_linear_forward(Xd, spec.M, spec.K, Yd, spec.N, ws, ws.numel(), stream)
+            ev_fw[i] = torch.cuda.Event()
+            ev_fw[i].record(stream)
+            s_out.wait_event(ev_fw[i])
+            with torch.cuda.stream(s_out):
+                Yh[i % 2].copy_(Yd, non_blocking=True)
+            ev_out[i] = torch.cuda.Event()
+            ev_out[i].record(s_out)
+        return ev_out[n - 1]
+
+    run(3)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    s_in.wait_event(e0)
+    last = run(steps)
+    s_out.wait_event(last)
+    e1.record(s_out)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, steps, int(Xh.numel() * 2), int(Yh[0].numel() * 2)
+
+
 def unfused_comparator(lin, layers, sets, layers0, sets0, steps, stream, k2_bare_ms):
     """The same layer with the low-rank branch unfused (the pages' naive version, for context):
     kernel 1 and kernel 2 of the rank-0 layer, plus a separate down projection that reads X again
@@ -508,29 +564,16 @@ def run_ours(args):
         line["lowrank_overhead_unfused"] = unfused_comparator(lin, layers, sets, layers0, sets0, n_over, stream, k2_0)
         for l0 in layers0:
             l0.close()
-        # End to end through the public API: pinned host X -> device, forward, Y -> pinned host.
-        Xh = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).pin_memory()
-        Yh = torch.empty((spec.M, spec.N), dtype=torch.bfloat16).pin_memory()
-        Xe, Ye, wse = sets[0]
-        n_e2e = min(args.steps, 30)
-        for _ in range(3):
-            Xe.copy_(Xh, non_blocking=True)
-            lin.svdq_linear_forward(Xe, spec.M, spec.K, Ye, spec.N, wse, wse.numel(), stream)
-            Yh.copy_(Ye, non_blocking=True)
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n_e2e):
-            Xe.copy_(Xh, non_blocking=True)
-            lin.svdq_linear_forward(Xe, spec.M, spec.K, Ye, spec.N, wse, wse.numel(), stream)
-            Yh.copy_(Ye, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
+        # End to end through the public API: every step copies X from pinned host memory to the
+        # device, runs the forward and copies Y back to pinned host memory.  Steps are pipelined
+        # over three streams and two device buffer sets (the copy in of step i+1 and the copy out
+        # of step i-1 overlap the forward of step i), as a serving loop would run them.
+        e2e_ms, n_e2e, h2d, d2h = e2e_pipelined(lin, X, spec, sets, stream)
+        e2e_ms = max_over_ranks(e2e_ms, world)
         line["e2e"] = {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
-                       "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yh.numel() * 2),
-                       "ms_per_step": e2e_ms, "steps": n_e2e}
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": e2e_ms, "steps": n_e2e,
+                       "pipeline": "3 streams (copy in, forward, copy out), 2 device buffer sets"}
         if world == 1:
             line["cpu_baseline"] = oracle_cpu_baseline(X, lin.export_weights(), args.precision, spec)
     for l in layers:
