@@ -30,6 +30,7 @@ METRIC = "W4A4+rank-32 linear TFLOP/s & % FP4 peak; low-rank overhead % on one B
 UNIT = "TFLOP/s"
 DEFAULT_WORKLOAD = "flux_qkv_4608x3072x9216_r32"
 FP4_PER_BF16 = 4.0  # nominal dense ratio: 9 PFLOP/s fp4 / 2.25 PFLOP/s bf16
+INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POP/s int8 / 2.25 PFLOP/s bf16 (INT4 runs on kind::i8)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCE = os.path.join(ROOT, "w4a4_rank_corrected_smooth_b200", "csrc", "kernels.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
@@ -514,8 +515,12 @@ def run_ours(args):
     value, total_ms = weak_scaling_value(flops, args.steps, total_ms, world)
     k2_flops = spec.flops_4bit + 2 * spec.M * spec.rank * spec.N
     k2_tflops = k2_flops / (k2_ms / 1e3) / 1e12
-    fp4_peak_sustained = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
-    fp4_peak_burst = peaks["bf16_tflops"] * FP4_PER_BF16
+    nvfp4 = args.precision == "nvfp4"
+    ratio = FP4_PER_BF16 if nvfp4 else INT8_PER_BF16
+    tensor_kind = "fp4" if nvfp4 else "int8"
+    fp4_peak_sustained = peaks["bf16_tflops_sustained"] * ratio  # the GEMM's own tensor dtype
+    fp4_peak_burst = peaks["bf16_tflops"] * ratio
+    sfx = "" if nvfp4 else "_int4"
     k1_bytes = (2 * spec.M * spec.K + spec.M * spec.K // 2 + spec.M * spec.K // 16 + 2 * spec.K * spec.rank
                 + 2 * spec.M * spec.rank)
     k2_bytes = (spec.M * spec.K // 2 + spec.M * spec.K // 16 + spec.N * spec.K // 2 + spec.N * spec.K // 16
@@ -528,17 +533,17 @@ def run_ours(args):
         "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "rank": spec.rank,
                    "precision": args.precision, "parallelism": f"replicas x{world}",
                    "l2": f"{args.sets} rotating copies of X/Y/workspace/weights (> 3x L2), no flush"},
-        "fp4_peak_frac": value / world / fp4_peak_sustained,
+        "tensor_peak_frac": value / world / fp4_peak_sustained,
         "kernel_ms": {"quant_down": k1_ms, "gemm": k2_ms},
         "roofline": {"bound": "tensor", "achieved": k2_tflops, "peak": fp4_peak_sustained, "unit": "TFLOP/s",
-                     "frac": k2_tflops / fp4_peak_sustained, "traffic": stored_traffic("gemm", spec.name),
-                     "kernel": "gemm_nvfp4_kernel",
-                     "peak_source": f"{peak_src} bf16 sustained x {FP4_PER_BF16:g} (nominal fp4/bf16)",
+                     "frac": k2_tflops / fp4_peak_sustained, "traffic": stored_traffic("gemm" + sfx, spec.name),
+                     "kernel": "gemm_nvfp4_kernel" if nvfp4 else "gemm_int4_kernel",
+                     "peak_source": f"{peak_src} bf16 sustained x {ratio:g} (nominal {tensor_kind}/bf16)",
                      "frac_of_burst_peak": k2_tflops / fp4_peak_burst,
                      "algorithmic_flops_per_launch": k2_flops},
         "quant_down_roofline": {"bound": "hbm", "achieved": k1_bytes / (k1_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                                 "unit": "GB/s", "frac": k1_bytes / (k1_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-                                "traffic": stored_traffic("quant_down", spec.name),
+                                "traffic": stored_traffic("quant_down" + sfx, spec.name),
                                 "algorithmic_bytes_per_launch": k1_bytes},
         "gemm_algorithmic_bytes_per_launch": k2_bytes,
         "gpu_launches": 2 * args.steps,
