@@ -25,7 +25,7 @@ computed as "Quantize"+"Down Projection" on the input and
 compute_dtype bfloat16; section "Introducing Nunchaku Lite": INT4 and NVFP4
 variants of the svdq_w4a4 kernel family.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   R1 lam_k = a_k^alpha * w_k^(alpha-1) with alpha = 0.5, i.e. sqrt(a_k / w_k),
      a_k = max_m |X[m,k]|, w_k = max_n |W[n,k]|; lam_k = 1 if a_k or w_k is 0.
   R2 X_hat = fp32(x) * fp32(1/lam): one fp32 multiply by the fp32 reciprocal.
