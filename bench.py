@@ -32,7 +32,8 @@ DEFAULT_WORKLOAD = "flux_qkv_4608x3072x9216_r32"
 FP4_PER_BF16 = 4.0  # nominal dense ratio: 9 PFLOP/s fp4 / 2.25 PFLOP/s bf16
 INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POP/s int8 / 2.25 PFLOP/s bf16 (INT4 runs on kind::i8)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCE = os.path.join(ROOT, "w4a4_rank_corrected_smooth_b200", "csrc", "kernels.cu")
+KERNEL_SOURCES = [os.path.join(ROOT, "w4a4_rank_corrected_smooth_b200", "csrc", f)
+                  for f in ("kernels.cu", "ptx.cuh", "layout.h")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 
 
@@ -63,12 +64,15 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    """sha256 of the kernel source's code: comments, trailing blanks and blank lines removed, so a
-    comment edit does not orphan the ncu counters while any change to the code does."""
+    """sha256 of the kernel sources' code (kernels.cu and the headers it compiles with): comments,
+    trailing blanks and blank lines removed, so a comment edit does not orphan the ncu counters
+    while any change to the code does."""
     import re
 
-    with open(KERNEL_SOURCE, encoding="utf-8") as f:
-        text = f.read()
+    text = ""
+    for path in KERNEL_SOURCES:
+        with open(path, encoding="utf-8") as f:
+            text += f.read() + "\n"
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     lines = []
     for line in text.splitlines():
