@@ -43,6 +43,13 @@ Readings where the pages are silent:
      global scale.
   R7 packing: element 2i in bits 3:0, element 2i+1 in bits 7:4 of byte i.
   R8 output Y is returned here in fp64; the device returns bf16.
+  R9 W4A16 (the "awq_w4a16" family of "Introducing Nunchaku Lite" and the
+     quantization_config of "Native loading in Diffusers": precision int4,
+     group_size 64, 4-bit weights with 16-bit activations): the pages fix only
+     the weight format.  Reading: the same smoothing as R1; the smoothed weight
+     W_hat is quantized per row with R6's INT4 quantizer (no low-rank branch);
+     the 16-bit activations are bf16(X_hat) with X_hat as in R2; the output is
+     bf16(X_hat) dequant(Q4(W_hat))^T + b (exact here, fp32 on a device).
 """
 from __future__ import annotations
 
@@ -375,6 +382,32 @@ def linear(X_bf16: np.ndarray, ops: Dict[str, np.ndarray], precision: str) -> Di
     T = lowrank_down(xh, ops["L1"])
     Y = forward(cx, sx, T, ops["codes_w"], ops["scales_w"], ops["L2"], ops["bias"], precision)
     return {"x_hat": xh, "codes_x": cx, "scales_x": sx, "T": T, "Y": Y}
+
+
+# ---------------------------------------------------------------------------
+# W4A16 ("awq_w4a16", R9): 4-bit weights, 16-bit activations
+# ---------------------------------------------------------------------------
+
+
+def prepare_w4a16(W_bf16: np.ndarray, bias_bf16: Optional[np.ndarray], a: np.ndarray,
+                  alpha: float = 0.5) -> Dict[str, np.ndarray]:
+    """Offline prepare of a W4A16 layer: smoothing (R1), INT4 group-64 codes and fp32 scales of
+    the smoothed weight (R6), no low-rank branch.  Keys as ``prepare`` returns them."""
+    return prepare(W_bf16, bias_bf16, a, INT4, 0, alpha)
+
+
+def linear_w4a16(X_bf16: np.ndarray, ops: Dict[str, np.ndarray]) -> Dict[str, np.ndarray]:
+    """Y (fp64) = bf16(X_hat) dequant(Q4(W_hat))^T + b, the sum taken exactly (R9).
+
+    Every dequantized weight (int4 code x fp32 scale) and every bf16 activation is exact in fp64;
+    the product is taken with a library matmul."""
+    xh = smooth_activations(X_bf16, ops["inv_lambda"])
+    xb16 = f32_to_bf16(xh)
+    Wd = dequantize_rows(ops["codes_w"], ops["scales_w"], INT4)
+    Y = bf16_to_f32(xb16).astype(np.float64) @ Wd.T
+    if ops.get("bias") is not None:
+        Y = Y + bf16_to_f32(ops["bias"]).astype(np.float64)[None, :]
+    return {"x_hat_bf16": xb16, "Y": Y}
 
 
 def exact_linear(X_bf16: np.ndarray, W_bf16: np.ndarray, bias_bf16: Optional[np.ndarray]) -> np.ndarray:

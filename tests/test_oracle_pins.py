@@ -415,6 +415,74 @@ def test_svdquant_error_ordering_on_outlier_data():
         assert e_svdq < e_smooth < e_plain, (prec, e_svdq, e_smooth, e_plain)
 
 
+# ---------------------------------------------------------------- W4A16 (R9)
+
+
+def test_w4a16_lossless_on_grid_equals_exact_product():
+    """lam = 1 and weights already on the INT4 grid (groups of 64 values q * 2^e with a |q| = 7
+    in every group): quantization is lossless, so the W4A16 forward equals X W^T + b."""
+    rng = np.random.default_rng(21)
+    M, K, N = 5, 128, 6
+    q = rng.integers(-7, 8, (N, K)).astype(np.float64)
+    q[:, ::64] = 7.0  # every group's maximum is 7, so its scale is exactly 2^e
+    e = rng.integers(-8, -2, (N, K // 64)).astype(np.float64)
+    W = (q * np.repeat(2.0 ** e, 64, axis=1)).astype(np.float32)
+    Wb = O.f32_to_bf16(W)
+    assert np.array_equal(O.bf16_to_f32(Wb), W)
+    X = O.f32_to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    b = O.f32_to_bf16(rng.standard_normal(N).astype(np.float32))
+    ops = O.prepare_w4a16(Wb, b, np.zeros(K, np.float32))  # a = 0 -> lam = 1
+    assert np.all(ops["inv_lambda"] == 1.0)
+    Y = O.linear_w4a16(X, ops)["Y"]
+    np.testing.assert_allclose(Y, O.exact_linear(X, Wb, b), rtol=1e-12, atol=1e-12)
+
+
+def test_w4a16_brute_force_loops():
+    """The forward restated as plain loops over (m, n, group, k) on the unpacked codes, in another
+    order than the library matmul: bf16 activations times code times group scale, plus bias."""
+    rng = np.random.default_rng(22)
+    M, K, N = 3, 128, 4
+    X = O.f32_to_bf16((rng.standard_normal((M, K)) * 3).astype(np.float32))
+    W = O.f32_to_bf16((rng.standard_normal((N, K)) * 0.05).astype(np.float32))
+    b = O.f32_to_bf16(rng.standard_normal(N).astype(np.float32))
+    a = (np.abs(rng.standard_normal(K)) + 0.1).astype(np.float32)
+    ops = O.prepare_w4a16(W, b, a)
+    out = O.linear_w4a16(X, ops)
+    nib = O.unpack_nibbles(ops["codes_w"])
+    qv = np.where(nib >= 8, nib.astype(np.int64) - 16, nib.astype(np.int64))
+    xb = O.bf16_to_f32(out["x_hat_bf16"])
+    bias = O.bf16_to_f32(b)
+    for m in range(M):
+        for n in range(N):
+            acc = 0.0
+            for g in range(K // 64):
+                part = 0.0
+                for k in range(g * 64 + 63, g * 64 - 1, -1):
+                    part += float(xb[m, k]) * float(qv[n, k])
+                acc += float(ops["scales_w"][n, g]) * part
+            acc += float(bias[n])
+            assert abs(acc - out["Y"][m, n]) <= 1e-12 * max(1.0, abs(acc))
+    # the 16-bit activations are bf16 of the fp32 smoothed activations
+    assert np.array_equal(out["x_hat_bf16"], O.f32_to_bf16(O.smooth_activations(X, ops["inv_lambda"])))
+
+
+def test_w4a16_smoothing_reduces_error_on_outlier_data():
+    """The pages use the W4A16 family for precision-sensitive layers; with the reading's
+    smoothing, the weight error that multiplies the outlier channels shrinks by lam, so on outlier
+    data the smoothed layer is closer to X W^T + b than the plain one."""
+    import synth
+
+    spec = synth.get("tiny_256x512x512_r16")
+    X = synth.activations_bf16(spec)
+    W = synth.weight_bf16(spec)
+    b = synth.bias_bf16(spec)
+    exact = O.exact_linear(X, W, b)
+    a = np.max(np.abs(O.bf16_to_f32(X)), axis=0)
+    e_plain = O.rel_fro(O.linear_w4a16(X, O.prepare_w4a16(W, b, np.zeros_like(a)))["Y"], exact)
+    e_smooth = O.rel_fro(O.linear_w4a16(X, O.prepare_w4a16(W, b, a))["Y"], exact)
+    assert e_smooth < 0.75 * e_plain, (e_smooth, e_plain)
+
+
 def test_pages_quantization_config_matches_oracle_groups():
     with open(os.path.join(HERE, "golden", "quantization_config.json")) as f:
         cfg = json.load(f)
