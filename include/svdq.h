@@ -55,7 +55,13 @@ typedef enum {
   SVDQ_ERR_INTERNAL = 6
 } svdq_status;
 
-typedef enum { SVDQ_NVFP4 = 0, SVDQ_INT4 = 1 } svdq_precision;
+/* SVDQ_NVFP4 and SVDQ_INT4: the W4A4 layer with its low-rank branch.  SVDQ_W4A16: 4-bit weights
+ * (the INT4 quantizer, group 64, of the smoothed weight) with 16-bit activations and no low-rank
+ * branch, the pages' "awq_w4a16" family ("Introducing Nunchaku Lite"; quantization_config
+ * precision int4, group_size 64) for small-M, memory-bound layers: rank must be 0, K <= 49152, the
+ * forward is one kernel that needs no workspace (svdq_workspace_size returns 0), and
+ * svdq_quant_down, svdq_gemm_up and svdq_export_activations return SVDQ_ERR_INVALID_ARG. */
+typedef enum { SVDQ_NVFP4 = 0, SVDQ_INT4 = 1, SVDQ_W4A16 = 2 } svdq_precision;
 
 /* Opaque prepared layer: device buffers owned by the library until svdq_free_weights. */
 typedef struct svdq_weights svdq_weights;

@@ -147,3 +147,23 @@ def test_prepare_rejects_bad_alpha():
     with pytest.raises(S.SVDQError) as ei:
         S.svdq_prepare_host(np.zeros((256, 256), np.uint16), None, np.ones(256, np.float32), "nvfp4", 16, alpha=1.5)
     assert "alpha" in str(ei.value)
+
+
+def test_host_prepare_w4a16_against_oracle():
+    """W4A16 (rank 0, INT4 weights of the smoothed weight): smoothing exact, codes and scales of the
+    library's own fp32 smoothed weight exactly as the oracle quantizes them."""
+    spec = synth.custom("w4a16_host", M=64, K=512, N=256, rank=0, seed=31)
+    X = synth.activations_bf16(spec)
+    W = synth.weight_bf16(spec)
+    a = synth.act_absmax(X)
+    lib = S.svdq_prepare_host(W, None, a, "w4a16", 0)
+    ref = O.prepare_w4a16(W, None, a)
+    assert np.array_equal(lib["inv_lambda"], ref["inv_lambda"])
+    oc, os_ = O.quantize_rows(lib["R"], O.INT4)
+    assert np.array_equal(lib["codes_w"], oc) and np.array_equal(lib["scales_w"], os_)
+    # the library's smoothed weight is the oracle's up to the last fp32 rounding
+    assert np.max(np.abs(lib["R"].astype(np.float64) - ref["R"].astype(np.float64))) <= \
+        1e-6 * np.max(np.abs(ref["R"]))
+    with pytest.raises(S.SVDQError) as ei:
+        S.svdq_prepare_host(W, None, a, "w4a16", 16)
+    assert ei.value.status == 1 and "no low-rank branch" in str(ei.value)

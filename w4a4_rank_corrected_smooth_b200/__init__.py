@@ -17,8 +17,9 @@ LIB_PATH = os.path.join(HERE, "lib", "libsvdq_b200.so")
 
 SVDQ_NVFP4 = 0
 SVDQ_INT4 = 1
-PRECISIONS = {"nvfp4": SVDQ_NVFP4, "int4": SVDQ_INT4}
-GROUP = {SVDQ_NVFP4: 16, SVDQ_INT4: 64}
+SVDQ_W4A16 = 2  # 4-bit weights, 16-bit activations, no low-rank branch (rank 0)
+PRECISIONS = {"nvfp4": SVDQ_NVFP4, "int4": SVDQ_INT4, "w4a16": SVDQ_W4A16}
+GROUP = {SVDQ_NVFP4: 16, SVDQ_INT4: 64, SVDQ_W4A16: 64}
 
 SVDQ_OK = 0
 STATUS_NAMES = {0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_UNSUPPORTED_DEVICE", 3: "SVDQ_ERR_CUDA",
@@ -285,5 +286,5 @@ class SVDQLinear:
 
 
 __all__ = ["SVDQLinear", "SVDQError", "svdq_check_device", "svdq_get_device_error", "svdq_selftest_wait_timeout",
-           "svdq_quantize_rows_host", "svdq_prepare_host", "SVDQ_NVFP4", "SVDQ_INT4", "LIB_PATH", "lib",
+           "svdq_quantize_rows_host", "svdq_prepare_host", "SVDQ_NVFP4", "SVDQ_INT4", "SVDQ_W4A16", "LIB_PATH", "lib",
            "DECLARED_SYMBOLS"]

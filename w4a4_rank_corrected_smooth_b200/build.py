@@ -22,7 +22,7 @@ NVCC = os.path.join(CUDA_HOME, "bin", "nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 HEADERS = ["ptx.cuh", "layout.h", "kernels.h", "host_prepare.h"]
-SOURCES = ["kernels.cu", "svdq_api.cpp", "host_prepare.cpp"]
+SOURCES = ["kernels.cu", "w4a16.cu", "svdq_api.cpp", "host_prepare.cpp"]
 
 
 def _newer(src_paths, dst):

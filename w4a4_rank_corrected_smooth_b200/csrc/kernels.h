@@ -31,9 +31,23 @@ struct GemmArgs {
   uint16_t* Y;
 };
 
+// W4A16 layer (4-bit weights in canonical row-major layout, 16-bit activations).
+struct W4A16Args {
+  const uint16_t* X;        // M x K bf16, row stride ldx
+  int M, K, ldx, N, ldy;
+  const float* inv_lambda;  // K
+  const uint8_t* codes;     // N x K/2 (element 2i in the low nibble of byte i)
+  const float* scales;      // N x K/64 fp32
+  const float* bias;        // N (fp32)
+  uint16_t* Y;              // M x N bf16, row stride ldy
+};
+
 // Returns a cudaError_t of the launch (cudaSuccess when the launch was queued).
 cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_w4a16(const W4A16Args& a, int num_sms, cudaStream_t stream);
+// Largest K the W4A16 kernel accepts (x_hat rows are staged in shared memory).
+constexpr int kW4A16MaxK = 49152;
 cudaError_t launch_selftest_wait(int spin_limit, cudaStream_t stream);
 cudaError_t read_and_clear_device_error(unsigned int* value, cudaStream_t stream);
 

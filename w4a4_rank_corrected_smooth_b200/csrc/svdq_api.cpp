@@ -59,10 +59,18 @@ struct DeviceGuard {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// The W4A16 layer quantizes its weights with the INT4 quantizer (group 64, fp32 scales).
+int quantizer_precision(int precision) { return precision == SVDQ_W4A16 ? SVDQ_INT4 : precision; }
+
 svdq_status check_shape(int N, int K, const svdq_prepare_params* p) {
   if (!p) return fail(SVDQ_ERR_INVALID_ARG, "params is NULL");
-  if (p->precision != SVDQ_NVFP4 && p->precision != SVDQ_INT4)
-    return fail(SVDQ_ERR_INVALID_ARG, "precision %d is neither SVDQ_NVFP4 (0) nor SVDQ_INT4 (1)", p->precision);
+  if (p->precision != SVDQ_NVFP4 && p->precision != SVDQ_INT4 && p->precision != SVDQ_W4A16)
+    return fail(SVDQ_ERR_INVALID_ARG, "precision %d is not SVDQ_NVFP4 (0), SVDQ_INT4 (1) or SVDQ_W4A16 (2)",
+                p->precision);
+  if (p->precision == SVDQ_W4A16 && p->rank != 0)
+    return fail(SVDQ_ERR_INVALID_ARG, "rank=%d: the W4A16 layer has no low-rank branch (rank must be 0)", p->rank);
+  if (p->precision == SVDQ_W4A16 && K > svdq::kW4A16MaxK)
+    return fail(SVDQ_ERR_INVALID_ARG, "K=%d exceeds %d for the W4A16 layer", K, svdq::kW4A16MaxK);
   if (N <= 0 || K <= 0) return fail(SVDQ_ERR_INVALID_ARG, "N=%d and K=%d must be positive", N, K);
   if (K % svdq::kBK != 0) return fail(SVDQ_ERR_INVALID_ARG, "K=%d must be a multiple of %d", K, svdq::kBK);
   if (N % 8 != 0) return fail(SVDQ_ERR_INVALID_ARG, "N=%d must be a multiple of 8", N);
@@ -101,6 +109,7 @@ svdq_status check_forward_common(const svdq_weights* w, int M, const void* ws, s
   if (!w) return fail(SVDQ_ERR_INVALID_ARG, "weights handle is NULL");
   if (M < 0) return fail(SVDQ_ERR_INVALID_ARG, "M=%d is negative", M);
   if (M == 0) return SVDQ_OK;
+  if (w->precision == SVDQ_W4A16) return SVDQ_OK;  // no workspace: one kernel, nothing in between
   const svdq::WorkspaceLayout L = svdq::workspace_layout(M, w->K, w->rank);
   if (!ws) return fail(SVDQ_ERR_INVALID_ARG, "workspace is NULL");
   if (!aligned(ws, 256)) return fail(SVDQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
@@ -159,6 +168,27 @@ svdq_status do_gemm(const svdq_weights* w, int M, void* Y, int ldy, const void* 
   a.Y = static_cast<uint16_t*>(Y);
   cudaError_t e = svdq::launch_gemm(a, w->num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launch of the 4-bit GEMM/up-projection kernel");
+  return SVDQ_OK;
+}
+
+svdq_status do_w4a16(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy, cudaStream_t stream) {
+  if (!X) return fail(SVDQ_ERR_INVALID_ARG, "X is NULL");
+  if (ldx < w->K || ldx % 8 != 0) return fail(SVDQ_ERR_INVALID_ARG, "ldx=%d must be >= K=%d and a multiple of 8", ldx, w->K);
+  if (!aligned(X, 16)) return fail(SVDQ_ERR_INVALID_ARG, "X must be 16-byte aligned");
+  svdq::W4A16Args a;
+  a.X = static_cast<const uint16_t*>(X);
+  a.M = M;
+  a.K = w->K;
+  a.ldx = ldx;
+  a.N = w->N;
+  a.ldy = ldy;
+  a.inv_lambda = w->d_inv_lambda;
+  a.codes = w->d_codes;
+  a.scales = reinterpret_cast<const float*>(w->d_sf);
+  a.bias = w->d_bias;
+  a.Y = static_cast<uint16_t*>(Y);
+  cudaError_t e = svdq::launch_w4a16(a, w->num_sms, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the W4A16 kernel");
   return SVDQ_OK;
 }
 
@@ -227,8 +257,8 @@ svdq_status svdq_prepare_host(const uint16_t* W_bf16, int N, int K, const uint16
   if (!W_bf16 || !act_absmax) return fail(SVDQ_ERR_INVALID_ARG, "W or act_absmax is NULL");
   svdq::CanonicalLayer c;
   try {
-    svdq::prepare_canonical(W_bf16, N, K, bias_bf16, act_absmax, params->precision, params->rank, params->alpha,
-                            params->svd_iters > 0 ? params->svd_iters : 12, params->seed, c);
+    svdq::prepare_canonical(W_bf16, N, K, bias_bf16, act_absmax, quantizer_precision(params->precision), params->rank,
+                            params->alpha, params->svd_iters > 0 ? params->svd_iters : 12, params->seed, c);
   } catch (const std::bad_alloc&) {
     return fail(SVDQ_ERR_OOM, "host allocation failed in prepare");
   }
@@ -268,9 +298,17 @@ svdq_status svdq_prepare_weights(const uint16_t* W_bf16, int N, int K, const uin
   cudaDeviceGetAttribute(&w->num_sms, cudaDevAttrMultiProcessorCount, device);
   svdq::DeviceImages img;
   try {
-    svdq::prepare_canonical(W_bf16, N, K, bias_bf16, act_absmax, params->precision, params->rank, params->alpha,
-                            params->svd_iters > 0 ? params->svd_iters : 12, params->seed, w->canon);
+    svdq::prepare_canonical(W_bf16, N, K, bias_bf16, act_absmax, quantizer_precision(params->precision), params->rank,
+                            params->alpha, params->svd_iters > 0 ? params->svd_iters : 12, params->seed, w->canon);
     svdq::pack_device_layouts(w->canon, img);
+    if (params->precision == SVDQ_W4A16) {
+      // Canonical row-major codes [N][K/2] and fp32 scales [N][K/64], zero rows up to the padded N.
+      const size_t npad = static_cast<size_t>((N + svdq::kBN - 1) / svdq::kBN) * svdq::kBN;
+      img.codes.assign(npad * K / 2, 0);
+      std::memcpy(img.codes.data(), w->canon.codes_w.data(), static_cast<size_t>(N) * K / 2);
+      img.sf.assign(npad * K / svdq::kBK * svdq::kSfBytesPerRowKb, 0);
+      std::memcpy(img.sf.data(), w->canon.scales_int4.data(), sizeof(float) * static_cast<size_t>(N) * K / 64);
+    }
   } catch (const std::bad_alloc&) {
     delete w;
     return fail(SVDQ_ERR_OOM, "host allocation failed in prepare");
@@ -386,7 +424,7 @@ svdq_status svdq_export_weights(const svdq_weights* w, float* inv_lambda, uint8_
 svdq_status svdq_workspace_size(const svdq_weights* w, int M, size_t* bytes) {
   if (!w || !bytes) return fail(SVDQ_ERR_INVALID_ARG, "NULL argument");
   if (M < 0) return fail(SVDQ_ERR_INVALID_ARG, "M=%d is negative", M);
-  *bytes = svdq::workspace_layout(M, w->K, w->rank).total;
+  *bytes = w->precision == SVDQ_W4A16 ? 0 : svdq::workspace_layout(M, w->K, w->rank).total;
   return SVDQ_OK;
 }
 
@@ -412,6 +450,8 @@ svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, in
 
 svdq_status svdq_quant_down(const svdq_weights* w, const void* X, int M, int ldx, void* workspace,
                             size_t workspace_bytes, void* stream) {
+  if (w && w->precision == SVDQ_W4A16)
+    return fail(SVDQ_ERR_INVALID_ARG, "the W4A16 layer runs as one kernel: use svdq_linear_forward");
   svdq_status s = check_forward_common(w, M, workspace, workspace_bytes);
   if (s != SVDQ_OK || M == 0) return s;
   DeviceGuard guard(w->device);
@@ -420,6 +460,8 @@ svdq_status svdq_quant_down(const svdq_weights* w, const void* X, int M, int ldx
 
 svdq_status svdq_gemm_up(const svdq_weights* w, int M, void* Y, int ldy, const void* workspace, size_t workspace_bytes,
                          void* stream) {
+  if (w && w->precision == SVDQ_W4A16)
+    return fail(SVDQ_ERR_INVALID_ARG, "the W4A16 layer runs as one kernel: use svdq_linear_forward");
   svdq_status s = check_forward_common(w, M, workspace, workspace_bytes);
   if (s != SVDQ_OK || M == 0) return s;
   DeviceGuard guard(w->device);
@@ -435,6 +477,7 @@ svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int
     return fail(SVDQ_ERR_INVALID_ARG, "Y must be 16-byte aligned with ldy >= N and a multiple of 8");
   DeviceGuard guard(w->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (w->precision == SVDQ_W4A16) return do_w4a16(w, X, M, ldx, Y, ldy, st);
   s = do_quant_down(w, X, M, ldx, workspace, st);
   if (s != SVDQ_OK) return s;
   return do_gemm(w, M, Y, ldy, workspace, st);
@@ -442,6 +485,8 @@ svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int
 
 svdq_status svdq_export_activations(const svdq_weights* w, const void* workspace, size_t workspace_bytes, int M,
                                     uint8_t* codes_x, void* scales_x, uint16_t* T, void* stream) {
+  if (w && w->precision == SVDQ_W4A16)
+    return fail(SVDQ_ERR_INVALID_ARG, "the W4A16 layer runs as one kernel: use svdq_linear_forward");
   svdq_status s = check_forward_common(w, M, workspace, workspace_bytes);
   if (s != SVDQ_OK || M == 0) return s;
   DeviceGuard guard(w->device);
