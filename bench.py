@@ -464,6 +464,59 @@ def unfused_comparator(lin, layers, sets, layers0, sets0, steps, stream, k2_bare
             "comparator": "down projection X (diag(1/lambda) L1) and up projection Y += T L2 as separate cuBLAS GEMMs"}
 
 
+W4A16_SHAPES = [(1, 3072, 18432), (2, 3072, 18432), (4, 3072, 18432), (1, 3072, 9216)]
+
+
+def w4a16_leg(dev, stream, peaks, peak_src, launches: int = 200):
+    """The W4A16 layer on FLUX's modulation projections (one token per image: M rows of K = 3072
+    into N = 6*3072 or 3*3072): each launch timed alone with CUDA events on the launching stream,
+    L2 flushed (a 256 MiB write) before every launch, median over ``launches``.  Weight-only
+    4-bit layers of this size are bound by HBM, so the roofline is the measured copy bandwidth."""
+    import numpy as np
+    import torch
+
+    import synth
+    import w4a4_rank_corrected_smooth_b200 as S
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = {}
+    prepared = {}
+    for (M, K, N) in W4A16_SHAPES:
+        if (K, N) not in prepared:
+            for lin_, _ in prepared.values():
+                lin_.close()
+            prepared.clear()
+            spec = synth.custom(f"flux_modulation_{K}x{N}", M=8, K=K, N=N, rank=0, seed=N)
+            X8 = synth.activations_bf16(spec)
+            prepared[(K, N)] = (S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(X8),
+                                             "w4a16", 0, device=dev.index), X8)
+        lin, X8 = prepared[(K, N)]
+        Xd = bf16_device(np.ascontiguousarray(X8[:M]), dev)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(5):
+            lin.svdq_linear_forward(Xd, M, K, Y, N, None, 0, stream)
+        ts = []
+        for _ in range(launches):
+            flush.fill_(1)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            lin.svdq_linear_forward(Xd, M, K, Y, N, None, 0, stream)
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        S.svdq_get_device_error(stream)
+        ms = float(np.median(ts))
+        nbytes = N * K // 2 + 4 * N * (K // 64) + 2 * M * K + 2 * M * N + 4 * K + 4 * N
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[f"{M}x{K}x{N}"] = {"us": ms * 1e3, "algorithmic_bytes_per_launch": nbytes, "achieved_gbs": gbs,
+                               "frac": gbs / peaks["hbm_gbs"]}
+    for lin_, _ in prepared.values():
+        lin_.close()
+    return {"kernel": "w4a16_kernel", "bound": "hbm", "peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src,
+            "timing": f"median of {launches} launches, each alone, L2 flushed before each", "shapes": out}
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -585,6 +638,7 @@ def run_ours(args):
                        "pipeline": "3 streams (copy in, forward, copy out), 2 device buffer sets"}
         if world == 1:
             line["cpu_baseline"] = oracle_cpu_baseline(X, lin.export_weights(), args.precision, spec)
+            line["w4a16_modulation"] = w4a16_leg(dev, stream, peaks, peak_src)
     for l in layers:
         l.close()
     if world > 1:
@@ -666,6 +720,7 @@ def run_sweep(args):
     for l, l0 in prepared.values():
         l.close()
         l0.close()
+    print(json.dumps({"sweep": True, "w4a16_modulation": w4a16_leg(dev, stream, peaks, peak_src)}), flush=True)
 
 
 def main():
