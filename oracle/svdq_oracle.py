@@ -50,6 +50,18 @@ Readings where the pages are silent:
      W_hat is quantized per row with R6's INT4 quantizer (no low-rank branch);
      the 16-bit activations are bf16(X_hat) with X_hat as in R2; the output is
      bf16(X_hat) dequant(Q4(W_hat))^T + b (exact here, fp32 on a device).
+  R10 fused QKV + Q/K normalization + rotary embedding ("Bringing Nunchaku
+     4-bit Diffusion Inference to Diffusers", section "Quantizing models with
+     structural rewrites": one operator consumes the grouped QKV projection,
+     norm_q, norm_k and the rotary embedding; Q, K and V are concatenated along
+     the output dimension in that order).  The pages name the steps only.
+     Reading: the layer output Y (before its rounding to bf16) splits into Q, K
+     and V of H heads of D channels each; every head vector of Q and K is
+     divided by sqrt(mean of its squares + eps) and multiplied by the norm's
+     per-channel weight (RMS normalization; eps = 1e-6); then channels 2i and
+     2i+1 of the head are turned as one pair by the angle of (row m, pair i),
+     given as cos and sin tables (out_2i = a cos - b sin, out_2i+1 = a sin +
+     b cos); V passes unchanged; one rounding to bf16 at the end.
 """
 from __future__ import annotations
 
@@ -408,6 +420,58 @@ def linear_w4a16(X_bf16: np.ndarray, ops: Dict[str, np.ndarray]) -> Dict[str, np
     if ops.get("bias") is not None:
         Y = Y + bf16_to_f32(ops["bias"]).astype(np.float64)[None, :]
     return {"x_hat_bf16": xb16, "Y": Y}
+
+
+# ---------------------------------------------------------------------------
+# Fused QKV + RMS normalization of Q and K + rotary embedding (R10)
+# ---------------------------------------------------------------------------
+
+
+def rms_norm_heads(heads: np.ndarray, weight: np.ndarray, eps: float) -> np.ndarray:
+    """heads [M, H, D] (fp64): each head vector over its D channels divided by the square root of
+    (its mean square + eps), then multiplied channel by channel by ``weight`` [D]."""
+    ms = np.mean(heads * heads, axis=-1, keepdims=True)
+    return heads / np.sqrt(ms + eps) * np.asarray(weight, np.float64)[None, None, :]
+
+
+def rotate_pairs(heads: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """heads [M, H, D] (fp64); channels (2i, 2i+1) of every head of row m turned by the angle
+    whose cosine and sine are cos[m, i] and sin[m, i] ([M, D/2])."""
+    a = heads[..., 0::2]
+    b = heads[..., 1::2]
+    c = np.asarray(cos, np.float64)[:, None, :]
+    s = np.asarray(sin, np.float64)[:, None, :]
+    out = np.empty_like(heads)
+    out[..., 0::2] = a * c - b * s
+    out[..., 1::2] = a * s + b * c
+    return out
+
+
+def qkv_norm_rope(Y: np.ndarray, head_dim: int, gamma_q: np.ndarray, gamma_k: np.ndarray,
+                  cos: np.ndarray, sin: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """The fused operator's steps after the projection (R10), in fp64: Y [M, 3 H D] = [Q | K | V];
+    Q and K normalized per head and rotated, V unchanged."""
+    Y = np.asarray(Y, np.float64)
+    M, N = Y.shape
+    assert N % (3 * head_dim) == 0 and head_dim % 2 == 0
+    H = N // (3 * head_dim)
+    out = Y.copy()
+    for part, gamma in ((0, gamma_q), (1, gamma_k)):
+        cols = slice(part * H * head_dim, (part + 1) * H * head_dim)
+        heads = Y[:, cols].reshape(M, H, head_dim)
+        out[:, cols] = rotate_pairs(rms_norm_heads(heads, gamma, eps), cos, sin).reshape(M, H * head_dim)
+    return out
+
+
+def linear_qkv_norm_rope(X_bf16: np.ndarray, ops: Dict[str, np.ndarray], precision: str, head_dim: int,
+                         gamma_q: np.ndarray, gamma_k: np.ndarray, cos: np.ndarray, sin: np.ndarray,
+                         eps: float = 1e-6) -> Dict[str, np.ndarray]:
+    """The grouped QKV layer followed by R10: the layer's forward (as ``linear``) and the fused
+    normalization and rotation of its exact output."""
+    r = linear(X_bf16, ops, precision)
+    r["Y_layer"] = r["Y"]
+    r["Y"] = qkv_norm_rope(r["Y"], head_dim, gamma_q, gamma_k, cos, sin, eps)
+    return r
 
 
 def exact_linear(X_bf16: np.ndarray, W_bf16: np.ndarray, bias_bf16: Optional[np.ndarray]) -> np.ndarray:

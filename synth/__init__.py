@@ -202,6 +202,36 @@ def act_absmax(x_bf16: np.ndarray) -> np.ndarray:
     return np.max(np.abs(bf16_bits_to_f32(x_bf16)), axis=0).astype(np.float32)
 
 
+def rms_norm_weight(head_dim: int, seed: int) -> np.ndarray:
+    """Per-channel weight of a Q or K RMS normalization: 1 + 0.1 N(0, 1), rounded to bf16 (a
+    bf16 model's parameter), returned as fp32."""
+    v = (1.0 + 0.1 * normal_f64(seed, 0, head_dim)).astype(np.float32)
+    return bf16_bits_to_f32(f32_to_bf16_bits(v))
+
+
+def rope_tables(M: int, head_dim: int = 128, text_tokens: int = 512, grid_w: int = 64,
+                axes: Tuple[int, ...] = (16, 56, 56), theta: float = 10000.0) -> Tuple[np.ndarray, np.ndarray]:
+    """cos and sin [M, head_dim / 2] (fp32) of FLUX-shaped rotary angles.
+
+    Rows below ``text_tokens`` are text tokens (every position 0); row r above is image token
+    r - text_tokens of a grid ``grid_w`` wide, at (h, w) = divmod(r - text_tokens, grid_w).  The
+    pairs of channels are split over three position axes (index, h, w) with ``axes[a]`` channels
+    each; pair i of axis a turns by pos_a * theta ** (-2 i / axes[a]).  Angles in fp64, cos and sin
+    rounded to fp32 (they are inputs of the rotation, as a model precomputes them)."""
+    assert sum(axes) == head_dim and all(a % 2 == 0 for a in axes)
+    r = np.arange(M, dtype=np.int64)
+    img = np.maximum(r - text_tokens, 0)
+    is_img = r >= text_tokens
+    pos = [np.zeros(M), np.where(is_img, img // grid_w, 0).astype(np.float64),
+           np.where(is_img, img % grid_w, 0).astype(np.float64)]
+    angles = []
+    for a, dim in enumerate(axes):
+        omega = theta ** (-np.arange(0, dim, 2, dtype=np.float64) / dim)
+        angles.append(pos[a][:, None] * omega[None, :])
+    ang = np.concatenate(angles, axis=1)
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
 def custom(name: str, M: int, K: int, N: int, rank: int, seed: int = 7, **kw) -> LayerSpec:
     """An ad-hoc layer (edge cases in tests): seeds derived from ``seed``."""
     return LayerSpec(name=name, M=M, K=K, N=N, rank=rank, seed_x=10000 + seed, seed_w=20000 + seed,
@@ -211,5 +241,5 @@ def custom(name: str, M: int, K: int, N: int, rank: int, seed: int = 7, **kw) ->
 __all__: List[str] = [
     "LayerSpec", "workloads", "get", "custom", "activations_bf16", "weight_bf16", "bias_bf16",
     "act_absmax", "f32_to_bf16_bits", "bf16_bits_to_f32", "normal_f64", "splitmix64",
-    "outlier_channels", "gelu_erf",
+    "outlier_channels", "gelu_erf", "rms_norm_weight", "rope_tables",
 ]

@@ -490,3 +490,137 @@ def test_pages_quantization_config_matches_oracle_groups():
     assert O.GROUP[O.NVFP4] == cfg["svdq_w4a4"]["group_size"] == 16
     assert cfg["svdq_w4a4"]["rank"] == 32
     assert O.GROUP[O.INT4] == 64
+
+
+# ---------------------------------------------------------------- fused QKV + RMS norm + rotary
+
+
+def _qkv(M, H, D, seed):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((M, 3 * H * D)) * rng.uniform(0.1, 10.0, size=(M, 1))
+
+
+def _parts(Y, H, D):
+    M = Y.shape[0]
+    return [Y[:, i * H * D:(i + 1) * H * D].reshape(M, H, D) for i in range(3)]
+
+
+def test_qkv_norm_unit_mean_square_and_v_untouched():
+    """Weight 1, eps 0, no turn: every Q and K head has mean square exactly 1 and V is Y's."""
+    M, H, D = 5, 3, 16
+    Y = _qkv(M, H, D, 1)
+    one = np.ones(D)
+    z = np.zeros((M, D // 2))
+    out = O.qkv_norm_rope(Y, D, one, one, np.ones((M, D // 2)), z, eps=0.0)
+    q, k, v = _parts(out, H, D)
+    assert np.allclose(np.mean(q * q, axis=-1), 1.0, rtol=0, atol=1e-13)
+    assert np.allclose(np.mean(k * k, axis=-1), 1.0, rtol=0, atol=1e-13)
+    assert np.array_equal(v, _parts(Y, H, D)[2])
+
+
+def test_qkv_norm_scale_invariance():
+    """With eps 0 the normalization forgets each head's scale; V keeps it."""
+    M, H, D = 4, 2, 8
+    Y = _qkv(M, H, D, 2)
+    rng = np.random.default_rng(3)
+    gq, gk = rng.uniform(0.5, 1.5, D), rng.uniform(0.5, 1.5, D)
+    ang = rng.uniform(-np.pi, np.pi, (M, D // 2))
+    a = O.qkv_norm_rope(Y, D, gq, gk, np.cos(ang), np.sin(ang), eps=0.0)
+    b = O.qkv_norm_rope(7.5 * Y, D, gq, gk, np.cos(ang), np.sin(ang), eps=0.0)
+    qa, ka, va = _parts(a, H, D)
+    qb, kb, vb = _parts(b, H, D)
+    assert np.allclose(qa, qb, rtol=1e-13, atol=0) and np.allclose(ka, kb, rtol=1e-13, atol=0)
+    assert np.allclose(vb, 7.5 * va, rtol=1e-15, atol=0)
+
+
+def test_qkv_norm_eps_closed_form():
+    """A head of constant value c: mean square c^2, so each channel becomes c / sqrt(c^2 + eps);
+    with c = 1e-3 and eps = 1e-6 that is 1/sqrt(2) (eps under the root, added to the mean)."""
+    M, H, D = 1, 1, 8
+    Y = np.full((M, 3 * D), 1e-3)
+    out = O.qkv_norm_rope(Y, D, np.ones(D), np.ones(D), np.ones((M, D // 2)), np.zeros((M, D // 2)), eps=1e-6)
+    assert np.allclose(out[:, :2 * D], 1.0 / math.sqrt(2.0), rtol=1e-14, atol=0)
+
+
+def test_qkv_norm_weight_is_per_channel():
+    """A one-hot norm weight keeps only its channel, at y_j / rms(y); Q and K use their own weights."""
+    M, H, D = 3, 2, 8
+    Y = _qkv(M, H, D, 4)
+    eq, ek = np.zeros(D), np.zeros(D)
+    eq[5], ek[2] = 1.0, 1.0
+    out = O.qkv_norm_rope(Y, D, eq, ek, np.ones((M, D // 2)), np.zeros((M, D // 2)), eps=0.0)
+    q, k, _ = _parts(out, H, D)
+    yq, yk, _ = _parts(Y, H, D)
+    for got, y, j in ((q, yq, 5), (k, yk, 2)):
+        rms = np.sqrt(np.mean(y * y, axis=-1))
+        assert np.count_nonzero(np.delete(got, j, axis=-1)) == 0
+        assert np.allclose(got[..., j], y[..., j] / rms, rtol=1e-14, atol=0)
+
+
+def test_rotary_quarter_turn_pairs_adjacent_channels():
+    """Head = e_{2i}; a quarter turn of pair i (cos 0, sin 1) moves it to e_{2i+1}: the pairs are
+    adjacent channels and the turn goes from the first channel of a pair towards the second."""
+    D, i = 8, 2
+    Y = np.zeros((1, 3 * D))
+    Y[0, 2 * i] = 1.0          # Q head 0
+    Y[0, D + 2 * i + 1] = 1.0  # K head 0: e_{2i+1} goes to -e_{2i}
+    cos = np.ones((1, D // 2))
+    sin = np.zeros((1, D // 2))
+    cos[0, i], sin[0, i] = 0.0, 1.0
+    out = O.qkv_norm_rope(Y, D, np.ones(D), np.ones(D), cos, sin, eps=0.0)
+    s = math.sqrt(D)  # a one-hot head has mean square 1/D
+    want_q = np.zeros(D)
+    want_q[2 * i + 1] = s
+    want_k = np.zeros(D)
+    want_k[2 * i] = -s
+    assert np.allclose(out[0, :D], want_q, rtol=0, atol=1e-15)
+    assert np.allclose(out[0, D:2 * D], want_k, rtol=0, atol=1e-15)
+
+
+def test_rotary_is_complex_multiplication():
+    """Each pair (a, b) read as the complex number a + ib is multiplied by exp(i theta)."""
+    M, H, D = 6, 2, 16
+    Y = _qkv(M, H, D, 5)
+    ang = np.random.default_rng(6).uniform(-np.pi, np.pi, (M, D // 2))
+    one = np.ones(D)
+    normed = O.qkv_norm_rope(Y, D, one, one, np.ones_like(ang), np.zeros_like(ang), eps=0.0)
+    turned = O.qkv_norm_rope(Y, D, one, one, np.cos(ang), np.sin(ang), eps=0.0)
+    for part in (0, 1):
+        n = _parts(normed, H, D)[part]
+        t = _parts(turned, H, D)[part]
+        z = (n[..., 0::2] + 1j * n[..., 1::2]) * np.exp(1j * ang)[:, None, :]
+        assert np.allclose(t[..., 0::2], z.real, rtol=0, atol=1e-13)
+        assert np.allclose(t[..., 1::2], z.imag, rtol=0, atol=1e-13)
+
+
+def test_rotary_turn_back_restores_the_normalized_heads():
+    """Weight 1 and eps 0: the output heads already have mean square 1, so applying the operator
+    again with the opposite angles gives the normalized input back."""
+    M, H, D = 4, 3, 8
+    Y = _qkv(M, H, D, 7)
+    ang = np.random.default_rng(8).uniform(-np.pi, np.pi, (M, D // 2))
+    one = np.ones(D)
+    fwd = O.qkv_norm_rope(Y, D, one, one, np.cos(ang), np.sin(ang), eps=0.0)
+    back = O.qkv_norm_rope(fwd, D, one, one, np.cos(ang), -np.sin(ang), eps=0.0)
+    normed = O.qkv_norm_rope(Y, D, one, one, np.ones_like(ang), np.zeros_like(ang), eps=0.0)
+    assert np.allclose(back, normed, rtol=0, atol=1e-13)
+
+
+def test_rotary_scores_depend_on_relative_position_only():
+    """With angles pos * omega_i, the dot product of a turned query at position m and a turned key
+    at position n depends on m - n only (the property rotary embeddings are built for)."""
+    D, H = 16, 1
+    omega = 10000.0 ** (-np.arange(0, D, 2) / D)
+    rng = np.random.default_rng(9)
+    qk = rng.standard_normal((1, 3 * H * D))
+    Y = np.repeat(qk, 4, axis=0)
+    pos = np.array([3.0, 11.0, 3.0 + 5.0, 11.0 + 5.0])  # (m, n) and (m + 5, n + 5)
+    ang = pos[:, None] * omega[None, :]
+    g = rng.uniform(0.5, 1.5, D)
+    out = O.qkv_norm_rope(Y, D, g, g, np.cos(ang), np.sin(ang))
+    q = out[:, :D]
+    k = out[:, D:2 * D]
+    s1 = float(q[0] @ k[1])
+    s2 = float(q[2] @ k[3])
+    assert abs(s1 - s2) <= 1e-12 * max(1.0, abs(s1))
+    assert abs(float(q[0] @ k[0]) - float(q[1] @ k[1])) <= 1e-12 * max(1.0, abs(float(q[0] @ k[0])))
