@@ -62,6 +62,12 @@ Readings where the pages are silent:
      2i+1 of the head are turned as one pair by the angle of (row m, pair i),
      given as cos and sin tables (out_2i = a cos - b sin, out_2i+1 = a sin +
      b cos); V passes unchanged; one rounding to bf16 at the end.
+  R11 fused GELU/MLP ("Introducing Nunchaku Lite": the engine's fused GELU/MLP
+     kernels; the pages give no formula).  Reading: the fused pair computes what
+     the unfused modules compute -- the up layer's output rounded to bf16, GELU
+     of it (x Phi(x), Phi the standard normal distribution function) rounded to
+     bf16, and that hidden activation as the down layer's input; fusing only
+     removes the hidden tensor's round trip through memory.
 """
 from __future__ import annotations
 
@@ -472,6 +478,50 @@ def linear_qkv_norm_rope(X_bf16: np.ndarray, ops: Dict[str, np.ndarray], precisi
     r["Y_layer"] = r["Y"]
     r["Y"] = qkv_norm_rope(r["Y"], head_dim, gamma_q, gamma_k, cos, sin, eps)
     return r
+
+
+# ---------------------------------------------------------------------------
+# Fused GELU/MLP pair (R11)
+# ---------------------------------------------------------------------------
+
+
+def f64_to_bf16(x: np.ndarray) -> np.ndarray:
+    """fp64 -> bf16 bit patterns, round to nearest, ties to even, in one step (no intermediate
+    fp32 rounding).  Same value-level rule as ``f32_to_bf16``: the two bf16 neighbours of x are
+    found by truncating its fp32-or-wider magnitude, and the nearer one wins."""
+    x = np.asarray(x, dtype=np.float64)
+    t = x.astype(np.float32)
+    # the fp32 nearest to x can lie on the other side of x; step back so that t is a truncation
+    over = np.abs(t.astype(np.float64)) > np.abs(x)
+    t = np.where(over, np.nextafter(t, np.float32(0), dtype=np.float32), t).astype(np.float32)
+    lo = (np.ascontiguousarray(t).view(np.uint32) >> np.uint32(16)).astype(np.uint32)
+    hi = lo + np.uint32(1)
+    v_lo = (lo << np.uint32(16)).view(np.float32).astype(np.float64)
+    v_hi = (hi << np.uint32(16)).view(np.float32).astype(np.float64)
+    d_lo = np.abs(x - v_lo)
+    d_hi = np.abs(v_hi - x)
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & ((lo & np.uint32(1)) == np.uint32(1)))
+    return np.where(pick_hi, hi, lo).astype(np.uint16)
+
+
+def gelu(y: np.ndarray) -> np.ndarray:
+    """GELU in fp64: y Phi(y), with Phi(y) = (1 + erf(y / sqrt 2)) / 2 (R11)."""
+    from scipy.special import erf  # a library primitive for the normal distribution function
+
+    y = np.asarray(y, dtype=np.float64)
+    return 0.5 * y * (1.0 + erf(y / np.sqrt(2.0)))
+
+
+def mlp_pair(X_bf16: np.ndarray, ops_up: Dict[str, np.ndarray], ops_down: Dict[str, np.ndarray],
+             precision: str) -> Dict[str, np.ndarray]:
+    """up layer -> bf16 -> GELU -> bf16 -> down layer (R11).  Returns the up layer's exact output,
+    the bf16 hidden activation, the down layer's 4-bit operands and T, and Y (fp64)."""
+    up = linear(X_bf16, ops_up, precision)
+    y_up_bf16 = f64_to_bf16(up["Y"])
+    h = f64_to_bf16(gelu(bf16_to_f32(y_up_bf16).astype(np.float64)))
+    down = linear(h, ops_down, precision)
+    return {"Y_up": up["Y"], "y_up_bf16": y_up_bf16, "h_bf16": h, "codes_h": down["codes_x"],
+            "scales_h": down["scales_x"], "T_h": down["T"], "Y": down["Y"]}
 
 
 def exact_linear(X_bf16: np.ndarray, W_bf16: np.ndarray, bias_bf16: Optional[np.ndarray]) -> np.ndarray:

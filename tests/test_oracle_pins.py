@@ -624,3 +624,109 @@ def test_rotary_scores_depend_on_relative_position_only():
     s2 = float(q[2] @ k[3])
     assert abs(s1 - s2) <= 1e-12 * max(1.0, abs(s1))
     assert abs(float(q[0] @ k[0]) - float(q[1] @ k[1])) <= 1e-12 * max(1.0, abs(float(q[0] @ k[0])))
+
+
+# ---------------------------------------------------------------- fused GELU/MLP pair
+
+
+def test_gelu_textbook_values():
+    """GELU(x) = x Phi(x) at values of the standard normal distribution function from tables."""
+    table = {1.0: 0.8413447460685429, 2.0: 0.9772498680518208, -0.5: 0.3085375387259869,
+             -1.96: 0.024997895148220435, 0.0: 0.5}
+    for x, phi in table.items():
+        assert abs(float(O.gelu(np.array([x]))[0]) - x * phi) <= 1e-15 * max(1.0, abs(x))
+
+
+def test_gelu_odd_part_is_the_identity():
+    """Phi(x) + Phi(-x) = 1, so GELU(x) - GELU(-x) = x."""
+    x = np.random.default_rng(12).standard_normal(1000) * 5
+    assert np.allclose(O.gelu(x) - O.gelu(-x), x, rtol=0, atol=1e-14 * 20)
+
+
+def test_gelu_against_integrated_density():
+    """Phi(x) = 1/2 + the integral of the normal density from 0 to x (composite Simpson rule)."""
+    for x in (-3.7, -1.2, -0.3, 0.4, 1.5, 3.1):
+        n = 2000
+        t = np.linspace(0.0, x, n + 1)
+        f = np.exp(-0.5 * t * t) / math.sqrt(2 * math.pi)
+        h = x / n
+        integral = h / 3 * (f[0] + f[-1] + 4 * f[1:-1:2].sum() + 2 * f[2:-1:2].sum())
+        assert abs(float(O.gelu(np.array([x]))[0]) - x * (0.5 + integral)) <= 1e-12
+
+
+def test_gelu_minimum():
+    """GELU has one minimum, where Phi(x) + x phi(x) = 0 (x ~ -0.7518); neighbours lie above it."""
+    lo, hi = -1.0, -0.5
+    for _ in range(80):  # bisection on the derivative, written with math.erf
+        mid = 0.5 * (lo + hi)
+        d = 0.5 * (1 + math.erf(mid / math.sqrt(2))) + mid * math.exp(-0.5 * mid * mid) / math.sqrt(2 * math.pi)
+        lo, hi = (mid, hi) if d < 0 else (lo, mid)
+    xs = 0.5 * (lo + hi)
+    assert abs(xs + 0.7517915246935645) < 1e-12
+    g = O.gelu(np.array([xs - 1e-3, xs, xs + 1e-3]))
+    assert g[1] < g[0] and g[1] < g[2]
+
+
+def _bf16_nearest_brute(x: float) -> int:
+    """Nearest bf16 by search over every finite bf16 pattern (ties: even mantissa)."""
+    pats = np.arange(1 << 16, dtype=np.uint32)
+    with np.errstate(invalid="ignore"):
+        vals = (pats << np.uint32(16)).view(np.float32).astype(np.float64)
+    ok = np.isfinite(vals)
+    d = np.where(ok, np.abs(vals - x), np.inf)
+    best = np.min(d)
+    cands = pats[d == best]
+    cands = cands[(cands & 0x7FFF) != 0] if x != 0 else cands  # -0/+0: keep the sign of x below
+    if x == 0:
+        return 0x8000 if math.copysign(1.0, x) < 0 else 0
+    even = cands[(cands & 1) == 0]
+    pick = even if len(even) else cands
+    # the pattern with the sign of x
+    pick = [int(c) for c in pick if ((c >> 15) & 1) == (1 if x < 0 else 0)] or [int(pick[0])]
+    return pick[0]
+
+
+def test_f64_to_bf16_single_rounding():
+    rng = np.random.default_rng(13)
+    x = np.concatenate([rng.standard_normal(40) * 10.0 ** rng.integers(-8, 8, 40),
+                        [9.031250271464623, 1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8), 3.0, -0.0]])
+    got = O.f64_to_bf16(x)
+    for xi, g in zip(x, got):
+        assert int(g) == _bf16_nearest_brute(float(xi)), xi
+    # one step from fp64: 9.031250271... lies above the midpoint 9.03125 of (9.0, 9.0625), which an
+    # fp32 intermediate would hit exactly and round to even (9.0)
+    assert O.bf16_to_f32(O.f64_to_bf16(np.array([9.031250271464623])))[0] == np.float32(9.0625)
+    # on fp32 inputs it agrees with the fp32 rule
+    v = rng.standard_normal(5000).astype(np.float32) * 100
+    assert np.array_equal(O.f64_to_bf16(v.astype(np.float64)), O.f32_to_bf16(v))
+
+
+def test_mlp_pair_is_the_module_sequence():
+    """On layers quantized losslessly (lam = 1, r = 0, on-grid operands) the up layer's output is
+    the exact product; the pair must then be: round to bf16, GELU, round to bf16, down layer."""
+    rng = np.random.default_rng(14)
+    M, K, H, N = 4, 64, 64, 48
+    v, _, _ = _random_on_grid_nvfp4(rng, M, K, 0x20, 0x50)
+    wu, _, _ = _random_on_grid_nvfp4(rng, H, K, 0x20, 0x50)
+    wd, _, _ = _random_on_grid_nvfp4(rng, N, H, 0x20, 0x50)
+    xb = O.f32_to_bf16(v)
+    bu = O.f32_to_bf16(rng.standard_normal(H).astype(np.float32))
+    bd = O.f32_to_bf16(rng.standard_normal(N).astype(np.float32))
+
+    def ops(w, b, k):
+        cw, sw = O.quantize_rows(w, O.NVFP4)
+        return {"inv_lambda": np.ones(k, np.float32), "codes_w": cw, "scales_w": sw,
+                "L1": np.zeros((k, 0), np.uint16), "L2": np.zeros((0, w.shape[0]), np.uint16), "bias": b}
+
+    out = O.mlp_pair(xb, ops(wu, bu, K), ops(wd, bd, H), O.NVFP4)
+    y_up = v.astype(np.float64) @ wu.astype(np.float64).T + O.bf16_to_f32(bu)[None, :]
+    assert np.array_equal(out["Y_up"], y_up)
+    h = np.zeros((M, H), np.uint16)
+    for m in range(M):
+        for j in range(H):
+            a = float(O.bf16_to_f32(np.array([_bf16_nearest_brute(float(y_up[m, j]))], np.uint16))[0])
+            g = a * 0.5 * (1.0 + math.erf(a / math.sqrt(2.0)))
+            h[m, j] = _bf16_nearest_brute(g)
+    assert np.array_equal(out["h_bf16"], h)
+    down = O.linear(h, ops(wd, bd, H), O.NVFP4)
+    assert np.array_equal(out["Y"], down["Y"]) and np.array_equal(out["codes_h"], down["codes_x"])
