@@ -2,20 +2,22 @@
 // Design" (b): Down Projection fused with Quantize because they read the same input; Up
 // Projection fused with 4-Bit Compute because they write the same output), for sm_100a.
 //
-// Kernel 1, quant_down: one CTA per (128-row M tile, K slice); the K slices of one M tile form
-// a thread-block cluster.  Eight worker warps stream X from HBM once, apply the smoothing
-// factor, quantize every K-group (NVFP4: UE4M3 scale per 16; INT4: fp32 scale per 64) into the
-// tiled layouts kernel 2 copies verbatim, and stage bf16(x_hat) in shared memory; one warp feeds
-// it with L1 to tcgen05 bf16 MMAs that accumulate T = x_hat L1 in tensor memory.  The cluster
-// reduces its fp32 partials of T through distributed shared memory in a fixed order (so the
-// result is deterministic) and writes bf16 T once.
+// Kernel 1, quant_down: one CTA per (128-row M tile, K slice).  A TMA warp streams X (and the
+// stage's 1/lambda) into a ring of shared-memory stages; sixteen worker warps apply the smoothing
+// factor and quantize every K-group (NVFP4: UE4M3 scale per 16; INT4: fp32 scale per 64) into
+// the tiled layouts kernel 2 copies verbatim, and write bf16(x_hat) back into the stage; one warp
+// feeds it with L1 to tcgen05 bf16 MMAs that accumulate T = x_hat L1 in tensor memory.  When K
+// is split over several CTAs, each writes its fp32 partial of T and counts itself in the tile's
+// counter; the last to arrive adds the partials in slice order (so the result is deterministic)
+// and writes bf16 T once.
 //
-// Kernel 2, gemm: persistent, warp specialised.  Warp 0 streams each (k-block) stage with 1-D
-// bulk copies (the operands are stored as shared-memory images); warp 1 issues the tcgen05 MMAs:
-// first the bf16 up projection T L2 (kind::f16) and then the block-scaled 4-bit GEMM
-// (kind::mxf4nvf4 with UE4M3 scales copied into tensor memory by tcgen05.cp) into the same fp32
-// accumulator in tensor memory; eight epilogue warps drain the accumulator, add the bias and
-// write bf16 Y once.
+// Kernel 2, gemm (NVFP4): persistent, warp specialised, on pairs of CTAs (cta_group::2 MMAs on
+// 256 x 256 tiles).  Two producer threads stream each k-block stage (operand tiles and scale
+// tiles) by TMA; four scale warps write the stage's UE4M3 scales into tensor memory with
+// tcgen05.st; the MMA thread of the leader CTA issues the block-scaled 4-bit MMAs
+// (kind::mxf4nvf4) and the bf16 up projection T L2 (kind::f16) into one fp32 accumulator in
+// tensor memory; eight epilogue warps drain it, add the bias and write bf16 Y once by TMA.
+// Kernel 2, gemm (INT4): as described at its own section below.
 #include <cuda.h>
 #include <atomic>
 #include <mutex>
