@@ -169,7 +169,8 @@ svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int
  * wrong results, so order them on one stream or use svdq_linear_forward with separate
  * workspaces.  Nothing in the array has to start at zero.  Shapes whose workspace
  * (svdq_workspace_size) exceeds 20 MiB are rejected with SVDQ_ERR_INVALID_ARG; at K = 3072 and
- * rank 32 that allows every M up to 9984.  Other arguments and errors as svdq_linear_forward. */
+ * rank 32 that allows every M up to 9984.  A W4A16 layer uses no scratch and has no such limit.
+ * Other arguments and errors as svdq_linear_forward. */
 svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
                                         void* stream);
 

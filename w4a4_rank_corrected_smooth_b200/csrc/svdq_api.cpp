@@ -433,7 +433,7 @@ svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, in
   if (!w) return fail(SVDQ_ERR_INVALID_ARG, "weights handle is NULL");
   if (M < 0) return fail(SVDQ_ERR_INVALID_ARG, "M=%d is negative", M);
   if (M == 0) return SVDQ_OK;
-  const size_t need = svdq::workspace_layout(M, w->K, w->rank).total;
+  const size_t need = w->precision == SVDQ_W4A16 ? 0 : svdq::workspace_layout(M, w->K, w->rank).total;
   const size_t have = svdq::noalloc_scratch_bytes();
   if (need > have)
     return fail(SVDQ_ERR_INVALID_ARG,
