@@ -638,7 +638,10 @@ def run_ours(args):
                        "pipeline": "3 streams (copy in, forward, copy out), 2 device buffer sets"}
         if world == 1:
             line["cpu_baseline"] = oracle_cpu_baseline(X, lin.export_weights(), args.precision, spec)
-            line["w4a16_modulation"] = w4a16_leg(dev, stream, peaks, peak_src)
+            try:  # an auxiliary leg: its failure is reported in the line, not fatal to it
+                line["w4a16_modulation"] = w4a16_leg(dev, stream, peaks, peak_src)
+            except Exception as exc:  # noqa: BLE001
+                line["w4a16_modulation"] = {"error": f"{type(exc).__name__}: {exc}"}
     for l in layers:
         l.close()
     if world > 1:
