@@ -64,3 +64,21 @@ def test_noalloc_forward_rejects_shapes_beyond_the_fixed_scratch():
         lin.svdq_linear_forward_noalloc(Xd, M, spec.K, Y, spec.N)
     assert ei.value.status == 1 and "fixed scratch" in str(ei.value)
     lin.close()
+
+
+def test_noalloc_w4a16_needs_no_scratch_and_has_no_row_limit():
+    """The W4A16 layer's one kernel uses no scratch: the allocation-free forward takes any M (here
+    beyond the W4A4 layer's 20 MiB limit) and equals the ordinary forward bit for bit."""
+    spec = synth.custom("noalloc_w4a16", M=64, K=3072, N=256, rank=0, seed=23)
+    Xs = synth.activations_bf16(spec)
+    lin = S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(Xs), "w4a16", 0)
+    M = 12000
+    X = np.tile(Xs, (M // 64 + 1, 1))[:M]
+    Xd = _bf16_dev(X)
+    Y_ref = lin.forward(Xd)
+    Y = torch.full((M, spec.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lin.svdq_linear_forward_noalloc(Xd, M, spec.K, Y, spec.N)
+    torch.cuda.synchronize()
+    S.svdq_get_device_error()
+    assert torch.equal(Y.view(torch.int16), Y_ref.view(torch.int16))
+    lin.close()
