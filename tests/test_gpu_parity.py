@@ -178,6 +178,23 @@ def test_forward_edge_shapes(M, K, N, r, prec):
     check_y(Y, O.linear(X, ops, prec)["Y"])
 
 
+@pytest.mark.parametrize("prec", ["nvfp4", "int4"])
+def test_forward_padded_x_stride(prec):
+    """X as rows of a wider buffer (row stride K + 64 elements, the padding filled with large
+    values that must not leak in): Y bit-identical to the forward of the contiguous X."""
+    spec = synth.custom("x_stride", M=300, K=512, N=512, rank=32, seed=33)
+    X, W, b, lin = make_layer(spec, prec)
+    Y_ref = run_forward(lin, X)
+    buf = torch.full((spec.M, spec.K + 64), 1000.0, dtype=torch.bfloat16, device="cuda")
+    buf[:, :spec.K] = to_dev_bf16(X)
+    ws = lin.new_workspace(spec.M)
+    Y = torch.full((spec.M, spec.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lin.svdq_linear_forward(buf, spec.M, buf.stride(0), Y, Y.stride(0), ws, ws.numel())
+    S.svdq_get_device_error()
+    assert torch.equal(Y.view(torch.int16), Y_ref.view(torch.int16))
+    lin.close()
+
+
 def test_forward_m_zero_is_noop():
     spec = synth.custom("m0", M=16, K=256, N=256, rank=16)
     X, W, b, lin = make_layer(spec, "nvfp4")
