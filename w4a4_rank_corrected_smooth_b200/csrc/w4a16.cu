@@ -68,6 +68,7 @@ __global__ void __launch_bounds__(256) w4a16_kernel(const W4A16Params p) {
     float acc[MT];
 #pragma unroll
     for (int mi = 0; mi < MT; ++mi) acc[mi] = 0.0f;
+#pragma unroll 4
     for (int k0 = lane * 8; k0 < p.K; k0 += 256) {
       const uint32_t c = __ldg(crow + k0 / 8);  // elements k0 .. k0 + 7, element j in nibble j
       const float s = __ldg(srow + k0 / 64);
