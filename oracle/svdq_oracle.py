@@ -512,13 +512,54 @@ def gelu(y: np.ndarray) -> np.ndarray:
     return 0.5 * y * (1.0 + erf(y / np.sqrt(2.0)))
 
 
+_GELU_BF16 = {}
+
+
+def gelu_bf16(y_bf16: np.ndarray) -> np.ndarray:
+    """bf16 GELU of bf16 inputs: y Phi(y) evaluated to 50 significant digits (mpmath, with
+    Phi(y) = erfc(-y / sqrt 2) / 2, free of the cancellation of 1 + erf in the negative tail) and
+    rounded once to the nearest bf16, ties to even (R11).  A bf16 input has 2^16 patterns, so the
+    values are computed once per distinct pattern and cached."""
+    import mpmath
+
+    y_bf16 = np.asarray(y_bf16, dtype=np.uint16)
+    uniq = np.unique(y_bf16)
+    todo = [int(u) for u in uniq if int(u) not in _GELU_BF16]
+    if todo:
+        with mpmath.workdps(50):
+            two = mpmath.mpf(2)
+            for u in todo:
+                y = mpmath.mpf(float(bf16_to_f32(np.array([u], np.uint16))[0]))
+                _GELU_BF16[u] = _mp_to_bf16(y * mpmath.erfc(-y / mpmath.sqrt(two)) / two)
+    lut = np.array([_GELU_BF16[int(u)] for u in uniq], dtype=np.uint16)
+    return lut[np.searchsorted(uniq, y_bf16)]
+
+
+def _mp_to_bf16(g) -> int:
+    """Nearest bf16 (ties to even) of a high-precision value: 8 significant bits for normal
+    magnitudes, spacing 2^-133 below 2^-126 (subnormals)."""
+    import mpmath
+
+    if g == 0:
+        return 0x8000 if mpmath.sign(g) < 0 else 0
+    a = abs(g)
+    q = max(int(mpmath.floor(mpmath.log(a, 2))), -126) - 7  # exponent of the bf16 spacing at a
+    m = a / mpmath.mpf(2) ** q  # in [2^7, 2^8) for normal a
+    n = int(mpmath.floor(m))
+    frac = m - n
+    if frac > 0.5 or (frac == 0.5 and n % 2 == 1):
+        n += 1
+    bits = int(np.array([np.float32(n * 2.0 ** q)], np.float32).view(np.uint32)[0] >> 16)
+    return bits | (0x8000 if g < 0 else 0)
+
+
 def mlp_pair(X_bf16: np.ndarray, ops_up: Dict[str, np.ndarray], ops_down: Dict[str, np.ndarray],
              precision: str) -> Dict[str, np.ndarray]:
     """up layer -> bf16 -> GELU -> bf16 -> down layer (R11).  Returns the up layer's exact output,
     the bf16 hidden activation, the down layer's 4-bit operands and T, and Y (fp64)."""
     up = linear(X_bf16, ops_up, precision)
     y_up_bf16 = f64_to_bf16(up["Y"])
-    h = f64_to_bf16(gelu(bf16_to_f32(y_up_bf16).astype(np.float64)))
+    h = gelu_bf16(y_up_bf16)
     down = linear(h, ops_down, precision)
     return {"Y_up": up["Y"], "y_up_bf16": y_up_bf16, "h_bf16": h, "codes_h": down["codes_x"],
             "scales_h": down["scales_x"], "T_h": down["T"], "Y": down["Y"]}

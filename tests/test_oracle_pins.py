@@ -379,6 +379,26 @@ def test_lowrank_branch_hand_computed():
     assert T0.shape == (1, 0)
 
 
+def test_lowrank_down_rounds_x_hat_to_bf16_before_the_product():
+    """The 16-bit branch multiplies bf16(x_hat), not x_hat: with x_hat = [1 + d, -1] and L1 = [[1, 2],
+    [1, 2]], T = [bf16(1 + d) - 1, 2 (bf16(1 + d) - 1)], worked out by hand on the bf16 grid (spacing
+    2^-7 on [1, 2)).  A branch that skipped the rounding would give d itself; one that rounded ties
+    away from zero would give 2^-7 for the tie d = 2^-8."""
+    d = np.array([2.0 ** -9, 3 * 2.0 ** -9, 2.0 ** -8, 3 * 2.0 ** -8, 2.0 ** -7 + 2.0 ** -10], np.float64)
+    # nearest bf16 of 1 + d: below / above the midpoint, a tie to the even neighbour 1.0, a tie to
+    # the even neighbour 1 + 2^-6, exactly 1 + 2^-7 plus less than half a spacing
+    t0 = np.array([0.0, 2.0 ** -7, 0.0, 2.0 ** -6, 2.0 ** -7])
+    x = np.zeros((len(d), 16), np.float32)
+    x[:, 0] = (1.0 + d).astype(np.float32)
+    x[:, 1] = -1.0
+    assert np.all(x[:, 0].astype(np.float64) == 1.0 + d)  # the inputs are exact in fp32
+    L1 = np.zeros((16, 2), np.float32)
+    L1[0] = L1[1] = [1.0, 2.0]
+    T = O.bf16_to_f32(O.lowrank_down(x, O.f32_to_bf16(L1))).astype(np.float64)
+    assert np.array_equal(T[:, 0], t0)
+    assert np.array_equal(T[:, 1], 2 * t0)
+
+
 def test_prepare_and_linear_reconstruct_exact_at_full_rank():
     """Full rank: L1 L2 reproduces W_hat, so the low-rank branch alone (with W's 4-bit
     part ~0) approximates X W^T to bf16 precision -- pins the orientation of L1/L2."""
@@ -676,8 +696,7 @@ def _bf16_nearest_brute(x: float) -> int:
     d = np.where(ok, np.abs(vals - x), np.inf)
     best = np.min(d)
     cands = pats[d == best]
-    cands = cands[(cands & 0x7FFF) != 0] if x != 0 else cands  # -0/+0: keep the sign of x below
-    if x == 0:
+    if x == 0 or np.all((cands & 0x7FFF) == 0):  # x itself, or its nearest, is zero: zero of x's sign
         return 0x8000 if math.copysign(1.0, x) < 0 else 0
     even = cands[(cands & 1) == 0]
     pick = even if len(even) else cands
@@ -699,6 +718,36 @@ def test_f64_to_bf16_single_rounding():
     # on fp32 inputs it agrees with the fp32 rule
     v = rng.standard_normal(5000).astype(np.float32) * 100
     assert np.array_equal(O.f64_to_bf16(v.astype(np.float64)), O.f32_to_bf16(v))
+
+
+def test_gelu_bf16_every_input():
+    """The bf16 GELU on all 65280 finite bf16 inputs.  (1) Wherever |y| >= 2^-125 it equals the fp64
+    y Phi(y) = y erfc(-y / sqrt 2) / 2 (library erfc, relative error ~1e-15) rounded once to bf16:
+    none of those exact values lies within 1e-12 (relative) of a bf16 rounding boundary, so fp64
+    decides every one of them.  (2) Below that, y / 2 is exact and GELU(y) = y / 2 + y^2 / sqrt
+    (2 pi) + O(y^4) lies just above it; y / 2 is a bf16 subnormal there (spacing 2^-133), so the
+    result is y / 2 rounded with ties upward.  (3) The
+    fp64 form 1 + erf(y / sqrt 2) cancels in the negative tail (it returns 0 below y ~ -8.3), and the
+    bf16 GELU must not follow it there."""
+    from scipy.special import erfc
+
+    pats = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    y = O.bf16_to_f32(pats).astype(np.float64)
+    fin = np.isfinite(y)
+    pats, y = pats[fin], y[fin]
+    got = O.gelu_bf16(pats)
+    g64 = 0.5 * y * erfc(-y / math.sqrt(2.0))
+    normal = np.abs(y) >= 2.0 ** -125
+    assert np.array_equal(got[normal], O.f64_to_bf16(g64[normal]))
+    sub = ~normal & (y != 0)
+    half = y[sub] / 2  # exact: a multiple of 2^-134
+    k = half / 2.0 ** -133  # in units of the bf16 subnormal spacing
+    expect = np.where(k - np.floor(k) == 0.5, np.ceil(k), np.round(k)) * 2.0 ** -133
+    assert np.array_equal(O.bf16_to_f32(got[sub]).astype(np.float64), expect)
+    assert np.all(O.bf16_to_f32(got[y == 0]) == 0)
+    tail = (y < -8.5) & (y > -13.0)
+    assert np.all(O.bf16_to_f32(got[tail]) < 0)  # small but not zero
+    assert np.all(0.5 * y[tail] * (1.0 + np.array([math.erf(v / math.sqrt(2.0)) for v in y[tail]])) == 0)
 
 
 def test_mlp_pair_is_the_module_sequence():
@@ -725,7 +774,7 @@ def test_mlp_pair_is_the_module_sequence():
     for m in range(M):
         for j in range(H):
             a = float(O.bf16_to_f32(np.array([_bf16_nearest_brute(float(y_up[m, j]))], np.uint16))[0])
-            g = a * 0.5 * (1.0 + math.erf(a / math.sqrt(2.0)))
+            g = a * 0.5 * math.erfc(-a / math.sqrt(2.0))  # Phi without 1 + erf's cancellation
             h[m, j] = _bf16_nearest_brute(g)
     assert np.array_equal(out["h_bf16"], h)
     down = O.linear(h, ops(wd, bd, H), O.NVFP4)
