@@ -524,6 +524,7 @@ def gelu_bf16(y_bf16: np.ndarray) -> np.ndarray:
 
     y_bf16 = np.asarray(y_bf16, dtype=np.uint16)
     uniq = np.unique(y_bf16)
+    _GELU_BF16[0x8000] = 0x8000  # y Phi(y) of -0 is -0 (a product with a negative zero)
     todo = [int(u) for u in uniq if int(u) not in _GELU_BF16]
     if todo:
         with mpmath.workdps(50):

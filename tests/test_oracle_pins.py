@@ -745,6 +745,7 @@ def test_gelu_bf16_every_input():
     expect = np.where(k - np.floor(k) == 0.5, np.ceil(k), np.round(k)) * 2.0 ** -133
     assert np.array_equal(O.bf16_to_f32(got[sub]).astype(np.float64), expect)
     assert np.all(O.bf16_to_f32(got[y == 0]) == 0)
+    assert list(O.gelu_bf16(np.array([0x0000, 0x8000], np.uint16))) == [0x0000, 0x8000]  # sign of zero kept
     tail = (y < -8.5) & (y > -13.0)
     assert np.all(O.bf16_to_f32(got[tail]) < 0)  # small but not zero
     assert np.all(0.5 * y[tail] * (1.0 + np.array([math.erf(v / math.sqrt(2.0)) for v in y[tail]])) == 0)
