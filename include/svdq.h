@@ -163,16 +163,64 @@ svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int
  * device) is not acceptable.  The scratch between the two kernels is a fixed 20 MiB array in the
  * library's own device module, which every GPU that loads the library keeps until the process
  * exits.  The first call on a device looks up that array's device address (cudaGetSymbolAddress,
- * with the device current) and caches it; make that first call before any stream capture.
+ * with the device current) and caches it; make that first call before any stream capture.  The
+ * cache is keyed by the device's current context as well, so after cudaDeviceReset the next call
+ * looks the address up again (in the new context, again before any capture).
  * All calls on a device share the one array and it keeps the contents of the last call: calls
  * whose kernels overlap on the GPU (different streams, no ordering between them) race and give
  * wrong results, so order them on one stream or use svdq_linear_forward with separate
  * workspaces.  Nothing in the array has to start at zero.  Shapes whose workspace
- * (svdq_workspace_size) exceeds 20 MiB are rejected with SVDQ_ERR_INVALID_ARG; at K = 3072 and
- * rank 32 that allows every M up to 9984.  A W4A16 layer uses no scratch and has no such limit.
+ * (svdq_workspace_size) exceeds 20 MiB are rejected with SVDQ_ERR_INVALID_ARG: the row limit is
+ * the largest M whose svdq_workspace_size fits in 20 MiB (at K = 3072 and rank 32 today every M
+ * up to 9984; it moves with the workspace layout, so query svdq_workspace_size rather than
+ * relying on that figure).  A W4A16 layer uses no scratch and has no such limit.
  * Other arguments and errors as svdq_linear_forward. */
 svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
                                         void* stream);
+
+/* The grouped QKV projection with its Q/K normalization and rotary embedding in one operator
+ * ([ND] "Quantizing models with structural rewrites": the fused operator consumes the QKV
+ * projection, norm_q, norm_k and the rotary embedding; Q, K and V are concatenated along the
+ * output dimension in that order).  The pages name the steps only; the library reads them as:
+ * the layer's output row (before its rounding to bf16) holds H heads of Q, then H of K, then H
+ * of V, `head_dim` channels each; every Q and K head vector x becomes
+ *   x / sqrt(mean(x^2) + eps) * gamma   (RMS normalization, gamma_q for Q, gamma_k for K),
+ * and then each channel pair (2i, 2i+1) of it is turned by the row's angle i:
+ *   (a, b) -> (a cos - b sin, a sin + b cos);
+ * V passes unchanged.  Y is rounded to bf16 once, as in svdq_linear_forward.
+ * The normalization and rotation run in the epilogue of kernel 2 (NVFP4: one thread holds one
+ * row of one head; INT4: half of it, the two halves exchanging their sums of squares).  NVFP4 or
+ * INT4 layer, head_dim = 128 and N a multiple of 3 * 128.
+ * gamma_q, gamma_k: device, head_dim fp32 each, 16-byte aligned.
+ * rope: device, M rows of head_dim/2 (cos, sin) fp32 pairs (row stride head_dim floats),
+ *       16-byte aligned: row m holds the angles of token m.
+ * eps:  >= 0 and finite (FLUX uses 1e-6).
+ * Other arguments, workspace rules and errors as svdq_linear_forward; INVALID_ARG also for a
+ * W4A16 layer, another head_dim, N not a multiple of 3 * head_dim, or a bad pointer. */
+svdq_status svdq_linear_forward_qkv_norm_rope(const svdq_weights* w, const void* X, int M, int ldx, void* Y,
+                                              int ldy, const float* gamma_q, const float* gamma_k, float eps,
+                                              const float* rope, int head_dim, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+
+/* The fused MLP pair ([ND] "Introducing Nunchaku Lite": fused GELU/MLP kernels; the pages give no
+ * formula).  The library reads it as the unfused module sequence: Y = down(h) with
+ *   h = bf16(GELU(bf16(up(X)))),  GELU(x) = x Phi(x) (Phi the standard normal distribution),
+ * fused so that h never goes through memory: the up layer's kernel 2 computes h in its epilogue
+ * and writes, instead of its output, the down layer's activation codes and scales of h and the
+ * fp32 partials of the down layer's T (warp-level bf16 MMAs per half tile); a small kernel adds
+ * the partials in a fixed order into T; the down layer's kernel 2 then runs as usual.  GELU is
+ * computed in fp32 (erff), so h can differ from an exact evaluation by one bf16 ulp where the
+ * value sits on a rounding boundary.
+ * Both layers NVFP4, up->N == down->K, the down layer's rank 0, 16 or 32, same device.
+ * ws_up: the up layer's workspace (svdq_workspace_size(up, M)).  ws_mid: the down layer's
+ * workspace followed by the T partials, svdq_mlp_workspace_size(up, down, M) bytes, 256-byte
+ * aligned (after the call it holds the down layer's kernel-1 outputs: svdq_export_activations
+ * (down, ws_mid, ...) reads them).  Y: M x down->N bf16, row stride ldy.
+ * No allocation, no synchronisation.  Errors: INVALID_ARG, CUDA. */
+svdq_status svdq_mlp_workspace_size(const svdq_weights* up, const svdq_weights* down, int M, size_t* bytes);
+svdq_status svdq_mlp_forward(const svdq_weights* up, const svdq_weights* down, const void* X, int M, int ldx,
+                             void* Y, int ldy, void* ws_up, size_t ws_up_bytes, void* ws_mid,
+                             size_t ws_mid_bytes, void* stream);
 
 /* Kernel 1 alone (same arguments as the forward minus Y): fills the workspace. */
 svdq_status svdq_quant_down(const svdq_weights* w, const void* X, int M, int ldx, void* workspace,
@@ -209,6 +257,14 @@ svdq_status svdq_prepare_host(const uint16_t* W_bf16, int N, int K, const uint16
  * it sets the device error word and returns.  Lets a test check that a wait that runs out
  * is reported as SVDQ_ERR_TIMEOUT by svdq_get_device_error while the context stays usable. */
 svdq_status svdq_selftest_wait_timeout(int spin_limit, void* stream);
+
+/* The bf16 GELU of the fused MLP pair's epilogue (svdq_mlp_forward), applied to n bf16 values:
+ * out[i] = the nearest bf16 (ties to even) of y Phi(y), y = in[i], Phi the standard normal
+ * distribution function ([ND] "Introducing Nunchaku Lite": fused GELU/MLP kernels; the library
+ * reads GELU as the exact erf form).  in, out: device, n uint16 bf16 patterns each; asynchronous
+ * on `stream`.  A test hook: a bf16 input has only 2^16 values, so a test can check the epilogue's
+ * GELU on every one of them.  Errors: INVALID_ARG (n < 0, NULL buffer with n > 0), CUDA. */
+svdq_status svdq_selftest_gelu_bf16(const uint16_t* in, uint16_t* out, int n, void* stream);
 
 #ifdef __cplusplus
 }

@@ -15,6 +15,7 @@ import pytest
 
 import synth
 from oracle import svdq_oracle as O
+from tbound import assert_t_close
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -48,6 +49,9 @@ def _check_rows(lin, X, Y, act, rows, prec, ops):
     assert np.array_equal(act["codes_x"][rows], cx), "activation codes differ from the oracle"
     assert np.array_equal(act["scales_x"][rows], sx), "activation scales differ from the oracle"
     T = O.lowrank_down(xh, ops["L1"])
+    if lin.rank:
+        assert_t_close(O.bf16_to_f32(act["T"][rows]).astype(np.float64), O.bf16_to_f32(T).astype(np.float64),
+                       O.bf16_to_f32(O.f32_to_bf16(xh)), O.bf16_to_f32(ops["L1"]))
     ref = O.forward(cx, sx, T, ops["codes_w"], ops["scales_w"], ops["L2"], ops["bias"], prec)
     got = O.bf16_to_f32(Y[torch.from_numpy(rows).cuda()].view(torch.int16).cpu().numpy().view(np.uint16)).astype(np.float64)
     assert np.all(np.isfinite(got))

@@ -3,8 +3,9 @@ low-rank branch) through the C ABI against the oracle's fp64 forward over the li
 operands.
 
 Cases: FLUX's modulation projections (one token per image: M = 1 ... 5 rows, K = 3072,
-N = 18432 and 9216), a ragged small layer with padded row strides, and a tall input that the
-launcher splits over several grids.  Bar as for the W4A4 layer: relative Frobenius error 5e-3 and
+N = 18432 and 9216) and M = 12, 16, 40 (the 16-row passes), a long K (several staged chunks), a
+ragged small layer with padded row strides, and a tall input that the launcher splits over
+several grids.  Bar as for the W4A4 layer: relative Frobenius error 5e-3 and
 max|dY| <= 1e-2 max|Y_ref|.
 """
 import numpy as np
@@ -68,6 +69,24 @@ def test_modulation_projection(M, N):
     lin.close()
 
 
+@pytest.mark.parametrize("M", [12, 16, 40])
+def test_sixteen_row_passes(M):
+    spec = synth.custom("w4a16_m16", M=M, K=3072, N=1024, rank=0, seed=21)
+    X = synth.activations_bf16(spec)
+    lin = S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(X), "w4a16", 0)
+    _check(_y64(_run(lin, X)), O.linear_w4a16(X, lin.export_weights())["Y"])
+    lin.close()
+
+
+def test_long_k_in_several_chunks():
+    # K = 16384: 256 groups, more than one staging of the activation fragments holds
+    spec = synth.custom("w4a16_longk", M=3, K=16384, N=512, rank=0, seed=22)
+    X = synth.activations_bf16(spec)
+    lin = S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(X), "w4a16", 0)
+    _check(_y64(_run(lin, X)), O.linear_w4a16(X, lin.export_weights())["Y"])
+    lin.close()
+
+
 def test_ragged_with_padded_strides():
     # K = 768 (three 256-element passes per warp), N = 40, M = 9 (a partial tile of 4 rows), row
     # strides padded (X by 24 elements, Y by 8)
@@ -94,16 +113,17 @@ def test_without_bias_and_zero_rows():
 
 
 def test_tall_input_over_several_grids():
-    # 262147 rows: more row tiles than one grid holds, so the launcher splits the rows; rows are
-    # independent, so sampled rows (both sides of each split) are an exact check.
+    # 16 * 65535 + 19 rows: more 16-row passes than one grid holds, so the launcher splits the rows;
+    # rows are independent, so sampled rows (both sides of the split) are an exact check.
     spec = synth.custom("w4a16_tall", M=1024, K=256, N=24, rank=0, seed=8)
     Xs = synth.activations_bf16(spec)
     lin = S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(Xs), "w4a16", 0)
     ops = lin.export_weights()
-    M = 262147
+    M = 16 * 65535 + 19
     X = np.tile(Xs, (M // 1024 + 1, 1))[:M]
     Y = _run(lin, X)
-    rows = np.array([0, 1, 1023, 131072, 262139, 262140, 262141, 262143, 262144, 262146])
+    split = 16 * 65535
+    rows = np.array([0, 1, 1023, 131072, split - 17, split - 1, split, split + 1, split + 8, M - 1])
     ref = O.linear_w4a16(Xs[rows % 1024], ops)["Y"]
     _check(_y64(Y, rows), ref)
     lin.close()

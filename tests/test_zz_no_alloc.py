@@ -49,6 +49,8 @@ def test_noalloc_forward_matches_workspace_forward_on_two_calls():
         assert np.all(np.isfinite(got))
         assert O.rel_fro(got, ref) <= REL_FRO_TOL
         assert np.max(np.abs(got - ref)) <= MAX_ABS_TOL * np.max(np.abs(ref))
+        # the same deterministic kernels on the same operands: identical bits, not just close
+        assert torch.equal(Y.view(torch.int16), Y_ws.view(torch.int16))
     lin.close()
 
 
@@ -56,8 +58,20 @@ def test_noalloc_forward_rejects_shapes_beyond_the_fixed_scratch():
     spec = synth.custom("noalloc_big", M=16, K=3072, N=256, rank=32, seed=22)
     X = synth.activations_bf16(spec)
     lin = S.SVDQLinear(synth.weight_bf16(spec), None, synth.act_absmax(X), "nvfp4", spec.rank)
-    M = 9985  # first M at K = 3072, rank 32 whose workspace exceeds 20 MiB
-    assert lin.workspace_size(M) > 20 << 20 >= max(lin.workspace_size(m) for m in (1, 4608, 9216, 9984))
+    # the row limit is the largest M whose workspace fits the 20 MiB scratch, found from the
+    # library's own svdq_workspace_size (it moves with the workspace layout)
+    lo, hi = 1, 1 << 20
+    assert lin.workspace_size(lo) <= 20 << 20 < lin.workspace_size(hi)
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        lo, hi = (mid, hi) if lin.workspace_size(mid) <= 20 << 20 else (lo, mid)
+    M = hi  # the first M that no longer fits
+    assert all(lin.workspace_size(m) <= 20 << 20 for m in (1, lo // 2, lo))
+    Yok = torch.zeros((lo, spec.N), dtype=torch.bfloat16, device="cuda")
+    lin.svdq_linear_forward_noalloc(torch.zeros((lo, spec.K), dtype=torch.bfloat16, device="cuda"), lo, spec.K,
+                                    Yok, spec.N)
+    torch.cuda.synchronize()
+    S.svdq_get_device_error()
     Xd = torch.zeros((M, spec.K), dtype=torch.bfloat16, device="cuda")
     Y = torch.zeros((M, spec.N), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(S.SVDQError) as ei:

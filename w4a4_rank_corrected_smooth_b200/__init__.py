@@ -60,12 +60,16 @@ def _load() -> ctypes.CDLL:
         "svdq_workspace_size": ([vp, i, ctypes.POINTER(sz)], i),
         "svdq_linear_forward": ([vp, vp, i, i, vp, i, vp, sz, vp], i),
         "svdq_linear_forward_noalloc": ([vp, vp, i, i, vp, i, vp], i),
+        "svdq_linear_forward_qkv_norm_rope": ([vp, vp, i, i, vp, i, vp, vp, ctypes.c_float, vp, i, vp, sz, vp], i),
+        "svdq_mlp_workspace_size": ([vp, vp, i, ctypes.POINTER(sz)], i),
+        "svdq_mlp_forward": ([vp, vp, vp, i, i, vp, i, vp, sz, vp, sz, vp], i),
         "svdq_quant_down": ([vp, vp, i, i, vp, sz, vp], i),
         "svdq_gemm_up": ([vp, i, vp, i, vp, sz, vp], i),
         "svdq_export_activations": ([vp, vp, sz, i, vp, vp, vp, vp], i),
         "svdq_quantize_rows_host": ([vp, i, i, i, vp, vp], i),
         "svdq_prepare_host": ([vp, i, i, vp, vp, ctypes.POINTER(PrepareParams), vp, vp, vp, vp, vp, vp, vp], i),
         "svdq_selftest_wait_timeout": ([i, vp], i),
+        "svdq_selftest_gelu_bf16": ([vp, vp, i, vp], i),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -78,8 +82,9 @@ _lib = _load()
 DECLARED_SYMBOLS = tuple(sorted([
     "svdq_status_string", "svdq_last_error", "svdq_check_device", "svdq_get_device_error", "svdq_prepare_weights",
     "svdq_free_weights", "svdq_clone_weights", "svdq_get_weights_info", "svdq_export_weights", "svdq_workspace_size", "svdq_linear_forward", "svdq_linear_forward_noalloc",
+    "svdq_linear_forward_qkv_norm_rope", "svdq_mlp_workspace_size", "svdq_mlp_forward",
     "svdq_quant_down", "svdq_gemm_up", "svdq_export_activations", "svdq_quantize_rows_host", "svdq_prepare_host",
-    "svdq_selftest_wait_timeout"]))
+    "svdq_selftest_wait_timeout", "svdq_selftest_gelu_bf16"]))
 
 
 def lib() -> ctypes.CDLL:
@@ -128,6 +133,11 @@ def svdq_get_device_error(stream=None) -> None:
 
 def svdq_selftest_wait_timeout(spin_limit: int, stream=None) -> None:
     _check(_lib.svdq_selftest_wait_timeout(spin_limit, _stream(stream)))
+
+
+def svdq_selftest_gelu_bf16(inp, out, n: int, stream=None) -> None:
+    """The fused MLP epilogue's bf16 GELU on ``n`` bf16 patterns (device tensors of 16-bit ints)."""
+    _check(_lib.svdq_selftest_gelu_bf16(_ptr(inp), _ptr(out), n, _stream(stream)))
 
 
 def svdq_quantize_rows_host(V: np.ndarray, precision):
@@ -245,6 +255,14 @@ class SVDQLinear:
         (for callers that cannot allocate device memory; see include/svdq.h)."""
         _check(_lib.svdq_linear_forward_noalloc(self._h, _ptr(X), M, ldx, _ptr(Y), ldy, _stream(stream)))
 
+    def svdq_linear_forward_qkv_norm_rope(self, X, M: int, ldx: int, Y, ldy: int, gamma_q, gamma_k, eps: float,
+                                          rope, head_dim: int, workspace, workspace_bytes: int, stream=None):
+        """The grouped QKV layer with RMS normalization of the Q and K heads and the rotary
+        embedding fused into its epilogue (device pointers; see include/svdq.h)."""
+        _check(_lib.svdq_linear_forward_qkv_norm_rope(self._h, _ptr(X), M, ldx, _ptr(Y), ldy, _ptr(gamma_q),
+                                                      _ptr(gamma_k), float(eps), _ptr(rope), head_dim,
+                                                      _ptr(workspace), workspace_bytes, _stream(stream)))
+
     def svdq_quant_down(self, X, M: int, ldx: int, workspace, workspace_bytes: int, stream=None):
         _check(_lib.svdq_quant_down(self._h, _ptr(X), M, ldx, _ptr(workspace), workspace_bytes, _stream(stream)))
 
@@ -285,6 +303,22 @@ class SVDQLinear:
     __call__ = forward
 
 
+def svdq_mlp_workspace_size(up: "SVDQLinear", down: "SVDQLinear", M: int) -> int:
+    """Bytes of the fused MLP pair's middle workspace for M rows (see include/svdq.h)."""
+    out = ctypes.c_size_t()
+    _check(_lib.svdq_mlp_workspace_size(up.handle, down.handle, M, ctypes.byref(out)))
+    return out.value
+
+
+def svdq_mlp_forward(up: "SVDQLinear", down: "SVDQLinear", X, M: int, ldx: int, Y, ldy: int, ws_up, ws_up_bytes: int,
+                     ws_mid, ws_mid_bytes: int, stream=None) -> None:
+    """Y = down(bf16(GELU(bf16(up(X))))) with the hidden activation kept out of memory (device
+    pointers; see include/svdq.h)."""
+    _check(_lib.svdq_mlp_forward(up.handle, down.handle, _ptr(X), M, ldx, _ptr(Y), ldy, _ptr(ws_up), ws_up_bytes,
+                                 _ptr(ws_mid), ws_mid_bytes, _stream(stream)))
+
+
 __all__ = ["SVDQLinear", "SVDQError", "svdq_check_device", "svdq_get_device_error", "svdq_selftest_wait_timeout",
-           "svdq_quantize_rows_host", "svdq_prepare_host", "SVDQ_NVFP4", "SVDQ_INT4", "SVDQ_W4A16", "LIB_PATH", "lib",
-           "DECLARED_SYMBOLS"]
+           "svdq_selftest_gelu_bf16",
+           "svdq_quantize_rows_host", "svdq_prepare_host", "svdq_mlp_workspace_size", "svdq_mlp_forward", "SVDQ_NVFP4",
+           "SVDQ_INT4", "SVDQ_W4A16", "LIB_PATH", "lib", "DECLARED_SYMBOLS"]

@@ -450,4 +450,51 @@ void pack_device_layouts(const CanonicalLayer& c, DeviceImages& d) {
   for (int n = 0; n < N; ++n) d.bias[n] = bf16_bits_to_float(c.bias[n]);
 }
 
+// W4A16 weights in the order the warp-level bf16 MMA (m16n8k16) takes its A operand from
+// registers: per block b of 16 rows and group g of 64 elements along K, 32 lanes x 16 bytes.
+// Lane l (row i = l / 4, pair t = l % 4) holds four 32-bit words, one per 16-deep k-step s;
+// nibble j of word s (j = 0..3) and nibble j + 4 are the two elements of fragment register j:
+//   j = 0: row i,     k = 64 g + 16 s + 2 t + {0, 1}
+//   j = 1: row i + 8, k = 64 g + 16 s + 2 t + {0, 1}
+//   j = 2: row i,     k = 64 g + 16 s + 8 + 2 t + {0, 1}
+//   j = 3: row i + 8, k = 64 g + 16 s + 8 + 2 t + {0, 1}
+// (the element with the lower k in nibble j, the other in nibble j + 4).  Scales: per (b, g)
+// eight pairs (s[16 b + i], s[16 b + i + 8]) as fp32.  Rows past N stay 0 up to the padded N.
+void pack_w4a16_fragments(const CanonicalLayer& c, DeviceImages& d) {
+  const int N = c.N, K = c.K, G = K / 64;
+  const size_t npad = static_cast<size_t>((N + kBN - 1) / kBN) * kBN;
+  const int NB = static_cast<int>(npad / 16);
+  d.codes.assign(npad * K / 2, 0);
+  d.sf.assign(npad * static_cast<size_t>(G) * sizeof(float), 0);
+  auto nib = [&](int n, int k) -> uint32_t {
+    if (n >= N) return 0;
+    const uint8_t byte = c.codes_w[static_cast<size_t>(n) * (K / 2) + k / 2];
+    return (k & 1) ? (byte >> 4) : (byte & 0xFu);
+  };
+  parallel_for(NB, [&](int b, int) {
+    for (int g = 0; g < G; ++g) {
+      uint8_t* dst = d.codes.data() + ((static_cast<size_t>(b) * G + g) * 32) * 16;
+      for (int l = 0; l < 32; ++l) {
+        const int i = l / 4, t = l % 4;
+        for (int s = 0; s < 4; ++s) {
+          uint32_t word = 0;
+          for (int j = 0; j < 4; ++j) {
+            const int n = 16 * b + i + 8 * (j & 1);
+            const int k = 64 * g + 16 * s + 8 * (j >> 1) + 2 * t;
+            word |= nib(n, k) << (4 * j);
+            word |= nib(n, k + 1) << (4 * (j + 4));
+          }
+          std::memcpy(dst + 16 * l + 4 * s, &word, 4);
+        }
+      }
+      float* sdst = reinterpret_cast<float*>(d.sf.data()) + (static_cast<size_t>(b) * G + g) * 16;
+      for (int i = 0; i < 8; ++i)
+        for (int h = 0; h < 2; ++h) {
+          const int n = 16 * b + i + 8 * h;
+          sdst[2 * i + h] = n < N ? c.scales_int4[static_cast<size_t>(n) * G + g] : 0.0f;
+        }
+    }
+  });
+}
+
 }  // namespace svdq

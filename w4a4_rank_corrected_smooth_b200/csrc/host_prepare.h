@@ -40,4 +40,7 @@ int prepare_canonical(const uint16_t* W_bf16, int N, int K, const uint16_t* bias
 
 void pack_device_layouts(const CanonicalLayer& c, DeviceImages& d);
 
+// W4A16: codes and scales in the warp-level MMA's fragment order (see host_prepare.cpp).
+void pack_w4a16_fragments(const CanonicalLayer& c, DeviceImages& d);
+
 }  // namespace svdq

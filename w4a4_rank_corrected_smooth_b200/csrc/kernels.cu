@@ -656,11 +656,24 @@ static cudaError_t make_rows_map(CUtensorMap* map, const void* base, uint64_t by
 // stages before the k-blocks.  Kernel 2 is launched as a programmatic dependent of kernel 1.
 
 constexpr int kGStages = 5;
+// Warp roles, four warpgroups: 0 = the scale warps (warp w writes TMEM lane quadrant w); 1 = the
+// operand producer, the MMA issuer, the scale producer and one idle warp; 2 and 3 = the epilogue.
 constexpr int kGSfWarps = 4;
+constexpr int kGProducerWarp = 4;
+constexpr int kGMmaWarp = 5;
+constexpr int kGScaleProducerWarp = 6;
 constexpr int kGEpiWarps = 8;
-constexpr int kGFirstEpiWarp = 2 + kGSfWarps;
-constexpr int kGScaleProducerWarp = kGFirstEpiWarp + kGEpiWarps;
-constexpr int kGThreads = (kGScaleProducerWarp + 1) * 32;
+constexpr int kGFirstEpiWarp = 8;
+constexpr int kGThreads = (kGFirstEpiWarp + kGEpiWarps) * 32;
+// Register split: the block is launched with kGRegsLaunch registers a thread (512 x 128 = the
+// SM's 65536); warpgroup 0 then gives back down to kGRegsSf, warpgroup 1 to kGRegsLow, and the
+// two epilogue warpgroups take kGRegsEpi (one thread holds a row's 128 accumulator columns).
+constexpr int kGRegsLaunch = 128, kGRegsSf = 72, kGRegsLow = 72, kGRegsEpi = 184;
+static_assert(128 * kGRegsSf + 128 * kGRegsLow + 2 * 128 * kGRegsEpi <= kGThreads * kGRegsLaunch,
+              "register split exceeds the block's");
+static_assert(kGRegsSf % 8 == 0 && kGRegsLow % 8 == 0 && kGRegsEpi % 8 == 0 && kGRegsLow >= 24 && kGRegsEpi <= 256,
+              "setmaxnreg range");
+static_assert(kGThreads * kGRegsLaunch <= 65536, "launch registers");
 constexpr uint32_t kGA = kBM * kRowBytes;                   // 16 KB: own 128 rows of A
 constexpr uint32_t kGB = (kBN / 2) * kRowBytes;             // 16 KB: own half of B
 constexpr uint32_t kGSfa = kBM * kSfBytesPerRowKb;          // 2 KB of A scales per (m-tile, k-block)
@@ -670,6 +683,7 @@ constexpr uint32_t kGOutBox = 32 * 128;                     // staging box: 32 r
 constexpr uint32_t kGStaging = kGEpiWarps * kGOutBox;       // 32 KB: one box per epilogue warp
 constexpr uint32_t kGLrL2Offset = 16384;                    // L2 half in staging (T before it; rank <= 64)
 constexpr uint32_t kTmemCols = 512;
+constexpr int kRopeAhead = 4;  // fused Q/K epilogue: rotary-table units in flight per thread
 // Per-stage scale buffer: 12 blocks of 4 columns (SFA k-steps 0..3, then SFB k-steps 0..3 with
 // two 128-row blocks each), in the order of the 12 blocks of 512 B of the global scale layout.
 constexpr uint32_t kTmemSf = 256, kTmemSfCols = 48;
@@ -678,6 +692,19 @@ static_assert(kTmemSf + kGStages * kTmemSfCols <= kTmemCols, "TMEM columns");
 struct GemmParams {
   int M, N, K, rank, KB, MT2, NT, ldy;
   const float* bias;
+  int qk_cols;  // fused Q/K normalization and rotary embedding on columns [0, qk_cols)
+  const float* gamma_q;
+  const float* gamma_k;
+  const float* rope;
+  float eps;
+  // fused MLP pair (see GemmArgs)
+  const float* il_down;
+  uint8_t* codes_down;
+  uint8_t* sf_down;
+  const uint8_t* l1_down;
+  int r_down;
+  float* tpart;
+  int mlp_smax;  // slots per (row, column half) of tpart
 };
 
 // Box heights (256-byte rows) of the operand maps.
@@ -769,12 +796,66 @@ __device__ __forceinline__ float4 ldg_f4_in_order(const float* ptr) {
   return r;
 }
 
+// ---------------------------------------------------------------------------- bf16 GELU
+// GELU(y) = y Phi(y) of a bf16 input y, rounded once to the nearest bf16 (ties to even), as the
+// exact definition gives it.  Phi(y) = erfc(-y / sqrt 2) / 2 keeps full relative accuracy in the
+// negative tail, where 1 + erf(y / sqrt 2) cancels.
+//
+// Nearest bf16 (as fp32) of a double, ties to even: the two bf16 neighbours of g come from
+// truncating g toward zero to fp32 and then to bf16; both differences to g are exact in double.
+__device__ __noinline__ float bf16_nearest_of_double(double g) {
+  const uint32_t tb = __float_as_uint(__double2float_rz(g));
+  const uint32_t lo = tb & 0xFFFF0000u, hi = lo + 0x10000u;
+  const double dlo = fabs(g - static_cast<double>(__uint_as_float(lo)));
+  const double dhi = fabs(static_cast<double>(__uint_as_float(hi)) - g);
+  const bool up = dhi < dlo || (dhi == dlo && (lo & 0x10000u));
+  return __uint_as_float(up ? hi : lo);
+}
+
+// The rare inputs whose fp32 evaluation does not decide the rounding.
+__device__ __noinline__ float gelu_bf16_slow(float y) {
+  const double yd = static_cast<double>(y);
+  return bf16_nearest_of_double(0.5 * yd * erfc(-yd * 0.70710678118654752440));
+}
+
+// |y| < 2^-125, +-0 included: GELU(y) = y / 2 + y^2 / sqrt(2 pi) + O(y^4).  y / 2 is exact and a
+// bf16 subnormal (spacing 2^-133) or zero here, and the correction, positive and far below half a
+// spacing, only breaks ties, toward +infinity.  The bf16 magnitude bits of such a y are y in units
+// of 2^-133, so this is integer arithmetic on the bits (no subnormal floating-point step); a zero
+// keeps its sign, as y Phi(y) does.
+__device__ __forceinline__ float gelu_bf16_tiny(uint32_t yb) {
+  const uint32_t u = (yb >> 16) & 0x7FFFu;
+  const uint32_t neg = yb & 0x80000000u;
+  const uint32_t half = neg ? (u >> 1) : ((u + 1u) >> 1);
+  return __uint_as_float(neg | (half << 16));
+}
+
+__device__ __forceinline__ float gelu_bf16(float y) {
+  if ((__float_as_uint(y) & 0x7FFFFFFFu) < 0x01000000u) return gelu_bf16_tiny(__float_as_uint(y));
+  const float z = __fmul_rn(y, -0.70710678118654752f);
+  const float g = __fmul_rn(__fmul_rn(0.5f, y), erfcf(z));
+  // Relative error of g: erfcf's documented 4 ulp, two roundings of the argument amplified by
+  // |d ln erfc(z) / d ln z| <= 2 z^2 + 1 where z > 0 (the tail; for z <= 0 erfc lies in [1, 2] and
+  // barely moves), and the last product; (16 + 2 z^2) 2^-23 covers them with room for the roundings
+  // of the bracket itself.  Past z = 16 the value is far below fp32's normal range, where the
+  // absolute term, |y| times a few units of erfcf's last place (2^-149), takes over; the floor
+  // 2^-140 lies far below half a bf16 spacing anywhere (>= 2^-134).
+  const float zp = fminf(fmaxf(z, 0.0f), 16.0f);
+  const float rel = __fmul_rn(__fmaf_rn(__fmul_rn(2.0f, zp), zp, 16.0f), 0x1p-23f);
+  const float d = __fmaf_rn(fabsf(g), rel, __fmaf_rn(fabsf(y), 0x1p-146f, 0x1p-140f));
+  const float lo = __bfloat162float(__float2bfloat16_rn(__fsub_rn(g, d)));
+  const float hi = __bfloat162float(__float2bfloat16_rn(__fadd_rn(g, d)));
+  return __float_as_uint(lo) == __float_as_uint(hi) ? lo : gelu_bf16_slow(y);
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
 // Staging box layout: 32 rows of 128 bytes (64 bf16); 16-byte unit u of row l sits at
 // u ^ (l % 8), the tensor map's 128-byte swizzle, so lanes 8i..8i+7 hit distinct bank groups.
+// kEpi: 0 = bias and bf16 Y; 1 = fused Q/K normalization and rotary embedding; 2 = fused MLP pair.
+template <int kEpi>
 __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_constant__ GemmMaps maps,
                                                                     const GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -788,6 +869,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
   uint64_t* lr_full = acc_empty + 1;        // (leader) both CTAs' low-rank operands landed in staging
   uint64_t* stg_free = lr_full + 1;         // (both) the epilogue's stores finished reading staging
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stg_free + 1);
+  float* gamma_sm = reinterpret_cast<float*>(staging + kGStaging + 256);  // fused Q/K: gamma_q, gamma_k
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -804,6 +886,12 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
   const bool lr_in_staging = r > 0 && r <= 64;
   const int nlr_ring = lr_in_staging ? 0 : nlr;
   const int nstages_tile = nlr_ring + p.KB;
+  // Tiles of this pair: interleaved (pair, pair + npairs, ...), except in the fused MLP mode, which
+  // walks a contiguous m-major range so that consecutive tiles share rows and their partials of the
+  // down layer's T accumulate in one slot.
+  const int t_first = kEpi == 2 ? static_cast<int>(static_cast<long long>(pair) * tiles / npairs) : pair;
+  const int t_end = kEpi == 2 ? static_cast<int>(static_cast<long long>(pair + 1) * tiles / npairs) : tiles;
+  const int t_step = kEpi == 2 ? 1 : npairs;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGStages; ++s) {
@@ -818,7 +906,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kGMmaWarp) {
     tmem_alloc2(tmem_slot, kTmemCols);
     tmem_relinquish2();
   }
@@ -829,143 +917,309 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
   // Launched as a programmatic dependent of kernel 1: everything above overlapped its tail; the
   // activation codes, scales and T are read only after it has completed.
   pdl_wait_primary();
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ producer (both CTAs)
-      int st = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      for (int tile = pair; tile < tiles && ok; tile += npairs) {
-        const int m2 = tile / p.NT, nt = tile % p.NT;
-        const int mt = 2 * m2 + static_cast<int>(rank);  // this CTA's 128-row tile
-        for (int j = 0; j < nstages_tile; ++j) {
-          if (*abort_flag || !wait_parity_bounded(&empty[st], ph ^ 1u, kErrWaitGemm)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sb = smem + st * kGStage;
-          if (j < nlr_ring) {
-            const uint32_t cw = lr_chunk_width(r, j);
-            const uint32_t tb = kBM * cw * 2, lb = (kBN / 2) * cw * 2;
-            mbar_arrive_expect_tx(&full[st], tb + lb);
-            const int trow = static_cast<int>((static_cast<size_t>(mt) * kBM * r * 2 + static_cast<size_t>(kBM) * kLrChunk * 2 * j) / 256);
-            const int lrow = static_cast<int>((static_cast<size_t>(nt) * kBN * r * 2 + static_cast<size_t>(kBN) * kLrChunk * 2 * j + rank * lb) / 256);
-            for (uint32_t q = 0; q < tb / 4096; ++q) tma_load_2d(sb + 4096 * q, &maps.t, 0, trow + 16 * q, &full[st]);
-            for (uint32_t q = 0; q < lb / 4096; ++q) tma_load_2d(sb + kGA + 4096 * q, &maps.l2, 0, lrow + 16 * q, &full[st]);
-          } else {
-            const int kb = j - nlr_ring;
-            mbar_arrive_expect_tx(&full[st], kGStage);
-            tma_load_2d(sb, &maps.a, 0, static_cast<int>(codes_chunk_offset(mt, kb, p.KB, kBM) / 256), &full[st]);
-            tma_load_2d(sb + kGA, &maps.b, 0, static_cast<int>((codes_chunk_offset(nt, kb, p.KB, kBN) + rank * kGB) / 256),
-                        &full[st]);
-          }
-          if (++st == kGStages) {
-            st = 0;
-            ph ^= 1u;
-          }
-        }
-      }
-      if (!ok) *abort_flag = 1;
+  if (warp >= kGFirstEpiWarp) {
+    setmaxnreg_inc<kGRegsEpi>();
+    if constexpr (kEpi == 1) {  // the normalization weights, read by every row, into shared memory
+      const int et = threadIdx.x - kGFirstEpiWarp * 32;
+      gamma_sm[et] = et < kQkvHeadDim ? p.gamma_q[et] : p.gamma_k[et - kQkvHeadDim];
+      asm volatile("bar.sync 1, %0;" ::"n"(kGEpiWarps * 32) : "memory");
     }
-  } else if (warp == kGScaleProducerWarp) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ scale producer (both CTAs)
-      // Copies each k-block stage's two scale tiles onto full[s], which the operand producer arms
-      // with the whole stage's bytes (a copy may complete before that arrival; the phase cannot).
-      int st = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      for (int tile = pair; tile < tiles && ok; tile += npairs) {
-        const int m2 = tile / p.NT, nt = tile % p.NT;
-        const int mt = 2 * m2 + static_cast<int>(rank);
-        for (int j = 0; j < nstages_tile; ++j) {
-          if (j >= nlr_ring) {
-            if (*abort_flag || !wait_parity_bounded(&empty[st], ph ^ 1u, kErrWaitGemm)) {
-              ok = false;
-              break;
-            }
-            const int kb = j - nlr_ring;
-            uint8_t* sb = smem + st * kGStage;
-            tma_load_2d(sb + kGA + kGB, &maps.sfa, 0, static_cast<int>(sf_chunk_offset(mt, kb, p.KB, kBM) / 256), &full[st]);
-            tma_load_2d(sb + kGA + kGB + kGSfa, &maps.sfb, 0, static_cast<int>(sf_chunk_offset(nt, kb, p.KB, kBN) / 256),
-                        &full[st]);
-          }
-          if (++st == kGStages) {
-            st = 0;
-            ph ^= 1u;
-          }
-        }
-      }
-      if (!ok) *abort_flag = 1;
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && leader) {
-      // ------------------------------------------------------------ MMA issuer (leader CTA)
-      const uint32_t id_lr = idesc_bf16(256, 256);
-      const uint32_t id_fp4 = idesc_nvfp4(256, 256);
-      int st = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      int local = 0;
-      for (int tile = pair; tile < tiles && ok; tile += npairs, ++local) {
-        if (*abort_flag || !wait_parity_bounded(acc_empty, (static_cast<uint32_t>(local) & 1u) ^ 1u, kErrWaitGemm)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        uint32_t accum = 0;
-        for (int j = 0; j < nstages_tile; ++j) {
-          if (*abort_flag || !wait_parity_bounded(&ready[st], ph, kErrWaitGemm)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sb = smem_u32(smem + st * kGStage);
-          if (j < nlr_ring) {
-            const uint32_t cw = lr_chunk_width(r, j);
-            const uint64_t ad = smem_desc(sb, 128, cw * 16, kLayoutNone);
-            const uint64_t bd = smem_desc(sb + kGA, 128, cw * 16, kLayoutNone);
-            for (uint32_t ks = 0; ks < cw / 16; ++ks) {
-              mma2_bf16(tmem, ad + 16 * ks, bd + 16 * ks, id_lr, accum);
-              accum = 1;
-            }
-          } else {
-            const uint32_t sf = tmem + kTmemSf + kTmemSfCols * static_cast<uint32_t>(st);
-            const uint64_t ad = smem_desc(sb, 16, 1024, kLayoutSw128);
-            const uint64_t bd = smem_desc(sb + kGA, 16, 1024, kLayoutSw128);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              mma2_nvfp4(tmem, ad + 2 * kk, bd + 2 * kk, id_fp4, sf + 4 * kk, sf + 16 + 8 * kk, accum);
-              accum = 1;
-            }
-          }
-          tc_commit2_both(smem_u32(&empty[st]));
-          if (++st == kGStages) {
-            st = 0;
-            ph ^= 1u;
-          }
-        }
-        if (!ok) break;
-        if (lr_in_staging) {
-          if (*abort_flag || !wait_parity_bounded(lr_full, static_cast<uint32_t>(local) & 1u, kErrWaitGemm)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sg = smem_u32(staging);
-          const uint64_t ad = smem_desc(sg, 128, static_cast<uint32_t>(r) * 16, kLayoutNone);
-          const uint64_t bd = smem_desc(sg + kGLrL2Offset, 128, static_cast<uint32_t>(r) * 16, kLayoutNone);
-          for (int ks = 0; ks < r / 16; ++ks) mma2_bf16(tmem, ad + 16 * ks, bd + 16 * ks, id_lr, 1u);
-        }
-        tc_commit2_both(smem_u32(acc_full));
-      }
-      if (!ok) {
+    // ------------------------------------------------------------ epilogue (8 warps per CTA)
+    // Warp (q, h): rows 32 q .. 32 q + 31 of this CTA's 128, columns 128 h .. 128 h + 127 of the
+    // tile; lane l holds row 32 q + l.  One staging box of 32 rows x 64 columns (128-byte rows,
+    // 16-byte units swizzled by row % 8), filled and stored by TMA twice per tile.
+    const int q = warp & 3, h = (warp - kGFirstEpiWarp) >> 2;
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+    uint8_t* box = staging + (warp - kGFirstEpiWarp) * kGOutBox;
+    const uint32_t lrow = static_cast<uint32_t>(lane) * 128u;
+    const bool lr_issuer = lr_in_staging && warp == kGFirstEpiWarp && lane == 0;
+    const uint32_t lr_full_leader = mapa_shared(smem_u32(lr_full), 0);
+    // This CTA's T rows and half of L2 for `tile`, into staging (T at 0, L2 at kGLrL2Offset),
+    // completing on the leader's lr_full, which the leader arms with both CTAs' bytes.
+    auto issue_lr = [&](int tile) {
+      const int m2 = tile / p.NT, nt = tile % p.NT;
+      const int mt = 2 * m2 + static_cast<int>(rank);
+      const uint32_t tb = kBM * static_cast<uint32_t>(r) * 2, lb = (kBN / 2) * static_cast<uint32_t>(r) * 2;
+      if (leader) mbar_arrive_expect_tx(lr_full, 2 * (tb + lb));
+      const int trow = static_cast<int>(static_cast<size_t>(mt) * kBM * r * 2 / 256);
+      const int lrow = static_cast<int>((static_cast<size_t>(nt) * kBN * r * 2 + rank * lb) / 256);
+      for (uint32_t q = 0; q < tb / 4096; ++q) tma_rows_cg2(staging + 4096 * q, &maps.t, trow + 16 * q, lr_full_leader);
+      for (uint32_t q = 0; q < lb / 4096; ++q)
+        tma_rows_cg2(staging + kGLrL2Offset + 4096 * q, &maps.l2, lrow + 16 * q, lr_full_leader);
+    };
+    if (lr_issuer && t_first < t_end) issue_lr(t_first);
+    int local = 0;
+    for (int tile = t_first; tile < t_end; tile += t_step, ++local) {
+      if (!warp_wait(acc_full, static_cast<uint32_t>(local) & 1u, abort_flag)) {
         *abort_flag = 1;
-        tc_commit2_both(smem_u32(acc_full));  // completes once every issued tcgen05 op has
+        break;
+      }
+      tc_fence_after();
+      const int m2 = tile / p.NT, nt = tile % p.NT;
+      const int row0 = (2 * m2 + static_cast<int>(rank)) * kBM + q * 32;
+      const int n0 = nt * kBN + h * 128;
+      const uint32_t tacc = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * 128);
+      // All 128 columns are read before the accumulator is released (the next tile's MMAs wait
+      // for it), then biased, rounded and staged.
+      uint32_t v[2][2][32];
+      tmem_ld32(tacc, v[0][0]);
+      tmem_ld32(tacc + 32, v[0][1]);
+      tmem_ld32(tacc + 64, v[1][0]);
+      tmem_ld32(tacc + 96, v[1][1]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(acc_empty_leader);  // the accumulator may be overwritten now
+      // Row l of the box starts at a multiple of 128 B, so unit u's address (row + ((u ^ l % 8) << 4))
+      // is (row ^ ((l % 8) << 4)) ^ (u << 4): one XOR per store.
+      const uint32_t srow_swz = smem_u32(box) + lrow ^ ((static_cast<uint32_t>(lane) & 7u) << 4);
+      if constexpr (kEpi == 2) {
+        // Fused MLP pair: the biased output rounded to bf16, GELU of it rounded to bf16, times the
+        // down layer's 1/lambda: the down layer's x_hat.  It is quantized here into the down
+        // layer's workspace (codes and UE4M3 scales of the 8 groups of 16 this thread holds, the
+        // same exact rounding as kernel 1), and this half-tile's fp32 partial of the down layer's
+        // T = bf16(x_hat) L1 comes from warp-level bf16 MMAs on a copy staged in the box.  Rows
+        // past M hold zeros.
+        const int grow = row0 + lane;
+        const bool live = grow < p.M;
+        const int gmt = grow >> 7, rin = grow & 127;
+#pragma unroll
+        for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int hh = u >> 2, c = 8 * (u & 3);
+            const float4 b0 = ldg_f4_in_order(p.bias + n0 + 64 * bx + 8 * u);
+            const float4 b1 = ldg_f4_in_order(p.bias + n0 + 64 * bx + 8 * u + 4);
+            const float4 i0 = ldg_f4_in_order(p.il_down + n0 + 64 * bx + 8 * u);
+            const float4 i1 = ldg_f4_in_order(p.il_down + n0 + 64 * bx + 8 * u + 4);
+            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            const float il[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float y = __bfloat162float(__float2bfloat16_rn(__uint_as_float(v[bx][hh][c + j]) + bb[j]));
+              const float g = gelu_bf16(y);
+              v[bx][hh][c + j] = __float_as_uint(live ? __fmul_rn(g, il[j]) : 0.0f);
+            }
+          }
+        uint8_t* const cdst = p.codes_down + codes_chunk_offset(gmt, nt, p.N / kBK, kBM);
+        uint8_t* const sdst = p.sf_down + sf_chunk_offset(gmt, nt, p.N / kBK, kBM);
+        const float kInv6 = __frcp_rn(6.0f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {  // group j: columns 16 j .. 16 j + 15
+          const int bx = j >> 2, hh = (j >> 1) & 1, e0 = 16 * (j & 1);
+          uint64_t xp[2][4];
+          float pm[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const float lo = __uint_as_float(v[bx][hh][e0 + 2 * t]), hi = __uint_as_float(v[bx][hh][e0 + 2 * t + 1]);
+            xp[t >> 2][t & 3] = f2pack(lo, hi);
+            pm[t] = fmaxf(fabsf(lo), fabsf(hi));
+          }
+          const float amax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                   fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+          const float s_est = __fmul_rn(amax, kInv6);
+          uint32_t sbits = cvt_e4m3(__fmul_rn(s_est, kNudgeLo));
+          const uint32_t sc_hi = cvt_e4m3(__fmul_rn(s_est, kNudgeHi));
+          uint2 code = make_uint2(0u, 0u);
+          bool slow = sbits != sc_hi;
+          if (!slow && sbits != 0) {
+            const float rr = __frcp_rn(e4m3_to_f32(sbits));
+            const float mlo = __fmul_rn(rr, kNudgeLo), mhi = __fmul_rn(rr, kNudgeHi);
+            code.x = e2m1x8_scaled(xp[0], mlo);
+            code.y = e2m1x8_scaled(xp[1], mlo);
+            slow = (code.x != e2m1x8_scaled(xp[0], mhi)) | (code.y != e2m1x8_scaled(xp[1], mhi));
+          }
+          if (slow) {  // rare: the exact quotients decide
+            float xh[2][8];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+              for (int t = 0; t < 4; ++t) f2unpack(xp[hf][t], xh[hf][2 * t], xh[hf][2 * t + 1]);
+            sbits = cvt_e4m3(__fdiv_rn(amax, 6.0f));
+            const float sd = e4m3_to_f32(sbits);
+            code.x = sd != 0.0f ? e2m1x8_div(xh[0], sd) : 0u;
+            code.y = sd != 0.0f ? e2m1x8_div(xh[1], sd) : 0u;
+          }
+          *reinterpret_cast<uint2*>(cdst + swz128(rin, 64 * h + 8 * j)) = code;
+          sdst[sf_nvfp4_offset(rin, 8 * h + j, kBM)] = static_cast<uint8_t>(sbits);
+        }
+        if (p.r_down > 0) {
+          // D (mi, ni): rows 16 mi .. 16 mi + 15 of the warp's 32, T columns 8 ni .. 8 ni + 7 (rank <= 32)
+          const int nti = p.r_down >> 3, g8 = lane >> 2, t4 = lane & 3;
+          float d[2][4][4];
+#pragma unroll
+          for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+            for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) d[mi][ni][e] = 0.0f;
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {  // 64 columns at a time through the box
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {  // unit u: columns 64 hf + 8 u .. + 7 as bf16(x_hat)
+              const int hh = u >> 2, c = 8 * (u & 3);
+              st_shared_v4(srow_swz ^ (static_cast<uint32_t>(u) << 4),
+                           make_uint4(pack_bf16x2(__uint_as_float(v[hf][hh][c]), __uint_as_float(v[hf][hh][c + 1])),
+                                      pack_bf16x2(__uint_as_float(v[hf][hh][c + 2]), __uint_as_float(v[hf][hh][c + 3])),
+                                      pack_bf16x2(__uint_as_float(v[hf][hh][c + 4]), __uint_as_float(v[hf][hh][c + 5])),
+                                      pack_bf16x2(__uint_as_float(v[hf][hh][c + 6]), __uint_as_float(v[hf][hh][c + 7]))));
+            }
+            __syncwarp();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              uint32_t a[2][4];
+#pragma unroll
+              for (int mi = 0; mi < 2; ++mi) {
+                const uint32_t rr = 16u * mi + (lane & 7) + 8u * ((lane >> 3) & 1);
+                const uint32_t un = 2u * ks + (lane >> 4);
+                ldmatrix_x4(a[mi], smem_u32(box) + rr * 128u + ((un ^ (rr & 7u)) << 4));
+              }
+              const int kcol = n0 + 64 * hf + 16 * ks + 2 * t4;  // the down layer's k of b0
+#pragma unroll
+              for (int ni = 0; ni < 4; ++ni) {
+                if (ni < nti) {
+                  const uint32_t b0 = __ldg(reinterpret_cast<const uint32_t*>(
+                      p.l1_down + l1_offset(static_cast<uint32_t>(kcol), 8u * ni + g8, p.r_down)));
+                  const uint32_t b1 = __ldg(reinterpret_cast<const uint32_t*>(
+                      p.l1_down + l1_offset(static_cast<uint32_t>(kcol + 8), 8u * ni + g8, p.r_down)));
+                  mma_sync_bf16_16816(d[0][ni], a[0], b0, b1);
+                  mma_sync_bf16_16816(d[1][ni], a[1], b0, b1);
+                }
+              }
+            }
+            __syncwarp();  // the box is rewritten by the next half
+          }
+          // This pair's slot among the pairs whose tile ranges meet these rows (it owns the slot):
+          // the first tile of the pair's run on these rows stores, the later ones add in tile order.
+          const int p_first = static_cast<int>((static_cast<long long>(m2 * p.NT + 1) * npairs - 1) / tiles);
+          const int slot = pair - p_first;
+          const bool seg_start = tile == t_first || (tile - 1) / p.NT != m2;
+          const int nslots = 2 * p.mlp_smax;
+          float* const tp = p.tpart + static_cast<size_t>(row0) * nslots * p.r_down + (h * p.mlp_smax + slot) * p.r_down;
+#pragma unroll
+          for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+            for (int ni = 0; ni < 4; ++ni)
+              if (ni < nti)
+#pragma unroll
+                for (int jh = 0; jh < 2; ++jh) {
+                  const int rl = 16 * mi + g8 + 8 * jh;
+                  float2* dst = reinterpret_cast<float2*>(tp + static_cast<size_t>(rl) * nslots * p.r_down + 8 * ni + 2 * t4);
+                  float2 v = make_float2(d[mi][ni][2 * jh], d[mi][ni][2 * jh + 1]);
+                  if (!seg_start) {
+                    const float2 o = *dst;
+                    v = make_float2(o.x + v.x, o.y + v.y);
+                  }
+                  *dst = v;
+                }
+          fence_proxy_async_smem();  // the box's generic reads precede the next tile's bulk copies into staging
+        }
+      } else {
+        // Fused Q/K path: the thread's 128 columns are one head of its row.  Bias first, and the
+        // head's mean square; the rows past M (never stored) read the last row's angles.
+        bool qk = false;
+        float nrm = 0.0f;
+        const float* gam = nullptr;
+        const float* rp = nullptr;
+        float4 rq[kRopeAhead][2];  // the row's (cos, sin) pairs, kRopeAhead 16-byte units ahead
+        if constexpr (kEpi == 1) {
+          qk = n0 < p.qk_cols;
+          if (qk) {
+            float ss = 0.0f;
+#pragma unroll
+            for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const int hh = u >> 2, c = 8 * (u & 3);
+                const float4 b0 = ldg_f4_in_order(p.bias + n0 + 64 * bx + 8 * u);
+                const float4 b1 = ldg_f4_in_order(p.bias + n0 + 64 * bx + 8 * u + 4);
+                const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const float x = __uint_as_float(v[bx][hh][c + j]) + bb[j];
+                  v[bx][hh][c + j] = __float_as_uint(x);
+                  ss = fmaf(x, x, ss);
+                }
+              }
+            nrm = rsqrtf(fmaf(ss, 1.0f / kQkvHeadDim, p.eps));
+            gam = gamma_sm + (n0 < p.qk_cols / 2 ? 0 : kQkvHeadDim);
+            const int m = row0 + lane < p.M ? row0 + lane : p.M - 1;
+            rp = p.rope + static_cast<size_t>(m) * kQkvHeadDim;
+            // Each lane reads its own row of the table from L2: the loads run kRopeAhead units ahead
+            // of their use so that their latency overlaps the arithmetic of the units before.
+#pragma unroll
+            for (int k = 0; k < kRopeAhead; ++k) {
+              rq[k][0] = __ldg(reinterpret_cast<const float4*>(rp + 8 * k));
+              rq[k][1] = __ldg(reinterpret_cast<const float4*>(rp + 8 * k + 4));
+            }
+          }
+        }
+#pragma unroll
+        for (int bx = 0; bx < 2; ++bx) {
+          bulk_wait_read0();  // (lane 0's groups) the box's previous store has finished reading it
+          __syncwarp();
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {  // 16-byte unit u: columns 8u .. 8u + 7 of the box
+            const int hh = u >> 2, c = 8 * (u & 3);
+            uint4 o;
+            if (kEpi == 1 && qk) {
+              // normalize (x / rms * gamma), then turn pairs (2i, 2i + 1) by the row's angle i
+              const int k = 8 * bx + u, slot = k % kRopeAhead;
+              const float4 g0 = *reinterpret_cast<const float4*>(gam + 8 * k);
+              const float4 g1 = *reinterpret_cast<const float4*>(gam + 8 * k + 4);
+              const float4 r0 = rq[slot][0];  // (cos, sin) of pairs 0, 1
+              const float4 r1 = rq[slot][1];  // pairs 2, 3
+              if (k + kRopeAhead < 16) {
+                rq[slot][0] = __ldg(reinterpret_cast<const float4*>(rp + 8 * (k + kRopeAhead)));
+                rq[slot][1] = __ldg(reinterpret_cast<const float4*>(rp + 8 * (k + kRopeAhead) + 4));
+              }
+              const float x0 = __uint_as_float(v[bx][hh][c + 0]) * nrm * g0.x;
+              const float x1 = __uint_as_float(v[bx][hh][c + 1]) * nrm * g0.y;
+              const float x2 = __uint_as_float(v[bx][hh][c + 2]) * nrm * g0.z;
+              const float x3 = __uint_as_float(v[bx][hh][c + 3]) * nrm * g0.w;
+              const float x4 = __uint_as_float(v[bx][hh][c + 4]) * nrm * g1.x;
+              const float x5 = __uint_as_float(v[bx][hh][c + 5]) * nrm * g1.y;
+              const float x6 = __uint_as_float(v[bx][hh][c + 6]) * nrm * g1.z;
+              const float x7 = __uint_as_float(v[bx][hh][c + 7]) * nrm * g1.w;
+              o.x = pack_bf16x2(x0 * r0.x - x1 * r0.y, x0 * r0.y + x1 * r0.x);
+              o.y = pack_bf16x2(x2 * r0.z - x3 * r0.w, x2 * r0.w + x3 * r0.z);
+              o.z = pack_bf16x2(x4 * r1.x - x5 * r1.y, x4 * r1.y + x5 * r1.x);
+              o.w = pack_bf16x2(x6 * r1.z - x7 * r1.w, x6 * r1.w + x7 * r1.z);
+            } else {
+              const float4 b0 = ldg_f4_in_order(p.bias + n0 + 64 * bx + 8 * u);
+              const float4 b1 = ldg_f4_in_order(p.bias + n0 + 64 * bx + 8 * u + 4);
+              o.x = pack_bf16x2(__uint_as_float(v[bx][hh][c + 0]) + b0.x, __uint_as_float(v[bx][hh][c + 1]) + b0.y);
+              o.y = pack_bf16x2(__uint_as_float(v[bx][hh][c + 2]) + b0.z, __uint_as_float(v[bx][hh][c + 3]) + b0.w);
+              o.z = pack_bf16x2(__uint_as_float(v[bx][hh][c + 4]) + b1.x, __uint_as_float(v[bx][hh][c + 5]) + b1.y);
+              o.w = pack_bf16x2(__uint_as_float(v[bx][hh][c + 6]) + b1.z, __uint_as_float(v[bx][hh][c + 7]) + b1.w);
+            }
+            st_shared_v4(srow_swz ^ (static_cast<uint32_t>(u) << 4), o);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (row0 < p.M && n0 + 64 * bx < p.N) tma_store_2d(&maps.y, smem_u32(box), n0 + 64 * bx, row0);
+            bulk_commit();
+          }
+        }
+      }
+      if (lr_in_staging && tile + t_step < t_end) {
+        // staging is about to receive the next tile's low-rank operands
+        bulk_wait_read0();  // (lane 0's groups)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(stg_free);
+        if (lr_issuer) {
+          if (*abort_flag || !wait_parity_bounded(stg_free, static_cast<uint32_t>(local) & 1u, kErrWaitGemm)) {
+            *abort_flag = 1;
+            break;
+          }
+          issue_lr(tile + t_step);
+        }
       }
     }
-  } else if (warp < kGFirstEpiWarp) {
+    if (lane == 0) bulk_wait0();
+  } else if (warp < kGSfWarps) {
+    setmaxnreg_dec<kGRegsSf>();
     // ------------------------------------------------------------ scale warps (both CTAs)
     // Warp of lane quadrant q: lane l copies, for each of the stage's 12 scale blocks of 512 B in
     // shared memory, bytes [16 l, 16 l + 16) into TMEM lane 32 q + l, four columns per block (the
@@ -976,7 +1230,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
     int st = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int tile = pair; tile < tiles && ok; tile += npairs) {
+    for (int tile = t_first; tile < t_end && ok; tile += t_step) {
       for (int j = 0; j < nstages_tile; ++j) {
         if (!warp_wait(&full[st], ph, abort_flag)) {
           ok = false;
@@ -1011,104 +1265,154 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
     }
     if (!ok) *abort_flag = 1;
   } else {
-    // ------------------------------------------------------------ epilogue (8 warps per CTA)
-    // Warp (q, h): rows 32 q .. 32 q + 31 of this CTA's 128, columns 128 h .. 128 h + 127 of the
-    // tile; lane l holds row 32 q + l.  One staging box of 32 rows x 64 columns (128-byte rows,
-    // 16-byte units swizzled by row % 8), filled and stored by TMA twice per tile.
-    const int q = warp & 3, h = (warp - kGFirstEpiWarp) >> 2;
-    const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
-    uint8_t* box = staging + (warp - kGFirstEpiWarp) * kGOutBox;
-    const uint32_t lrow = static_cast<uint32_t>(lane) * 128u;
-    const bool lr_issuer = lr_in_staging && warp == kGFirstEpiWarp && lane == 0;
-    const uint32_t lr_full_leader = mapa_shared(smem_u32(lr_full), 0);
-    // This CTA's T rows and half of L2 for `tile`, into staging (T at 0, L2 at kGLrL2Offset),
-    // completing on the leader's lr_full, which the leader arms with both CTAs' bytes.
-    auto issue_lr = [&](int tile) {
-      const int m2 = tile / p.NT, nt = tile % p.NT;
-      const int mt = 2 * m2 + static_cast<int>(rank);
-      const uint32_t tb = kBM * static_cast<uint32_t>(r) * 2, lb = (kBN / 2) * static_cast<uint32_t>(r) * 2;
-      if (leader) mbar_arrive_expect_tx(lr_full, 2 * (tb + lb));
-      const int trow = static_cast<int>(static_cast<size_t>(mt) * kBM * r * 2 / 256);
-      const int lrow = static_cast<int>((static_cast<size_t>(nt) * kBN * r * 2 + rank * lb) / 256);
-      for (uint32_t q = 0; q < tb / 4096; ++q) tma_rows_cg2(staging + 4096 * q, &maps.t, trow + 16 * q, lr_full_leader);
-      for (uint32_t q = 0; q < lb / 4096; ++q)
-        tma_rows_cg2(staging + kGLrL2Offset + 4096 * q, &maps.l2, lrow + 16 * q, lr_full_leader);
-    };
-    if (lr_issuer && pair < tiles) issue_lr(pair);
-    int local = 0;
-    for (int tile = pair; tile < tiles; tile += npairs, ++local) {
-      if (!warp_wait(acc_full, static_cast<uint32_t>(local) & 1u, abort_flag)) {
-        *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
-      const int m2 = tile / p.NT, nt = tile % p.NT;
-      const int row0 = (2 * m2 + static_cast<int>(rank)) * kBM + q * 32;
-      const int n0 = nt * kBN + h * 128;
-      const uint32_t tacc = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * 128);
-      // All 128 columns are read before the accumulator is released (the next tile's MMAs wait
-      // for it), then biased, rounded and staged.
-      uint32_t v[2][2][32];
-      tmem_ld32(tacc, v[0][0]);
-      tmem_ld32(tacc + 32, v[0][1]);
-      tmem_ld32(tacc + 64, v[1][0]);
-      tmem_ld32(tacc + 96, v[1][1]);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(acc_empty_leader);  // the accumulator may be overwritten now
-      // Row l of the box starts at a multiple of 128 B, so unit u's address (row + ((u ^ l % 8) << 4))
-      // is (row ^ ((l % 8) << 4)) ^ (u << 4): one XOR per store.
-      const uint32_t srow_swz = smem_u32(box) + lrow ^ ((static_cast<uint32_t>(lane) & 7u) << 4);
-#pragma unroll
-      for (int bx = 0; bx < 2; ++bx) {
-        bulk_wait_read0();  // (lane 0's groups) the box's previous store has finished reading it
-        __syncwarp();
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {  // 16-byte unit u: columns 8u .. 8u + 7 of the box
-          const int hh = u >> 2, c = 8 * (u & 3);
-          const float4 b0 = ldg_f4_in_order(p.bias + n0 + 64 * bx + 8 * u);
-          const float4 b1 = ldg_f4_in_order(p.bias + n0 + 64 * bx + 8 * u + 4);
-          uint4 o;
-          o.x = pack_bf16x2(__uint_as_float(v[bx][hh][c + 0]) + b0.x, __uint_as_float(v[bx][hh][c + 1]) + b0.y);
-          o.y = pack_bf16x2(__uint_as_float(v[bx][hh][c + 2]) + b0.z, __uint_as_float(v[bx][hh][c + 3]) + b0.w);
-          o.z = pack_bf16x2(__uint_as_float(v[bx][hh][c + 4]) + b1.x, __uint_as_float(v[bx][hh][c + 5]) + b1.y);
-          o.w = pack_bf16x2(__uint_as_float(v[bx][hh][c + 6]) + b1.z, __uint_as_float(v[bx][hh][c + 7]) + b1.w);
-          st_shared_v4(srow_swz ^ (static_cast<uint32_t>(u) << 4), o);
+    setmaxnreg_dec<kGRegsLow>();
+    if (warp == kGProducerWarp) {
+      if (lane == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        int st = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int tile = t_first; tile < t_end && ok; tile += t_step) {
+          const int m2 = tile / p.NT, nt = tile % p.NT;
+          const int mt = 2 * m2 + static_cast<int>(rank);  // this CTA's 128-row tile
+          for (int j = 0; j < nstages_tile; ++j) {
+            if (*abort_flag || !wait_parity_bounded(&empty[st], ph ^ 1u, kErrWaitGemm)) {
+              ok = false;
+              break;
+            }
+            uint8_t* sb = smem + st * kGStage;
+            if (j < nlr_ring) {
+              const uint32_t cw = lr_chunk_width(r, j);
+              const uint32_t tb = kBM * cw * 2, lb = (kBN / 2) * cw * 2;
+              mbar_arrive_expect_tx(&full[st], tb + lb);
+              const int trow = static_cast<int>((static_cast<size_t>(mt) * kBM * r * 2 + static_cast<size_t>(kBM) * kLrChunk * 2 * j) / 256);
+              const int lrow = static_cast<int>((static_cast<size_t>(nt) * kBN * r * 2 + static_cast<size_t>(kBN) * kLrChunk * 2 * j + rank * lb) / 256);
+              for (uint32_t q = 0; q < tb / 4096; ++q) tma_load_2d(sb + 4096 * q, &maps.t, 0, trow + 16 * q, &full[st]);
+              for (uint32_t q = 0; q < lb / 4096; ++q) tma_load_2d(sb + kGA + 4096 * q, &maps.l2, 0, lrow + 16 * q, &full[st]);
+            } else {
+              const int kb = j - nlr_ring;
+              mbar_arrive_expect_tx(&full[st], kGStage);
+              tma_load_2d(sb, &maps.a, 0, static_cast<int>(codes_chunk_offset(mt, kb, p.KB, kBM) / 256), &full[st]);
+              tma_load_2d(sb + kGA, &maps.b, 0, static_cast<int>((codes_chunk_offset(nt, kb, p.KB, kBN) + rank * kGB) / 256),
+                          &full[st]);
+            }
+            if (++st == kGStages) {
+              st = 0;
+              ph ^= 1u;
+            }
+          }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (row0 < p.M && n0 + 64 * bx < p.N) tma_store_2d(&maps.y, smem_u32(box), n0 + 64 * bx, row0);
-          bulk_commit();
-        }
+        if (!ok) *abort_flag = 1;
       }
-      if (lr_in_staging && tile + npairs < tiles) {
-        // staging is about to receive the next tile's low-rank operands
-        bulk_wait_read0();  // (lane 0's groups)
-        __syncwarp();
-        if (lane == 0) mbar_arrive(stg_free);
-        if (lr_issuer) {
-          if (*abort_flag || !wait_parity_bounded(stg_free, static_cast<uint32_t>(local) & 1u, kErrWaitGemm)) {
-            *abort_flag = 1;
+    } else if (warp == kGScaleProducerWarp) {
+      if (lane == 0) {
+        // ------------------------------------------------------------ scale producer (both CTAs)
+        // Copies each k-block stage's two scale tiles onto full[s], which the operand producer arms
+        // with the whole stage's bytes (a copy may complete before that arrival; the phase cannot).
+        int st = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int tile = t_first; tile < t_end && ok; tile += t_step) {
+          const int m2 = tile / p.NT, nt = tile % p.NT;
+          const int mt = 2 * m2 + static_cast<int>(rank);
+          for (int j = 0; j < nstages_tile; ++j) {
+            if (j >= nlr_ring) {
+              if (*abort_flag || !wait_parity_bounded(&empty[st], ph ^ 1u, kErrWaitGemm)) {
+                ok = false;
+                break;
+              }
+              const int kb = j - nlr_ring;
+              uint8_t* sb = smem + st * kGStage;
+              tma_load_2d(sb + kGA + kGB, &maps.sfa, 0, static_cast<int>(sf_chunk_offset(mt, kb, p.KB, kBM) / 256), &full[st]);
+              tma_load_2d(sb + kGA + kGB + kGSfa, &maps.sfb, 0, static_cast<int>(sf_chunk_offset(nt, kb, p.KB, kBN) / 256),
+                          &full[st]);
+            }
+            if (++st == kGStages) {
+              st = 0;
+              ph ^= 1u;
+            }
+          }
+        }
+        if (!ok) *abort_flag = 1;
+      }
+    } else if (warp == kGMmaWarp) {
+      if (lane == 0 && leader) {
+        // ------------------------------------------------------------ MMA issuer (leader CTA)
+        const uint32_t id_lr = idesc_bf16(256, 256);
+        const uint32_t id_fp4 = idesc_nvfp4(256, 256);
+        int st = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        int local = 0;
+        for (int tile = t_first; tile < t_end && ok; tile += t_step, ++local) {
+          if (*abort_flag || !wait_parity_bounded(acc_empty, (static_cast<uint32_t>(local) & 1u) ^ 1u, kErrWaitGemm)) {
+            ok = false;
             break;
           }
-          issue_lr(tile + npairs);
+          tc_fence_after();
+          uint32_t accum = 0;
+          for (int j = 0; j < nstages_tile; ++j) {
+            if (*abort_flag || !wait_parity_bounded(&ready[st], ph, kErrWaitGemm)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sb = smem_u32(smem + st * kGStage);
+            if (j < nlr_ring) {
+              const uint32_t cw = lr_chunk_width(r, j);
+              const uint64_t ad = smem_desc(sb, 128, cw * 16, kLayoutNone);
+              const uint64_t bd = smem_desc(sb + kGA, 128, cw * 16, kLayoutNone);
+              for (uint32_t ks = 0; ks < cw / 16; ++ks) {
+                mma2_bf16(tmem, ad + 16 * ks, bd + 16 * ks, id_lr, accum);
+                accum = 1;
+              }
+            } else {
+              const uint32_t sf = tmem + kTmemSf + kTmemSfCols * static_cast<uint32_t>(st);
+              const uint64_t ad = smem_desc(sb, 16, 1024, kLayoutSw128);
+              const uint64_t bd = smem_desc(sb + kGA, 16, 1024, kLayoutSw128);
+  #pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                mma2_nvfp4(tmem, ad + 2 * kk, bd + 2 * kk, id_fp4, sf + 4 * kk, sf + 16 + 8 * kk, accum);
+                accum = 1;
+              }
+            }
+            tc_commit2_both(smem_u32(&empty[st]));
+            if (++st == kGStages) {
+              st = 0;
+              ph ^= 1u;
+            }
+          }
+          if (!ok) break;
+          if (lr_in_staging) {
+            if (*abort_flag || !wait_parity_bounded(lr_full, static_cast<uint32_t>(local) & 1u, kErrWaitGemm)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sg = smem_u32(staging);
+            const uint64_t ad = smem_desc(sg, 128, static_cast<uint32_t>(r) * 16, kLayoutNone);
+            const uint64_t bd = smem_desc(sg + kGLrL2Offset, 128, static_cast<uint32_t>(r) * 16, kLayoutNone);
+            for (int ks = 0; ks < r / 16; ++ks) mma2_bf16(tmem, ad + 16 * ks, bd + 16 * ks, id_lr, 1u);
+          }
+          tc_commit2_both(smem_u32(acc_full));
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          tc_commit2_both(smem_u32(acc_full));  // completes once every issued tcgen05 op has
         }
       }
     }
-    if (lane == 0) bulk_wait0();
   }
 
   __syncthreads();
-  if (warp == 1 && leader && *abort_flag && lane == 0) {
+  if (warp == kGMmaWarp && leader && *abort_flag && lane == 0) {
     const unsigned long long t0 = globaltimer_ns();  // the abort-path commits land within microseconds
     while (globaltimer_ns() - t0 < 2000000ull) {
     }
   }
   tc_fence_before();
   cluster_sync();  // neither CTA releases TMEM or exits while its peer may still address it
-  if (warp == 1) {
+  if (warp == kGMmaWarp) {
     tc_fence_after();
     tmem_dealloc2(tmem, kTmemCols);
   }
@@ -1116,30 +1420,42 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
 
 // ============================================================================ kernel 2, INT4
 //
-// INT4 codes with one fp32 scale per 64 elements cannot use block-scaled MMAs, so the 4-bit GEMM
-// runs on kind::i8: converter warps sign-extend the packed nibbles into int8 tiles, one 64-element
-// group at a time; the MMA warp accumulates each group's int32 partial in one of four TMEM buffers
-// (the bf16 up projection T L2 first, as fp32); the epilogue warps keep the fp32 accumulator in
-// registers and add each partial converted exactly to fp32 and multiplied by s_x[m,g] s_w[n,g]
-// (packed f32x2 arithmetic).  The k-block's scales arrive by bulk copy in a ring of their own,
-// released by the epilogue once it has applied them.
+// INT4 codes with one fp32 scale per 64 elements cannot use block-scaled MMAs, so every 64-element
+// group is its own MMA: converter warps turn the packed nibbles of a group into f16 values (exact:
+// one LOP3 puts two sign-flipped codes into the mantissas of 1024, one f16x2 subtract of 1032
+// leaves the signed values), and kind::f16 MMAs accumulate the group's partial sum -- an integer
+// of magnitude <= 4096, exact in fp32 -- in one of four TMEM buffers (the bf16 up projection T L2
+// first).  Within a group, the MMA's k order is free as long as A and B share it: a 32-bit word of
+// codes (elements e0..e7) becomes the f16 pairs (e0, e4), (e1, e5), (e2, e6), (e3, e7) on both
+// sides, with no byte shuffles.  The epilogue warps keep the fp32 accumulator in registers and add
+// each partial times RN(s_x[m,g] s_w[n,g]) with packed f32x2 arithmetic.  The k-block's scales
+// arrive by bulk copy in a ring of their own, released by the epilogue once it has applied them.
+// Warp roles, four warpgroups: 0 = converters, 1 = producer, MMA issuer and two idle warps, 2 and 3
+// = epilogue; the converters and warpgroup 1 give registers to the epilogue (setmaxnreg).
 
 constexpr int kIStages = 3;                                   // packed stages
-constexpr int kIGroups = 4;                                   // int8 group buffers
+constexpr int kIGroups = 2;                                   // f16 group buffers
 constexpr int kISlots = 4;                                    // TMEM partial buffers (128 columns each)
 constexpr int kISfStages = 4;                                 // scale stages (one k-block each)
 constexpr uint32_t kISfA = kBM * 4 * 4;                       // 2 KB: fp32 [128 rows][4 groups]
 constexpr uint32_t kISfB = 4 * kBN * 4;                       // 4 KB: fp32 [4 groups][256 rows]
 constexpr int kIBN = 128;                                     // output columns per tile
-constexpr int kIConvWarps = 4;
-constexpr int kIEpiWarps = 8;
+constexpr int kIConvWarps = 4;                                // warps 0-3
+constexpr int kIProducerWarp = 4;
+constexpr int kIMmaWarp = 5;
+constexpr int kIFirstEpiWarp = 8;
+constexpr int kIEpiWarps = 8;                                 // warps 8-15
 constexpr int kIEpiCols = kIBN / (kIEpiWarps / 4);             // 64 accumulator columns per epilogue thread
-constexpr int kIThreads = (2 + kIConvWarps + kIEpiWarps) * 32;
+constexpr int kIThreads = (kIFirstEpiWarp + kIEpiWarps) * 32;
+constexpr int kIRegsLaunch = 128, kIRegsConv = 64, kIRegsLow = 40, kIRegsEpi = 200;
+static_assert(128 * kIRegsConv + 128 * kIRegsLow + 2 * 128 * kIRegsEpi <= kIThreads * kIRegsLaunch,
+              "register split exceeds the block's");
+static_assert(kIThreads * kIRegsLaunch <= 65536, "launch registers");
 constexpr uint32_t kIPackA = kBM * kRowBytes;                 // 16 KB
 constexpr uint32_t kIPackB = kIBN * kRowBytes;                // 16 KB
 constexpr uint32_t kIPack = kIPackA + kIPackB;
-constexpr uint32_t kIGrpA = kBM * 64;                         // 8 KB int8
-constexpr uint32_t kIGrpB = kIBN * 64;
+constexpr uint32_t kIGrpA = kBM * 128;                        // 16 KB: 128 rows x 64 f16
+constexpr uint32_t kIGrpB = kIBN * 128;
 constexpr uint32_t kIGrp = kIGrpA + kIGrpB;
 constexpr uint32_t kIStagePitch = kIBN * 2 + 16;              // bf16 output row + 16 B
 constexpr uint32_t kIStaging = kBM * kIStagePitch;
@@ -1154,29 +1470,36 @@ struct GemmI4Params {
   const uint8_t* l2;
   const float* bias;
   uint16_t* Y;
+  int qk_cols;  // fused Q/K normalization and rotary embedding on columns [0, qk_cols)
+  const float* gamma_q;
+  const float* gamma_k;
+  const float* rope;
+  float eps;
 };
 
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Four 4-bit two's-complement values, one per byte (0..15), sign-extended to int8 in place: a byte
-// with bit 3 set gets 0xF0 ORed in; (x & 0x08080808) * 0x1E puts exactly 0xF0 in those bytes (8 *
-// 0x1E = 0xF0 < 0x100, so no carry crosses a byte).
-__device__ __forceinline__ uint32_t sext_nibbles4(uint32_t x) { return x | ((x & 0x08080808u) * 0x1Eu); }
-
-// 8 packed int4 codes (4 bytes, element 2i in the low nibble) -> 8 int8 in element order.
-__device__ __forceinline__ uint2 unpack_int4x8(uint32_t w) {
-  const uint32_t lo = sext_nibbles4(w & 0x0F0F0F0Fu);          // elements 0,2,4,6
-  const uint32_t hi = sext_nibbles4((w >> 4) & 0x0F0F0F0Fu);   // elements 1,3,5,7
-  return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+// Eight packed int4 codes (element j in bits 4j..4j+3) -> four f16x2 registers holding the pairs
+// (e0, e4), (e1, e5), (e2, e6), (e3, e7), exactly: (w >> 4s) & 0x000F000F puts e_s and e_s+4 in the
+// low mantissa bits of two f16 halves; XOR 0x6408 sets each half to 1024 + (v ^ 8) = 1032 + q.
+__device__ __forceinline__ uint4 int4x8_to_f16_pairs(uint32_t w) {
+  uint32_t r[4];
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    uint32_t t;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w >> (4 * s)), "r"(0x000F000Fu), "r"(0x64086408u));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r[s]) : "r"(t), "r"(0x64086408u));
+  }
+  return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
 __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* packed = smem;                                  // kIStages x 32 KB
-  uint8_t* groups = packed + kIStages * kIPack;            // kIGroups x 16 KB
+  uint8_t* groups = packed + kIStages * kIPack;            // kIGroups x 32 KB
   uint8_t* sfring = groups + kIGroups * kIGrp;              // kISfStages x 6 KB
   uint8_t* staging = sfring + kISfStages * (kISfA + kISfB);
   uint64_t* pfull = reinterpret_cast<uint64_t*>(staging + kIStaging);
@@ -1187,7 +1510,8 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
   uint64_t* tempty = tfull + kISlots;
   uint64_t* sfull = tempty + kISlots;
   uint64_t* sempty = sfull + kISfStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + kISfStages);
+  uint64_t* sspair = sempty + kISfStages;  // (fused Q/K) both column halves' sums of squares written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sspair + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1214,10 +1538,11 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
       mbar_init(&sfull[b], 1);
       mbar_init(&sempty[b], kIEpiWarps);
     }
+    for (int q = 0; q < 4; ++q) mbar_init(&sspair[q], 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kIMmaWarp) {
     tmem_alloc(tmem_slot, kISlots * kIBN);
     tmem_relinquish();
   }
@@ -1226,140 +1551,172 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ producer
-      int st = 0;
-      uint32_t ph = 0;
-      int issued_phase[kIStages], sf_issued_phase[kISfStages];
-      for (int s = 0; s < kIStages; ++s) issued_phase[s] = -1;
-      for (int s = 0; s < kISfStages; ++s) sf_issued_phase[s] = -1;
-      int ss = 0;
-      uint32_t sph = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-        const int mt = tile / p.NT, n128 = tile % p.NT, n256 = n128 >> 1, nh = n128 & 1;
-        for (int j = 0; j < nst; ++j) {
-          if (*abort_flag || !wait_parity_bounded(&pempty[st], ph ^ 1u, kErrWaitGemm)) {
-            ok = false;
-            break;
+  if (warp >= kIFirstEpiWarp) {
+    setmaxnreg_inc<kIRegsEpi>();
+    // ------------------------------------------------------------ rescale + epilogue (8 warps)
+    const int ew = warp - kIFirstEpiWarp;
+    const int q = warp & 3, cg = ew >> 2;  // TMEM lane quadrant this warp may access (warp % 4), column group
+    const int rloc = q * 32 + lane;
+    uint8_t* srow = staging + rloc * kIStagePitch + cg * kIEpiCols * 2;
+    int slot = 0, ss = 0, qkn = 0;
+    uint32_t sph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      const int mt = tile / p.NT, n128 = tile % p.NT, nh = n128 & 1;
+      uint64_t acc[kIEpiCols / 2];  // this thread's fp32 accumulators as pairs
+#pragma unroll
+      for (int c = 0; c < kIEpiCols / 2; ++c) acc[c] = 0ull;
+      const int nslots = (nlr > 0 ? 1 : 0) + ngrp;
+      for (int si = 0; si < nslots; ++si) {
+        const uint32_t b = slot % kISlots;
+        const bool lr = nlr > 0 && si == 0;
+        const int g = lr ? 0 : si - (nlr > 0 ? 1 : 0);
+        const int gi = g & 3;
+        bool w = true;
+        if (lane == 0) {
+          w = !*abort_flag && wait_parity_bounded(&tfull[b], (slot / kISlots) & 1, kErrWaitGemm);
+          if (w && !lr && gi == 0) w = wait_parity_bounded(&sfull[ss], sph, kErrWaitGemm);
+        }
+        if (!__shfl_sync(0xffffffffu, w, 0)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // the slot's 64 fp32 partials of this thread's row; then the slot goes back to the MMA
+        uint32_t v0[32], v1[32];
+        const uint32_t ta = tmem + b * kIBN + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(cg * kIEpiCols);
+        tmem_ld32(ta, v0);
+        tmem_ld32(ta + 32, v1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[b]);
+        if (lr) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            acc[c] = f2pack(__uint_as_float(v0[2 * c]), __uint_as_float(v0[2 * c + 1]));
+            acc[16 + c] = f2pack(__uint_as_float(v1[2 * c]), __uint_as_float(v1[2 * c + 1]));
           }
-          uint8_t* sb = packed + st * kIPack;
-          if (j < nlr) {
-            const uint32_t cw = lr_chunk_width(r, j);
-            const uint32_t bytes = kBM * cw * 2;  // T rows and L2 rows alike (128 each)
-            mbar_arrive_expect_tx(&pfull[st], 2 * bytes);
-            bulk_g2s(sb, p.t + static_cast<size_t>(mt) * kBM * r * 2 + static_cast<size_t>(kBM) * kLrChunk * 2 * j, bytes,
-                     &pfull[st]);
-            bulk_g2s(sb + kIPackA,
-                     p.l2 + static_cast<size_t>(n256) * kBN * r * 2 + static_cast<size_t>(kBN) * kLrChunk * 2 * j + nh * bytes,
-                     bytes, &pfull[st]);
-          } else {
-            const int kb = j - nlr;
-            // the k-block's scales: A [128 rows][4 groups], B [4 groups][256 rows] (both halves)
-            if (*abort_flag || !wait_parity_bounded(&sempty[ss], sph ^ 1u, kErrWaitGemm)) {
-              ok = false;
-              break;
-            }
-            uint8_t* sfb = sfring + ss * (kISfA + kISfB);
-            mbar_arrive_expect_tx(&sfull[ss], kISfA + kISfB);
-            bulk_g2s(sfb, p.a_sf + (static_cast<size_t>(mt) * p.KB + kb) * (kBM * 4), kISfA, &sfull[ss]);
-            bulk_g2s(sfb + kISfA, p.b_sf + (static_cast<size_t>(n256) * p.KB + kb) * (kBN * 4), kISfB, &sfull[ss]);
-            sf_issued_phase[ss] = static_cast<int>(sph);
+        } else {
+          const uint8_t* sfb = sfring + ss * (kISfA + kISfB);
+          const float sx = reinterpret_cast<const float*>(sfb)[rloc * 4 + gi];
+          const float* swp = reinterpret_cast<const float*>(sfb + kISfA) + gi * kBN + nh * kIBN + cg * kIEpiCols;
+          const uint64_t sx2 = f2pack(sx, sx);
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const float4 sw0 = *reinterpret_cast<const float4*>(swp + c);  // same for all lanes
+            const float4 sw1 = *reinterpret_cast<const float4*>(swp + 32 + c);
+            acc[c / 2] = f2fma(f2pack(__uint_as_float(v0[c]), __uint_as_float(v0[c + 1])),
+                               f2mul(sx2, f2pack(sw0.x, sw0.y)), acc[c / 2]);
+            acc[c / 2 + 1] = f2fma(f2pack(__uint_as_float(v0[c + 2]), __uint_as_float(v0[c + 3])),
+                                   f2mul(sx2, f2pack(sw0.z, sw0.w)), acc[c / 2 + 1]);
+            acc[16 + c / 2] = f2fma(f2pack(__uint_as_float(v1[c]), __uint_as_float(v1[c + 1])),
+                                    f2mul(sx2, f2pack(sw1.x, sw1.y)), acc[16 + c / 2]);
+            acc[16 + c / 2 + 1] = f2fma(f2pack(__uint_as_float(v1[c + 2]), __uint_as_float(v1[c + 3])),
+                                        f2mul(sx2, f2pack(sw1.z, sw1.w)), acc[16 + c / 2 + 1]);
+          }
+          if (gi == 3) {  // the k-block's scales are applied
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sempty[ss]);
             if (++ss == kISfStages) {
               ss = 0;
               sph ^= 1u;
             }
-            mbar_arrive_expect_tx(&pfull[st], kIPack);
-            bulk_g2s(sb, p.a_codes + codes_chunk_offset(mt, kb, p.KB, kBM), kIPackA, &pfull[st]);
-            bulk_g2s(sb + kIPackA, p.b_codes + codes_chunk_offset(n256, kb, p.KB, kBN) + nh * kIPackB, kIPackB, &pfull[st]);
-          }
-          issued_phase[st] = static_cast<int>(ph);
-          if (++st == kIStages) {
-            st = 0;
-            ph ^= 1u;
           }
         }
+        ++slot;
       }
-      if (!ok) {
-        *abort_flag = 1;
-        for (int s = 0; s < kIStages; ++s)
-          if (issued_phase[s] >= 0) wait_parity_bounded(&pfull[s], static_cast<uint32_t>(issued_phase[s]), kErrWaitGemm);
-        for (int s = 0; s < kISfStages; ++s)
-          if (sf_issued_phase[s] >= 0)
-            wait_parity_bounded(&sfull[s], static_cast<uint32_t>(sf_issued_phase[s]), kErrWaitGemm);
+      if (!ok) break;
+      // bias, bf16, stage, one bulk store per row segment
+      const int row = mt * kBM + rloc;
+      const int n0 = n128 * kIBN + cg * kIEpiCols;
+      // Fused Q/K path: the tile's 128 columns are one head; this thread holds half of its row, so
+      // the two column halves exchange their sums of squares (double-buffered slots, one barrier
+      // phase per such tile, bounded wait) and add them in column order.
+      const bool qk = p.qk_cols > 0 && n128 * kIBN < p.qk_cols;
+      float nrm = 0.0f;
+      if (qk) {
+        float ssq = 0.0f;
+#pragma unroll
+        for (int u = 0; u < kIEpiCols / 8; ++u) {
+          const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8));
+          const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8 + 4));
+          const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float x0, x1;
+            f2unpack(acc[u * 4 + k], x0, x1);
+            x0 += bb[2 * k];
+            x1 += bb[2 * k + 1];
+            acc[u * 4 + k] = f2pack(x0, x1);
+            ssq = fmaf(x0, x0, ssq);
+            ssq = fmaf(x1, x1, ssq);
+          }
+        }
+        float* slots = reinterpret_cast<float*>(staging + kIStaging + 1024);  // [2 parities][2 halves][128 rows]
+        const int par = qkn & 1;
+        slots[(par * 2 + cg) * kBM + rloc] = ssq;
+        __syncwarp();
+        bool w = true;
+        if (lane == 0) {
+          mbar_arrive(&sspair[q]);
+          w = !*abort_flag && wait_parity_bounded(&sspair[q], static_cast<uint32_t>(par), kErrWaitGemm);
+        }
+        if (!__shfl_sync(0xffffffffu, w, 0)) {
+          ok = false;
+          break;
+        }
+        const float other = slots[(par * 2 + (cg ^ 1)) * kBM + rloc];
+        nrm = rsqrtf(fmaf(cg == 0 ? ssq + other : other + ssq, 1.0f / 128.0f, p.eps));
+        ++qkn;
       }
+      bulk_wait_read0();
+      const float* gam = n128 * kIBN < p.qk_cols / 2 ? p.gamma_q : p.gamma_k;
+      const int mrope = row < p.M ? row : p.M - 1;
+#pragma unroll
+      for (int u = 0; u < kIEpiCols / 8; ++u) {
+        uint4 o;
+        float a[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) f2unpack(acc[u * 4 + k], a[2 * k], a[2 * k + 1]);
+        if (qk) {
+          // normalize, then turn pairs (2i, 2i + 1) of the head by the row's angle i
+          const int hc = cg * kIEpiCols + u * 8;  // the head's channel of a[0]
+          const float4 g0 = __ldg(reinterpret_cast<const float4*>(gam + hc));
+          const float4 g1 = __ldg(reinterpret_cast<const float4*>(gam + hc + 4));
+          const float4 r0 = __ldg(reinterpret_cast<const float4*>(p.rope + static_cast<size_t>(mrope) * 128 + hc));
+          const float4 r1 = __ldg(reinterpret_cast<const float4*>(p.rope + static_cast<size_t>(mrope) * 128 + hc + 4));
+          const float x0 = a[0] * nrm * g0.x, x1 = a[1] * nrm * g0.y, x2 = a[2] * nrm * g0.z, x3 = a[3] * nrm * g0.w;
+          const float x4 = a[4] * nrm * g1.x, x5 = a[5] * nrm * g1.y, x6 = a[6] * nrm * g1.z, x7 = a[7] * nrm * g1.w;
+          o.x = pack_bf16x2(x0 * r0.x - x1 * r0.y, x0 * r0.y + x1 * r0.x);
+          o.y = pack_bf16x2(x2 * r0.z - x3 * r0.w, x2 * r0.w + x3 * r0.z);
+          o.z = pack_bf16x2(x4 * r1.x - x5 * r1.y, x4 * r1.y + x5 * r1.x);
+          o.w = pack_bf16x2(x6 * r1.z - x7 * r1.w, x6 * r1.w + x7 * r1.z);
+        } else {
+          const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8));
+          const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8 + 4));
+          o.x = pack_bf16x2(a[0] + b0.x, a[1] + b0.y);
+          o.y = pack_bf16x2(a[2] + b0.z, a[3] + b0.w);
+          o.z = pack_bf16x2(a[4] + b1.x, a[5] + b1.y);
+          o.w = pack_bf16x2(a[6] + b1.z, a[7] + b1.w);
+        }
+        *reinterpret_cast<uint4*>(srow + 16 * u) = o;
+      }
+      fence_proxy_async_smem();
+      if (row < p.M && n0 < p.N) {
+        const int ncols = (p.N - n0) < kIEpiCols ? (p.N - n0) : kIEpiCols;
+        bulk_s2g(p.Y + static_cast<size_t>(row) * p.ldy + n0, smem_u32(srow), static_cast<uint32_t>(ncols) * 2u);
+      }
+      bulk_commit();
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
-      const uint32_t id_lr = idesc_bf16(128, kIBN);
-      const uint32_t id_i8 = idesc_i8(128, kIBN);
-      int st = 0, gs = 0, slot = 0;
-      uint32_t ph = 0, gph = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-        // low-rank slot: T L2 in fp32 into TMEM buffer (slot % kISlots)
-        for (int j = 0; j < nlr && ok; ++j) {
-          const uint32_t b = slot % kISlots;
-          if (j == 0 && (*abort_flag || !wait_parity_bounded(&tempty[b], ((slot / kISlots) & 1) ^ 1u, kErrWaitGemm))) {
-            ok = false;
-            break;
-          }
-          if (*abort_flag || !wait_parity_bounded(&pfull[st], ph, kErrWaitGemm)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t cw = lr_chunk_width(r, j);
-          const uint32_t sb = smem_u32(packed + st * kIPack);
-          const uint64_t ad = smem_desc(sb, 128, cw * 16, kLayoutNone);
-          const uint64_t bd = smem_desc(sb + kIPackA, 128, cw * 16, kLayoutNone);
-          for (uint32_t ks = 0; ks < cw / 16; ++ks)
-            mma_bf16(tmem + b * kIBN, ad + 16 * ks, bd + 16 * ks, id_lr, (j | ks) != 0 ? 1u : 0u);
-          tc_commit(&pempty[st]);
-          if (++st == kIStages) {
-            st = 0;
-            ph ^= 1u;
-          }
-          if (j == nlr - 1) {
-            tc_commit(&tfull[b]);
-            ++slot;
-          }
-        }
-        // one slot per 64-element group
-        for (int g = 0; g < ngrp && ok; ++g) {
-          const uint32_t b = slot % kISlots;
-          if (*abort_flag || !wait_parity_bounded(&tempty[b], ((slot / kISlots) & 1) ^ 1u, kErrWaitGemm) ||
-              !wait_parity_bounded(&gfull[gs], gph, kErrWaitGemm)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t gb = smem_u32(groups + gs * kIGrp);
-          const uint64_t ad = smem_desc(gb, 128, 512, kLayoutNone);
-          const uint64_t bd = smem_desc(gb + kIGrpA, 128, 512, kLayoutNone);
-          mma_i8(tmem + b * kIBN, ad, bd, id_i8, 0u);
-          mma_i8(tmem + b * kIBN, ad + 16, bd + 16, id_i8, 1u);  // next 32 elements: 2 core matrices on
-          tc_commit(&gempty[gs]);
-          tc_commit(&tfull[b]);
-          ++slot;
-          if (++gs == kIGroups) {
-            gs = 0;
-            gph ^= 1u;
-          }
-        }
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        tc_commit(&tfull[0]);
-      }
-    }
-  } else if (warp < 2 + kIConvWarps) {
+    bulk_wait0();
+    if (!ok) *abort_flag = 1;
+  } else if (warp < kIConvWarps) {
+    setmaxnreg_dec<kIRegsConv>();
     // ------------------------------------------------------------ converters (4 warps)
     // After an abort a warp skips its work but still passes every named barrier, so the four
     // converter warps always execute the same barrier sequence.
-    const int t = threadIdx.x - 64;  // 0..127: one row of A and one of B
+    const int t = threadIdx.x;  // 0..127: one row of A and one of B
     int st = 0, gs = 0;
     uint32_t ph = 0, gph = 0;
     bool ok = true;
@@ -1386,14 +1743,17 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
             for (int op = 0; op < 2; ++op) {  // A then B: row t of each
               const uint8_t* src = pk + op * kIPackA;
               uint8_t* dst = gb + op * kIGrpA;
+              // row t of the group: eight 16-byte f16 units (one per packed 32-bit word), unit u
+              // at core matrix (t / 8, u) of the no-swizzle K-major layout (128 bytes between core
+              // matrices along K, 1024 bytes per 8-row block)
+              const uint32_t base = (t >> 3) * 1024u + (t & 7) * 16u;
 #pragma unroll
               for (int jj = 0; jj < 2; ++jj) {  // two packed 16-byte units = 64 codes of the group
                 const uint4 v = *reinterpret_cast<const uint4*>(src + swz128(t, (2 * gi + jj) * 16));
-                const uint2 a0 = unpack_int4x8(v.x), a1 = unpack_int4x8(v.y), a2 = unpack_int4x8(v.z),
-                            a3 = unpack_int4x8(v.w);
-                const uint32_t base = (t >> 3) * 512u + (t & 7) * 16u;
-                *reinterpret_cast<uint4*>(dst + base + (2 * jj) * 128u) = make_uint4(a0.x, a0.y, a1.x, a1.y);
-                *reinterpret_cast<uint4*>(dst + base + (2 * jj + 1) * 128u) = make_uint4(a2.x, a2.y, a3.x, a3.y);
+                *reinterpret_cast<uint4*>(dst + base + (4 * jj + 0) * 128u) = int4x8_to_f16_pairs(v.x);
+                *reinterpret_cast<uint4*>(dst + base + (4 * jj + 1) * 128u) = int4x8_to_f16_pairs(v.y);
+                *reinterpret_cast<uint4*>(dst + base + (4 * jj + 2) * 128u) = int4x8_to_f16_pairs(v.z);
+                *reinterpret_cast<uint4*>(dst + base + (4 * jj + 3) * 128u) = int4x8_to_f16_pairs(v.w);
               }
             }
             fence_proxy_async_smem();
@@ -1415,105 +1775,142 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
     }
     if (!ok) *abort_flag = 1;
   } else {
-    // ------------------------------------------------------------ rescale + epilogue (8 warps)
-    const int ew = warp - 2 - kIConvWarps;
-    const int q = warp & 3, cg = ew >> 2;  // TMEM lane quadrant this warp may access (warp % 4), column group
-    const int rloc = q * 32 + lane;
-    uint8_t* srow = staging + rloc * kIStagePitch + cg * kIEpiCols * 2;
-    // |partial| <= 64*8*8: adding 1.5*2^23 as an integer and subtracting it as a float is exact
-    const uint64_t magic2 = f2pack(12582912.0f, 12582912.0f);
-    int slot = 0, ss = 0;
-    uint32_t sph = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-      const int mt = tile / p.NT, n128 = tile % p.NT, nh = n128 & 1;
-      uint64_t acc[kIEpiCols / 2];  // this thread's fp32 accumulators as pairs
-#pragma unroll
-      for (int c = 0; c < kIEpiCols / 2; ++c) acc[c] = 0ull;
-      const int nslots = (nlr > 0 ? 1 : 0) + ngrp;
-      for (int si = 0; si < nslots; ++si) {
-        const uint32_t b = slot % kISlots;
-        const bool lr = nlr > 0 && si == 0;
-        const int g = lr ? 0 : si - (nlr > 0 ? 1 : 0);
-        const int gi = g & 3;
-        bool w = true;
-        if (lane == 0) {
-          w = !*abort_flag && wait_parity_bounded(&tfull[b], (slot / kISlots) & 1, kErrWaitGemm);
-          if (w && !lr && gi == 0) w = wait_parity_bounded(&sfull[ss], sph, kErrWaitGemm);
-        }
-        if (!__shfl_sync(0xffffffffu, w, 0)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint8_t* sfb = sfring + ss * (kISfA + kISfB);
-        const float sx = lr ? 0.0f : reinterpret_cast<const float*>(sfb)[rloc * 4 + gi];
-        const float* swp = reinterpret_cast<const float*>(sfb + kISfA) + gi * kBN + nh * kIBN + cg * kIEpiCols;
-        const uint64_t sx2 = f2pack(sx, sx);
-#pragma unroll
-        for (int half = 0; half < kIEpiCols / 32; ++half) {
-          uint32_t v[32];
-          tmem_ld32(tmem + b * kIBN + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(cg * kIEpiCols + half * 32), v);
-          tmem_wait_ld();
-          if (lr) {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) acc[half * 16 + c] = f2pack(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1]));
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; c += 4) {
-              const float4 sw = *reinterpret_cast<const float4*>(swp + half * 32 + c);  // same for all lanes
-              const uint64_t c01 = f2mul(sx2, f2pack(sw.x, sw.y)), c23 = f2mul(sx2, f2pack(sw.z, sw.w));
-              const uint64_t f01 = f2sub(f2pack(__uint_as_float(v[c] + 0x4B400000u), __uint_as_float(v[c + 1] + 0x4B400000u)), magic2);
-              const uint64_t f23 = f2sub(f2pack(__uint_as_float(v[c + 2] + 0x4B400000u), __uint_as_float(v[c + 3] + 0x4B400000u)), magic2);
-              acc[half * 16 + c / 2] = f2fma(f01, c01, acc[half * 16 + c / 2]);
-              acc[half * 16 + c / 2 + 1] = f2fma(f23, c23, acc[half * 16 + c / 2 + 1]);
+    setmaxnreg_dec<kIRegsLow>();
+    if (warp == kIProducerWarp) {
+      if (lane == 0) {
+        // ------------------------------------------------------------ producer
+        int st = 0;
+        uint32_t ph = 0;
+        int issued_phase[kIStages], sf_issued_phase[kISfStages];
+        for (int s = 0; s < kIStages; ++s) issued_phase[s] = -1;
+        for (int s = 0; s < kISfStages; ++s) sf_issued_phase[s] = -1;
+        int ss = 0;
+        uint32_t sph = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+          const int mt = tile / p.NT, n128 = tile % p.NT, n256 = n128 >> 1, nh = n128 & 1;
+          for (int j = 0; j < nst; ++j) {
+            if (*abort_flag || !wait_parity_bounded(&pempty[st], ph ^ 1u, kErrWaitGemm)) {
+              ok = false;
+              break;
+            }
+            uint8_t* sb = packed + st * kIPack;
+            if (j < nlr) {
+              const uint32_t cw = lr_chunk_width(r, j);
+              const uint32_t bytes = kBM * cw * 2;  // T rows and L2 rows alike (128 each)
+              mbar_arrive_expect_tx(&pfull[st], 2 * bytes);
+              bulk_g2s(sb, p.t + static_cast<size_t>(mt) * kBM * r * 2 + static_cast<size_t>(kBM) * kLrChunk * 2 * j, bytes,
+                       &pfull[st]);
+              bulk_g2s(sb + kIPackA,
+                       p.l2 + static_cast<size_t>(n256) * kBN * r * 2 + static_cast<size_t>(kBN) * kLrChunk * 2 * j + nh * bytes,
+                       bytes, &pfull[st]);
+            } else {
+              const int kb = j - nlr;
+              // the k-block's scales: A [128 rows][4 groups], B [4 groups][256 rows] (both halves)
+              if (*abort_flag || !wait_parity_bounded(&sempty[ss], sph ^ 1u, kErrWaitGemm)) {
+                ok = false;
+                break;
+              }
+              uint8_t* sfb = sfring + ss * (kISfA + kISfB);
+              mbar_arrive_expect_tx(&sfull[ss], kISfA + kISfB);
+              bulk_g2s(sfb, p.a_sf + (static_cast<size_t>(mt) * p.KB + kb) * (kBM * 4), kISfA, &sfull[ss]);
+              bulk_g2s(sfb + kISfA, p.b_sf + (static_cast<size_t>(n256) * p.KB + kb) * (kBN * 4), kISfB, &sfull[ss]);
+              sf_issued_phase[ss] = static_cast<int>(sph);
+              if (++ss == kISfStages) {
+                ss = 0;
+                sph ^= 1u;
+              }
+              mbar_arrive_expect_tx(&pfull[st], kIPack);
+              bulk_g2s(sb, p.a_codes + codes_chunk_offset(mt, kb, p.KB, kBM), kIPackA, &pfull[st]);
+              bulk_g2s(sb + kIPackA, p.b_codes + codes_chunk_offset(n256, kb, p.KB, kBN) + nh * kIPackB, kIPackB, &pfull[st]);
+            }
+            issued_phase[st] = static_cast<int>(ph);
+            if (++st == kIStages) {
+              st = 0;
+              ph ^= 1u;
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&tempty[b]);
-          if (!lr && gi == 3) mbar_arrive(&sempty[ss]);  // the k-block's scales are applied
+        if (!ok) {
+          *abort_flag = 1;
+          for (int s = 0; s < kIStages; ++s)
+            if (issued_phase[s] >= 0) wait_parity_bounded(&pfull[s], static_cast<uint32_t>(issued_phase[s]), kErrWaitGemm);
+          for (int s = 0; s < kISfStages; ++s)
+            if (sf_issued_phase[s] >= 0)
+              wait_parity_bounded(&sfull[s], static_cast<uint32_t>(sf_issued_phase[s]), kErrWaitGemm);
         }
-        if (!lr && gi == 3 && ++ss == kISfStages) {
-          ss = 0;
-          sph ^= 1u;
+      }
+    } else if (warp == kIMmaWarp) {
+      if (lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        const uint32_t id_lr = idesc_bf16(128, kIBN);
+        const uint32_t id_f16 = idesc_f16(128, kIBN);
+        int st = 0, gs = 0, slot = 0;
+        uint32_t ph = 0, gph = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+          // low-rank slot: T L2 in fp32 into TMEM buffer (slot % kISlots)
+          for (int j = 0; j < nlr && ok; ++j) {
+            const uint32_t b = slot % kISlots;
+            if (j == 0 && (*abort_flag || !wait_parity_bounded(&tempty[b], ((slot / kISlots) & 1) ^ 1u, kErrWaitGemm))) {
+              ok = false;
+              break;
+            }
+            if (*abort_flag || !wait_parity_bounded(&pfull[st], ph, kErrWaitGemm)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t cw = lr_chunk_width(r, j);
+            const uint32_t sb = smem_u32(packed + st * kIPack);
+            const uint64_t ad = smem_desc(sb, 128, cw * 16, kLayoutNone);
+            const uint64_t bd = smem_desc(sb + kIPackA, 128, cw * 16, kLayoutNone);
+            for (uint32_t ks = 0; ks < cw / 16; ++ks)
+              mma_bf16(tmem + b * kIBN, ad + 16 * ks, bd + 16 * ks, id_lr, (j | ks) != 0 ? 1u : 0u);
+            tc_commit(&pempty[st]);
+            if (++st == kIStages) {
+              st = 0;
+              ph ^= 1u;
+            }
+            if (j == nlr - 1) {
+              tc_commit(&tfull[b]);
+              ++slot;
+            }
+          }
+          // one slot per 64-element group
+          for (int g = 0; g < ngrp && ok; ++g) {
+            const uint32_t b = slot % kISlots;
+            if (*abort_flag || !wait_parity_bounded(&tempty[b], ((slot / kISlots) & 1) ^ 1u, kErrWaitGemm) ||
+                !wait_parity_bounded(&gfull[gs], gph, kErrWaitGemm)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t gb = smem_u32(groups + gs * kIGrp);
+            const uint64_t ad = smem_desc(gb, 128, 1024, kLayoutNone);
+            const uint64_t bd = smem_desc(gb + kIGrpA, 128, 1024, kLayoutNone);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)  // 16 f16 of K per MMA: 2 core matrices (256 bytes) on
+              mma_bf16(tmem + b * kIBN, ad + 16 * ks, bd + 16 * ks, id_f16, ks > 0 ? 1u : 0u);
+            tc_commit(&gempty[gs]);
+            tc_commit(&tfull[b]);
+            ++slot;
+            if (++gs == kIGroups) {
+              gs = 0;
+              gph ^= 1u;
+            }
+          }
         }
-        ++slot;
+        if (!ok) {
+          *abort_flag = 1;
+          tc_commit(&tfull[0]);
+        }
       }
-      if (!ok) break;
-      // bias, bf16, stage, one bulk store per row segment
-      const int row = mt * kBM + rloc;
-      const int n0 = n128 * kIBN + cg * kIEpiCols;
-      bulk_wait_read0();
-#pragma unroll
-      for (int u = 0; u < kIEpiCols / 8; ++u) {
-        const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8));
-        const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + u * 8 + 4));
-        uint4 o;
-        float a[8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) f2unpack(acc[u * 4 + k], a[2 * k], a[2 * k + 1]);
-        o.x = pack_bf16x2(a[0] + b0.x, a[1] + b0.y);
-        o.y = pack_bf16x2(a[2] + b0.z, a[3] + b0.w);
-        o.z = pack_bf16x2(a[4] + b1.x, a[5] + b1.y);
-        o.w = pack_bf16x2(a[6] + b1.z, a[7] + b1.w);
-        *reinterpret_cast<uint4*>(srow + 16 * u) = o;
-      }
-      fence_proxy_async_smem();
-      if (row < p.M && n0 < p.N) {
-        const int ncols = (p.N - n0) < kIEpiCols ? (p.N - n0) : kIEpiCols;
-        bulk_s2g(p.Y + static_cast<size_t>(row) * p.ldy + n0, smem_u32(srow), static_cast<uint32_t>(ncols) * 2u);
-      }
-      bulk_commit();
     }
-    bulk_wait0();
-    if (!ok) *abort_flag = 1;
   }
 
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kIMmaWarp) {
     if (*abort_flag && lane == 0) {
       const unsigned long long t0 = globaltimer_ns();  // the abort-path commit lands within microseconds
       while (globaltimer_ns() - t0 < 2000000ull) {
@@ -1526,7 +1923,8 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
 }
 
 static size_t gemm_int4_smem_bytes() {
-  return 1024 + kIStages * kIPack + kIGroups * kIGrp + kISfStages * (kISfA + kISfB) + kIStaging + 256;
+  // ... staging, then 1 KB of barriers and flags, then the fused Q/K sum-of-squares slots (2 KB)
+  return 1024 + kIStages * kIPack + kIGroups * kIGrp + kISfStages * (kISfA + kISfB) + kIStaging + 1024 + 2048;
 }
 
 static cudaError_t launch_gemm_int4(const GemmArgs& a, int num_sms, cudaStream_t stream) {
@@ -1547,7 +1945,22 @@ static cudaError_t launch_gemm_int4(const GemmArgs& a, int num_sms, cudaStream_t
   p.l2 = a.l2;
   p.bias = a.bias;
   p.Y = a.Y;
+  p.qk_cols = a.qk_cols;
+  p.gamma_q = a.gamma_q;
+  p.gamma_k = a.gamma_k;
+  p.rope = a.rope;
+  p.eps = a.eps;
   const size_t smem = gemm_int4_smem_bytes();
+  // setmaxnreg.inc waits until the block's pool (launch registers x threads) holds the epilogue's
+  // share: refuse a build whose launch register count differs from the one the split assumes.
+  static const cudaError_t regs_ok = [] {
+    cudaFuncAttributes fa;
+    const cudaError_t err = cudaFuncGetAttributes(&fa, gemm_int4_kernel);
+    if (err != cudaSuccess) return err;
+    return fa.numRegs == kIRegsLaunch && fa.maxThreadsPerBlock >= kIThreads ? cudaSuccess
+                                                                            : cudaErrorInvalidConfiguration;
+  }();
+  if (regs_ok != cudaSuccess) return regs_ok;
   cudaError_t e = cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int tiles = p.MT * p.NT;
@@ -1556,7 +1969,7 @@ static cudaError_t launch_gemm_int4(const GemmArgs& a, int num_sms, cudaStream_t
   return cudaGetLastError();
 }
 
-static size_t gemm_smem_bytes() { return 1024 + kGStages * kGStage + kGStaging + 256; }
+static size_t gemm_smem_bytes() { return 1024 + kGStages * kGStage + kGStaging + 256 + 2 * kQkvHeadDim * 4; }
 
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   if (a.precision != 0) return launch_gemm_int4(a, num_sms, stream);
@@ -1570,6 +1983,18 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   p.NT = (a.N + kBN - 1) / kBN;
   p.ldy = a.ldy;
   p.bias = a.bias;
+  p.qk_cols = a.qk_cols;
+  p.gamma_q = a.gamma_q;
+  p.gamma_k = a.gamma_k;
+  p.rope = a.rope;
+  p.eps = a.eps;
+  p.il_down = a.il_down;
+  p.codes_down = a.codes_down;
+  p.sf_down = a.sf_down;
+  p.l1_down = a.l1_down;
+  p.r_down = a.r_down;
+  p.tpart = a.tpart;
+  p.mlp_smax = a.mlp_smax;
   const size_t mt = static_cast<size_t>(p.MT2) * 2, nt = static_cast<size_t>(p.NT), KB = static_cast<size_t>(p.KB);
   const size_t rr = static_cast<size_t>(a.rank);
   GemmMaps maps;
@@ -1594,12 +2019,29 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
       return cudaErrorInvalidValue;
   }
   const size_t smem = gemm_smem_bytes();
-  cudaError_t e =
-      cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  const int mode = a.mlp ? 2 : (a.qk_cols > 0 ? 1 : 0);
+  auto kernel = mode == 2 ? gemm_nvfp4_kernel<2> : (mode == 1 ? gemm_nvfp4_kernel<1> : gemm_nvfp4_kernel<0>);
+  // The epilogue warpgroups' setmaxnreg.inc waits until the block's pool holds their share, and
+  // the pool is the launch's registers a thread x threads: refuse to launch a build whose count
+  // differs from the one the split was sized for (the wait would never end).
+  auto check_regs = [](const void* k) {
+    cudaFuncAttributes fa;
+    const cudaError_t err = cudaFuncGetAttributes(&fa, k);
+    if (err != cudaSuccess) return err;
+    return fa.numRegs == kGRegsLaunch && fa.maxThreadsPerBlock >= kGThreads ? cudaSuccess
+                                                                            : cudaErrorInvalidConfiguration;
+  };
+  static const cudaError_t regs_plain = check_regs(reinterpret_cast<const void*>(gemm_nvfp4_kernel<0>));
+  static const cudaError_t regs_qkv = check_regs(reinterpret_cast<const void*>(gemm_nvfp4_kernel<1>));
+  static const cudaError_t regs_mlp = check_regs(reinterpret_cast<const void*>(gemm_nvfp4_kernel<2>));
+  cudaError_t e = mode == 2 ? regs_mlp : (mode == 1 ? regs_qkv : regs_plain);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int tiles = p.MT2 * p.NT;
   int pairs = num_sms / 2;
   if (pairs > tiles) pairs = tiles;
+  if (mode == 2 && a.mlp_pairs != pairs) return cudaErrorInvalidValue;  // the T slots were sized for it
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
   cfg.blockDim = dim3(kGThreads);
@@ -1614,7 +2056,38 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, maps, p);
+  return cudaLaunchKernelEx(&cfg, kernel, maps, p);
+}
+
+// ============================================================================ fused MLP: T of the down layer
+
+// One thread per (row, T column): the partials of the pairs whose tile ranges met the row's 256-row
+// block, both column halves, added in a fixed order (deterministic), rounded to bf16 once, stored
+// in kernel 2's T layout.  A pair's range is [p tiles / npairs, (p + 1) tiles / npairs).
+__global__ void __launch_bounds__(256) mlp_t_reduce_kernel(const float* part, int mpad, int smax, int r, int nt_up,
+                                                           int npairs, int tiles, uint8_t* t) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= mpad * r) return;
+  const int m = idx / r, i = idx - (idx / r) * r;
+  const int m2 = m / (2 * kBM);
+  auto pair_of = [&](long long tile) { return static_cast<int>(((tile + 1) * npairs - 1) / tiles); };
+  const int p0 = pair_of(static_cast<long long>(m2) * nt_up), p1 = pair_of(static_cast<long long>(m2) * nt_up + nt_up - 1);
+  const float* src = part + static_cast<size_t>(m) * 2 * smax * r + i;
+  float sum = 0.0f;
+  for (int h = 0; h < 2; ++h)
+    for (int sl = 0; sl <= p1 - p0; ++sl) sum += src[static_cast<size_t>(h * smax + sl) * r];
+  const __nv_bfloat16 b = __float2bfloat16_rn(sum);
+  *reinterpret_cast<__nv_bfloat16*>(t + static_cast<size_t>(m >> 7) * kBM * r * 2 +
+                                    lr_offset(static_cast<uint32_t>(m & 127), static_cast<uint32_t>(i), kBM, r)) = b;
+}
+
+cudaError_t launch_mlp_t_reduce(const float* part, int mpad, int smax, int r, int nt_up, int npairs, int tiles,
+                                uint8_t* t, cudaStream_t stream) {
+  const long long n = static_cast<long long>(mpad) * r;
+  if (n <= 0) return cudaSuccess;
+  mlp_t_reduce_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(part, mpad, smax, r, nt_up, npairs,
+                                                                                  tiles, t);
+  return cudaGetLastError();
 }
 
 // ============================================================================ fixed scratch
@@ -1628,21 +2101,41 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes]
 size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
 // Device address of the fixed scratch on the current device.  The host-side name of the array is
-// only a stand-in, so the address is looked up once per device (with that device current) and
-// cached.
+// only a stand-in, so the address is looked up (with the device current) once per device and
+// context, and cached: a new context on the device (after cudaDeviceReset, say) loads the module
+// again at another address, so a change of the current context triggers a fresh lookup.
+using CtxGetCurrentFn = int (*)(void**);  // cuCtxGetCurrent(CUcontext*), reached through the runtime
+
+static CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(p);
+    return static_cast<CtxGetCurrentFn>(nullptr);
+  }();
+  return fn;
+}
+
 cudaError_t noalloc_scratch_address(void** ptr) {
   static std::mutex mu;
   static void* addr[128] = {};
+  static void* ctx_of[128] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  void* ctx = nullptr;
+  CtxGetCurrentFn get_ctx = ctx_get_current();
+  if (!get_ctx || get_ctx(&ctx) != 0) return cudaErrorInitializationError;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  if (!addr[dev] || ctx_of[dev] != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
     addr[dev] = p;
+    ctx_of[dev] = ctx;
   }
   *ptr = addr[dev];
   return cudaSuccess;
@@ -1662,6 +2155,21 @@ __global__ void selftest_wait_kernel(int spin_limit) {
     for (int i = 0; i < spin_limit && !ok; ++i) ok = mbar_try_wait(&bar, 0);  // nothing ever arrives
     if (!ok) atomicOr(&g_device_error, kErrWaitSelftest);
   }
+}
+
+// The fused MLP epilogue's bf16 GELU on a list of bf16 inputs (a test hook).
+__global__ void selftest_gelu_kernel(const uint16_t* in, uint16_t* out, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    const float g = gelu_bf16(__uint_as_float(static_cast<uint32_t>(in[i]) << 16));
+    out[i] = static_cast<uint16_t>(__float_as_uint(g) >> 16);
+  }
+}
+
+cudaError_t launch_selftest_gelu(const uint16_t* in, uint16_t* out, int n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  selftest_gelu_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(in, out, n);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_selftest_wait(int spin_limit, cudaStream_t stream) {

@@ -29,7 +29,33 @@ struct GemmArgs {
   const uint8_t* l2;
   const float* bias;  // N (padded to a multiple of 256)
   uint16_t* Y;
+  // Fused RMS normalization of Q and K and rotary embedding (NVFP4 only; qk_cols = 0: off).
+  // Columns [0, qk_cols) are the Q heads then the K heads, kQkvHeadDim channels each.
+  int qk_cols = 0;
+  const float* gamma_q = nullptr;  // kQkvHeadDim
+  const float* gamma_k = nullptr;  // kQkvHeadDim
+  const float* rope = nullptr;     // M rows of kQkvHeadDim / 2 (cos, sin) pairs
+  float eps = 0.0f;
+  // Fused MLP pair (NVFP4 only; mlp = false: off): instead of Y, the epilogue writes the down
+  // layer's activation codes and scales of GELU(Y) and the fp32 partials of its T.
+  bool mlp = false;
+  const float* il_down = nullptr;  // N (= the down layer's K): the down layer's 1/lambda
+  uint8_t* codes_down = nullptr;   // the down layer's workspace: codes, scales
+  uint8_t* sf_down = nullptr;
+  const uint8_t* l1_down = nullptr;  // the down layer's L1 (kernel 1's B-operand layout)
+  int r_down = 0;                  // 0, 16 or 32
+  float* tpart = nullptr;          // [M padded][2 column halves][mlp_smax][r_down] fp32 partials of T
+  int mlp_smax = 0;                // slots per (row, column half): pairs meeting one 256-row block
+  int mlp_pairs = 0;               // CTA pairs of the up layer's kernel 2 (the slots assume it)
 };
+
+// The down layer's T from the fused MLP epilogue's partials (see the kernel), written in kernel 2's
+// T layout.
+cudaError_t launch_mlp_t_reduce(const float* part, int mpad, int smax, int r, int nt_up, int npairs, int tiles,
+                                uint8_t* t, cudaStream_t stream);
+
+// Head size of the fused QKV operator: one epilogue thread holds one row of one head.
+constexpr int kQkvHeadDim = 128;
 
 // W4A16 layer (4-bit weights in canonical row-major layout, 16-bit activations).
 struct W4A16Args {
@@ -49,6 +75,7 @@ cudaError_t launch_w4a16(const W4A16Args& a, int num_sms, cudaStream_t stream);
 // Largest K the W4A16 kernel accepts (x_hat rows are staged in shared memory).
 constexpr int kW4A16MaxK = 49152;
 cudaError_t launch_selftest_wait(int spin_limit, cudaStream_t stream);
+cudaError_t launch_selftest_gelu(const uint16_t* in, uint16_t* out, int n, cudaStream_t stream);
 cudaError_t read_and_clear_device_error(unsigned int* value, cudaStream_t stream);
 
 // Fixed-size scratch in the library's device module (for the allocation-free forward).

@@ -246,6 +246,23 @@ __host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
          | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f16 with f16 A/B and f32 D.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+  return (1u << 4)  // D format f32 (A and B format fields 0: f16)
+         | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Register reallocation between warpgroups (every thread of the warpgroup executes it): dec
+// gives registers back to the block's pool, inc waits until the pool holds enough.
+template <int kRegs>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <int kRegs>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
 // Instruction descriptor, kind::i8: signed int8 A/B, s32 D.
 __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
   return (2u << 4)     // D format s32
@@ -273,6 +290,23 @@ __device__ __forceinline__ uint32_t cvt_e4m3(float x) {
   uint16_t out;
   asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(x));
   return static_cast<uint32_t>(out) & 0xFFu;
+}
+
+// Four 8x8 b16 matrices from shared memory (lane i gives the address of row i % 8 of matrix i / 8);
+// register j of lane l holds row l / 4, elements 2 (l % 4) and 2 (l % 4) + 1 of matrix j.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t saddr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr));
+}
+
+// Warp-level D += A B, m16n8k16, bf16 inputs, fp32 accumulation (A row-major 16x16, B 16x8).
+__device__ __forceinline__ void mma_sync_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // E4M3 byte -> fp32 (exact, via f16).

@@ -145,7 +145,41 @@ svdq_status do_quant_down(const svdq_weights* w, const void* X, int M, int ldx, 
   return SVDQ_OK;
 }
 
-svdq_status do_gemm(const svdq_weights* w, int M, void* Y, int ldy, const void* ws, cudaStream_t stream) {
+// The fused MLP pair's epilogue of the up layer's kernel 2: the down layer's operands.
+struct MlpEpilogue {
+  const svdq_weights* down;
+  uint8_t* mid;  // the down layer's workspace, then the T partials
+  size_t part_offset;
+  int smax, pairs;
+};
+
+// The fused MLP's schedule of the up layer's kernel 2: CTA pairs (as the launch picks them) and the
+// T-partial slots one 256-row block can receive (pairs whose contiguous tile ranges meet it).
+struct MlpSchedule {
+  int tiles, nt, pairs, smax;
+};
+MlpSchedule mlp_schedule(const svdq_weights* up, int M) {
+  MlpSchedule s;
+  const int mt2 = (M + 2 * svdq::kBM - 1) / (2 * svdq::kBM);
+  s.nt = (up->N + svdq::kBN - 1) / svdq::kBN;
+  s.tiles = mt2 * s.nt;
+  s.pairs = up->num_sms / 2 < s.tiles ? up->num_sms / 2 : s.tiles;
+  if (s.pairs < 1) s.pairs = 1;
+  s.smax = s.nt / (s.tiles / s.pairs) + 2;
+  return s;
+}
+
+// The fused Q/K normalization and rotary embedding of kernel 2's epilogue.
+struct QkvEpilogue {
+  int qk_cols;
+  const float* gamma_q;
+  const float* gamma_k;
+  const float* rope;
+  float eps;
+};
+
+svdq_status do_gemm(const svdq_weights* w, int M, void* Y, int ldy, const void* ws, cudaStream_t stream,
+                    const QkvEpilogue* qkv = nullptr, const MlpEpilogue* mlp = nullptr) {
   if (!Y) return fail(SVDQ_ERR_INVALID_ARG, "Y is NULL");
   if (ldy < w->N || ldy % 8 != 0) return fail(SVDQ_ERR_INVALID_ARG, "ldy=%d must be >= N=%d and a multiple of 8", ldy, w->N);
   if (!aligned(Y, 16)) return fail(SVDQ_ERR_INVALID_ARG, "Y must be 16-byte aligned");
@@ -166,6 +200,25 @@ svdq_status do_gemm(const svdq_weights* w, int M, void* Y, int ldy, const void* 
   a.l2 = w->d_l2;
   a.bias = w->d_bias;
   a.Y = static_cast<uint16_t*>(Y);
+  if (qkv) {
+    a.qk_cols = qkv->qk_cols;
+    a.gamma_q = qkv->gamma_q;
+    a.gamma_k = qkv->gamma_k;
+    a.rope = qkv->rope;
+    a.eps = qkv->eps;
+  }
+  if (mlp) {
+    const svdq::WorkspaceLayout Ld = svdq::workspace_layout(M, mlp->down->K, mlp->down->rank);
+    a.mlp = true;
+    a.il_down = mlp->down->d_inv_lambda;
+    a.codes_down = mlp->mid + Ld.codes;
+    a.sf_down = mlp->mid + Ld.sf;
+    a.l1_down = mlp->down->d_l1;
+    a.r_down = mlp->down->rank;
+    a.tpart = reinterpret_cast<float*>(mlp->mid + mlp->part_offset);
+    a.mlp_smax = mlp->smax;
+    a.mlp_pairs = mlp->pairs;
+  }
   cudaError_t e = svdq::launch_gemm(a, w->num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launch of the 4-bit GEMM/up-projection kernel");
   return SVDQ_OK;
@@ -301,14 +354,8 @@ svdq_status svdq_prepare_weights(const uint16_t* W_bf16, int N, int K, const uin
     svdq::prepare_canonical(W_bf16, N, K, bias_bf16, act_absmax, quantizer_precision(params->precision), params->rank,
                             params->alpha, params->svd_iters > 0 ? params->svd_iters : 12, params->seed, w->canon);
     svdq::pack_device_layouts(w->canon, img);
-    if (params->precision == SVDQ_W4A16) {
-      // Canonical row-major codes [N][K/2] and fp32 scales [N][K/64], zero rows up to the padded N.
-      const size_t npad = static_cast<size_t>((N + svdq::kBN - 1) / svdq::kBN) * svdq::kBN;
-      img.codes.assign(npad * K / 2, 0);
-      std::memcpy(img.codes.data(), w->canon.codes_w.data(), static_cast<size_t>(N) * K / 2);
-      img.sf.assign(npad * K / svdq::kBK * svdq::kSfBytesPerRowKb, 0);
-      std::memcpy(img.sf.data(), w->canon.scales_int4.data(), sizeof(float) * static_cast<size_t>(N) * K / 64);
-    }
+    // W4A16: codes and scales in the warp-level MMA's fragment order (same sizes as above).
+    if (params->precision == SVDQ_W4A16) svdq::pack_w4a16_fragments(w->canon, img);
   } catch (const std::bad_alloc&) {
     delete w;
     return fail(SVDQ_ERR_OOM, "host allocation failed in prepare");
@@ -448,6 +495,116 @@ svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, in
   return svdq_linear_forward(w, X, M, ldx, Y, ldy, scratch, have, stream);
 }
 
+svdq_status svdq_linear_forward_qkv_norm_rope(const svdq_weights* w, const void* X, int M, int ldx, void* Y,
+                                              int ldy, const float* gamma_q, const float* gamma_k, float eps,
+                                              const float* rope, int head_dim, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  if (w && w->precision == SVDQ_W4A16)
+    return fail(SVDQ_ERR_INVALID_ARG, "the fused QKV operator runs on a W4A4 layer (NVFP4 or INT4), not W4A16");
+  if (head_dim != svdq::kQkvHeadDim)
+    return fail(SVDQ_ERR_INVALID_ARG, "head_dim=%d: the fused QKV operator supports %d", head_dim,
+                svdq::kQkvHeadDim);
+  if (w && w->N % (3 * head_dim) != 0)
+    return fail(SVDQ_ERR_INVALID_ARG, "N=%d is not 3 x heads x head_dim (head_dim=%d)", w->N, head_dim);
+  if (!(eps >= 0.0f && eps <= 3.4e38f)) return fail(SVDQ_ERR_INVALID_ARG, "eps=%g must be >= 0 and finite", eps);
+  svdq_status s = check_forward_common(w, M, workspace, workspace_bytes);
+  if (s != SVDQ_OK || M == 0) return s;
+  if (!gamma_q || !gamma_k || !rope) return fail(SVDQ_ERR_INVALID_ARG, "gamma_q, gamma_k and rope must not be NULL");
+  if (!aligned(gamma_q, 16) || !aligned(gamma_k, 16) || !aligned(rope, 16))
+    return fail(SVDQ_ERR_INVALID_ARG, "gamma_q, gamma_k and rope must be 16-byte aligned");
+  if (!Y) return fail(SVDQ_ERR_INVALID_ARG, "Y is NULL");
+  if (ldy < w->N || ldy % 8 != 0 || !aligned(Y, 16))
+    return fail(SVDQ_ERR_INVALID_ARG, "Y must be 16-byte aligned with ldy >= N and a multiple of 8");
+  DeviceGuard guard(w->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = do_quant_down(w, X, M, ldx, workspace, st);
+  if (s != SVDQ_OK) return s;
+  QkvEpilogue q;
+  q.qk_cols = 2 * (w->N / 3);
+  q.gamma_q = gamma_q;
+  q.gamma_k = gamma_k;
+  q.rope = rope;
+  q.eps = eps;
+  return do_gemm(w, M, Y, ldy, workspace, st, &q);
+}
+
+namespace {
+
+svdq_status mlp_check(const svdq_weights* up, const svdq_weights* down) {
+  if (!up || !down) return fail(SVDQ_ERR_INVALID_ARG, "weights handle is NULL");
+  if (up->precision != SVDQ_NVFP4 || down->precision != SVDQ_NVFP4)
+    return fail(SVDQ_ERR_INVALID_ARG, "the fused MLP pair runs on NVFP4 layers only");
+  if (up->N != down->K)
+    return fail(SVDQ_ERR_INVALID_ARG, "the up layer's N=%d is not the down layer's K=%d", up->N, down->K);
+  if (down->rank != 0 && down->rank != 16 && down->rank != 32)
+    return fail(SVDQ_ERR_INVALID_ARG, "the fused MLP pair supports a down-layer rank of 0, 16 or 32 (got %d)",
+                down->rank);
+  if (up->device != down->device) return fail(SVDQ_ERR_INVALID_ARG, "the two layers live on different devices");
+  return SVDQ_OK;
+}
+
+// The middle workspace: the down layer's workspace for M rows, then [M padded][2 N_up/256][r]
+// fp32 partials of its T.
+size_t mlp_part_offset(const svdq_weights* down, int M) {
+  return svdq::align_up(svdq::workspace_layout(M, down->K, down->rank).total, 1024);
+}
+size_t mlp_part_bytes(const svdq_weights* up, const svdq_weights* down, int M) {
+  const svdq::WorkspaceLayout L = svdq::workspace_layout(M, down->K, down->rank);
+  const MlpSchedule sc = mlp_schedule(up, M);
+  return static_cast<size_t>(L.m_tiles) * svdq::kBM * 2 * sc.smax * down->rank * sizeof(float);
+}
+
+}  // namespace
+
+svdq_status svdq_mlp_workspace_size(const svdq_weights* up, const svdq_weights* down, int M, size_t* bytes) {
+  if (!bytes) return fail(SVDQ_ERR_INVALID_ARG, "bytes is NULL");
+  svdq_status s = mlp_check(up, down);
+  if (s != SVDQ_OK) return s;
+  if (M < 0) return fail(SVDQ_ERR_INVALID_ARG, "M=%d is negative", M);
+  *bytes = M == 0 ? 0 : mlp_part_offset(down, M) + mlp_part_bytes(up, down, M);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_mlp_forward(const svdq_weights* up, const svdq_weights* down, const void* X, int M, int ldx,
+                             void* Y, int ldy, void* ws_up, size_t ws_up_bytes, void* ws_mid, size_t ws_mid_bytes,
+                             void* stream) {
+  svdq_status s = mlp_check(up, down);
+  if (s != SVDQ_OK) return s;
+  s = check_forward_common(up, M, ws_up, ws_up_bytes);
+  if (s != SVDQ_OK || M == 0) return s;
+  const size_t need = mlp_part_offset(down, M) + mlp_part_bytes(up, down, M);
+  if (!ws_mid) return fail(SVDQ_ERR_INVALID_ARG, "the middle workspace is NULL");
+  if (!aligned(ws_mid, 256)) return fail(SVDQ_ERR_INVALID_ARG, "the middle workspace must be 256-byte aligned");
+  if (ws_mid_bytes < need)
+    return fail(SVDQ_ERR_INVALID_ARG, "middle workspace of %zu bytes is smaller than the %zu bytes needed for M=%d",
+                ws_mid_bytes, need, M);
+  if (!Y) return fail(SVDQ_ERR_INVALID_ARG, "Y is NULL");
+  if (ldy < down->N || ldy % 8 != 0 || !aligned(Y, 16))
+    return fail(SVDQ_ERR_INVALID_ARG, "Y must be 16-byte aligned with ldy >= N and a multiple of 8");
+  DeviceGuard guard(up->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = do_quant_down(up, X, M, ldx, ws_up, st);
+  if (s != SVDQ_OK) return s;
+  MlpEpilogue m;
+  m.down = down;
+  m.mid = static_cast<uint8_t*>(ws_mid);
+  m.part_offset = mlp_part_offset(down, M);
+  const MlpSchedule sc = mlp_schedule(up, M);
+  m.smax = sc.smax;
+  m.pairs = sc.pairs;
+  // the up layer's Y is not written: its tensor map (unused) points at the middle workspace
+  s = do_gemm(up, M, ws_mid, up->N, ws_up, st, nullptr, &m);
+  if (s != SVDQ_OK) return s;
+  if (down->rank > 0) {
+    const svdq::WorkspaceLayout Ld = svdq::workspace_layout(M, down->K, down->rank);
+    cudaError_t e = svdq::launch_mlp_t_reduce(reinterpret_cast<const float*>(m.mid + m.part_offset),
+                                              Ld.m_tiles * svdq::kBM, sc.smax, down->rank, sc.nt, sc.pairs, sc.tiles,
+                                              m.mid + Ld.t, st);
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the fused MLP's T reduction");
+  }
+  return do_gemm(down, M, Y, ldy, ws_mid, st);
+}
+
 svdq_status svdq_quant_down(const svdq_weights* w, const void* X, int M, int ldx, void* workspace,
                             size_t workspace_bytes, void* stream) {
   if (w && w->precision == SVDQ_W4A16)
@@ -537,6 +694,14 @@ svdq_status svdq_selftest_wait_timeout(int spin_limit, void* stream) {
   if (spin_limit < 0) return fail(SVDQ_ERR_INVALID_ARG, "spin_limit must be >= 0");
   cudaError_t e = svdq::launch_selftest_wait(spin_limit, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "launch of the wait self-test kernel");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_selftest_gelu_bf16(const uint16_t* in, uint16_t* out, int n, void* stream) {
+  if (n < 0) return fail(SVDQ_ERR_INVALID_ARG, "n=%d is negative", n);
+  if (n > 0 && (!in || !out)) return fail(SVDQ_ERR_INVALID_ARG, "NULL buffer");
+  cudaError_t e = svdq::launch_selftest_gelu(in, out, n, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the GELU self-test kernel");
   return SVDQ_OK;
 }
 

@@ -14,119 +14,257 @@ namespace svdq {
 
 // ============================================================================ W4A16
 //
-// The "awq_w4a16" layer family: 4-bit weights (INT4, one fp32 scale per 64 elements along K, the
-// smoothed weight's codes in canonical row-major layout), 16-bit activations, for small M (the
-// modulation projections run on one token per image).  Memory bound: the weights are read once.
-// A block stages MT rows of bf16(x_hat) = bf16(fp32(x) * (1/lambda)) in shared memory as fp32;
-// each warp then computes one output row n at a time: lane l takes 8 consecutive elements of every
-// 256 (a coalesced 4-byte word of codes), converts the codes exactly to fp32, dots them with x_hat,
-// scales the partial by the group scale and accumulates in fp32; a warp reduction and the bias
-// finish the row.
+// The "awq_w4a16" layer family: 4-bit weights with one fp32 scale per 64 elements along K, 16-bit
+// activations, used where M is small (FLUX's modulation projections run on one token per image).
+// HBM bound by the weights (half a byte an element), and at that rate a weight can afford about
+// three instructions on the CUDA cores -- less than a convert-and-FMA chain needs.  So the
+// contraction runs on the warp-level bf16 tensor-core MMA (m16n8k16, fp32 accumulation) with A
+// from registers: a lane turns one 32-bit word of codes into four bf16x2 fragment registers with
+// one LOP3 each (the code, sign-flipped, into the mantissa of 128: 136 + q exactly) and one
+// bf16x2 subtract of 136 (exact); the group's four k-steps accumulate from zero and the group
+// scale multiplies the result into the fp32 accumulator.  B (the activations) is staged once per
+// CTA in shared memory in fragment order: bf16(fp32(x) * (1/lambda)).
+//
+// Work split: a CTA owns R blocks of 16 weight rows and all of K; its 8 warps take the 64-wide
+// groups in turn (split K), each keeping the next group's codes and scales in flight while it
+// computes the current one; the warps' partial sums are added in warp order in shared memory
+// (deterministic), the bias added, and Y written.  grid.y runs over passes of 8 MB rows of X.
+
+constexpr int kWThreads = 256;
+constexpr int kWWarps = kWThreads / 32;
+constexpr int kWStageBytes = 96 * 1024;  // activation fragments staged per pass over K
 
 struct W4A16Params {
   const uint16_t* X;
   int M, K, ldx, N, ldy;
   const float* inv_lambda;
-  const uint8_t* codes;
-  const float* scales;
+  const uint4* codes;    // [N/16][K/64][32] x 16 B, fragment order
+  const float2* scales;  // [N/16][K/64][8] pairs (rows i, i + 8)
   const float* bias;
   uint16_t* Y;
+  int G;        // K / 64
+  int chunk_g;  // groups whose activation fragments are staged at a time
 };
 
-template <int MT>
-__global__ void __launch_bounds__(256) w4a16_kernel(const W4A16Params p) {
-  extern __shared__ __align__(16) float xs[];  // MT x K
-  const int m0 = blockIdx.y * MT;
-  const int k8n = p.K / 8;
-  for (int i = threadIdx.x; i < MT * k8n; i += blockDim.x) {
-    const int mi = i / k8n, k8 = (i - mi * k8n) * 8;
-    float v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = 0.0f;
-    if (m0 + mi < p.M) {
-      const uint4 x = *reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(m0 + mi) * p.ldx + k8);
-      const float4 i0 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + k8));
-      const float4 i1 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + k8 + 4));
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-      const float il[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        // x_hat = fp32(x) * (1/lambda) (one rounding), then the 16-bit activation bf16(x_hat)
-        v[2 * t] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(__uint_as_float(w[t] << 16), il[2 * t])));
-        v[2 * t + 1] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(__uint_as_float(w[t] & 0xFFFF0000u), il[2 * t + 1])));
-      }
-    }
-    float4* dst = reinterpret_cast<float4*>(xs + static_cast<size_t>(mi) * p.K + k8);
-    dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-    dst[1] = make_float4(v[4], v[5], v[6], v[7]);
-  }
-  __syncthreads();
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Two codes (nibbles at bits 0-3 and 16-19 of w) -> bf16x2 of their signed values, exactly.
+__device__ __forceinline__ uint32_t codes_to_bf16x2(uint32_t w) {
+  uint32_t t;
+  // (w & 0x000F000F) ^ 0x43084308: each half becomes bf16 128 + (v ^ 8) = 136 + q
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w), "r"(0x000F000Fu), "r"(0x43084308u));
+  uint32_t q;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(t), "r"(0x43084308u));
+  return q;
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int R, int MB>
+__global__ void __launch_bounds__(kWThreads) w4a16_kernel(const W4A16Params p) {
+  extern __shared__ __align__(16) uint8_t smem_w[];
+  uint4* xs = reinterpret_cast<uint4*>(smem_w);  // [MB][chunk_g][2 halves][32 lanes]
+  float* red = reinterpret_cast<float*>(smem_w + static_cast<size_t>(MB) * p.chunk_g * 1024);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int n = blockIdx.x * 8 + warp; n < p.N; n += gridDim.x * 8) {
-    const uint32_t* crow = reinterpret_cast<const uint32_t*>(p.codes + static_cast<size_t>(n) * (p.K / 2));
-    const float* srow = p.scales + static_cast<size_t>(n) * (p.K / 64);
-    float acc[MT];
-#pragma unroll
-    for (int mi = 0; mi < MT; ++mi) acc[mi] = 0.0f;
+  const int gid = lane >> 2;
+  const int m0 = blockIdx.y * 8 * MB;
+  const int nsets = (p.N + 16 * R - 1) / (16 * R);
+  const bool one_chunk = p.G <= p.chunk_g;
+
+  // Stage B for groups [gc, gc + ng): entry (mb, group gl, half h, lane l) holds, for X row
+  // m0 + 8 mb + l / 4 and the group's k-steps 2h and 2h + 1, the registers b0, b1 of each step
+  // (element pairs at k = 16 s + 2 (l % 4) + {0, 1} and that + 8).  Filled from 16-byte loads of
+  // 8 consecutive elements of a row (item = row, 8-element unit; consecutive threads take
+  // consecutive units): their four pairs are register j = 2 (s % 2) + (k % 16 >= 8) of the four
+  // lanes 4 (m % 8) + t, t = 0..3.
+  uint32_t* const xw = reinterpret_cast<uint32_t*>(xs);
+  auto stage = [&](int gc, int ng) {
+    const int units = ng * 8;  // 8-element units of the chunk per row
+    const int items = MB * 8 * units;
 #pragma unroll 4
-    for (int k0 = lane * 8; k0 < p.K; k0 += 256) {
-      const uint32_t c = __ldg(crow + k0 / 8);  // elements k0 .. k0 + 7, element j in nibble j
-      const float s = __ldg(srow + k0 / 64);
-      float q[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        // code nibble -> its signed value exactly: (nibble ^ 8) is value + 8 in [0, 15]; placed in
-        // the low mantissa bits of 2^23 and 2^23 + 8 subtracted
-        q[j] = __uint_as_float(((c >> (4 * j)) & 0xFu) ^ 0x4B000008u) - 8388616.0f;
+    for (int e = threadIdx.x; e < items; e += kWThreads) {
+      const int ml = e / units, u = e - ml * units;  // row of the pass, unit of the chunk
+      const int m = m0 + ml;
+      const int k0 = gc * 64 + 8 * u;
+      uint32_t v[4] = {0u, 0u, 0u, 0u};
+      if (m < p.M) {
+        const uint4 xx = *reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(m) * p.ldx + k0);
+        const float4 i0 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + k0));
+        const float4 i1 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + k0 + 4));
+        v[0] = bf16x2_bits(__fmul_rn(__uint_as_float(xx.x << 16), i0.x), __fmul_rn(__uint_as_float(xx.x & 0xFFFF0000u), i0.y));
+        v[1] = bf16x2_bits(__fmul_rn(__uint_as_float(xx.y << 16), i0.z), __fmul_rn(__uint_as_float(xx.y & 0xFFFF0000u), i0.w));
+        v[2] = bf16x2_bits(__fmul_rn(__uint_as_float(xx.z << 16), i1.x), __fmul_rn(__uint_as_float(xx.z & 0xFFFF0000u), i1.y));
+        v[3] = bf16x2_bits(__fmul_rn(__uint_as_float(xx.w << 16), i1.z), __fmul_rn(__uint_as_float(xx.w & 0xFFFF0000u), i1.w));
       }
+      const int kk = 8 * u;                 // element offset inside the chunk
+      const int gl = kk >> 6, s16 = (kk >> 4) & 3, hi8 = (kk >> 3) & 1;
+      const int mb = ml >> 3, gid = ml & 7;
+      const int j = 2 * (s16 & 1) + hi8;
+      uint32_t* dst = xw + ((((mb * ng + gl) * 2 + (s16 >> 1)) * 32 + 4 * gid) * 4 + j);
 #pragma unroll
-      for (int mi = 0; mi < MT; ++mi) {
-        const float4 xa = *reinterpret_cast<const float4*>(xs + static_cast<size_t>(mi) * p.K + k0);
-        const float4 xb = *reinterpret_cast<const float4*>(xs + static_cast<size_t>(mi) * p.K + k0 + 4);
-        float part = q[0] * xa.x;
-        part = fmaf(q[1], xa.y, part);
-        part = fmaf(q[2], xa.z, part);
-        part = fmaf(q[3], xa.w, part);
-        part = fmaf(q[4], xb.x, part);
-        part = fmaf(q[5], xb.y, part);
-        part = fmaf(q[6], xb.z, part);
-        part = fmaf(q[7], xb.w, part);
-        acc[mi] = fmaf(part, s, acc[mi]);
-      }
+      for (int t = 0; t < 4; ++t) dst[4 * t] = v[t];  // lane 4 gid + t: entries of 4 words
     }
+  };
+  if (one_chunk) {
+    stage(0, p.G);
+    __syncthreads();
+  }
+
+  for (int set = blockIdx.x; set < nsets; set += gridDim.x) {
+    const int b0 = set * R;
+    float acc[R][MB][4];
 #pragma unroll
-    for (int mi = 0; mi < MT; ++mi)
+    for (int r = 0; r < R; ++r)
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[mi] += __shfl_xor_sync(0xffffffffu, acc[mi], o);
-    if (lane == 0) {
-      const float b = p.bias[n];
+      for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
-      for (int mi = 0; mi < MT; ++mi)
-        if (m0 + mi < p.M) {
-          const __nv_bfloat16 y = __float2bfloat16_rn(acc[mi] + b);
-          p.Y[static_cast<size_t>(m0 + mi) * p.ldy + n] = *reinterpret_cast<const uint16_t*>(&y);
+        for (int j = 0; j < 4; ++j) acc[r][mb][j] = 0.0f;
+
+    for (int gc = 0; gc < p.G; gc += p.chunk_g) {
+      const int ng = p.G - gc < p.chunk_g ? p.G - gc : p.chunk_g;
+      if (!one_chunk) {
+        __syncthreads();  // the previous chunk's fragments are no longer read
+        stage(gc, ng);
+        __syncthreads();
+      }
+      int gl = warp;
+      uint4 c[R];
+      float2 s[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        c[r] = make_uint4(0u, 0u, 0u, 0u);
+        s[r] = make_float2(0.0f, 0.0f);
+      }
+      if (gl < ng) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const size_t cb = static_cast<size_t>(b0 + r) * p.G + gc + gl;
+          c[r] = __ldg(p.codes + cb * 32 + lane);
+          s[r] = __ldg(p.scales + cb * 8 + gid);
         }
+      }
+      for (; gl < ng; gl += kWWarps) {
+        // the next group's codes and scales go in flight before this group's math
+        uint4 cn[R];
+        float2 sn[R];
+        const int gn = gl + kWWarps;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          cn[r] = make_uint4(0u, 0u, 0u, 0u);
+          sn[r] = make_float2(0.0f, 0.0f);
+        }
+        if (gn < ng) {
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            const size_t cb = static_cast<size_t>(b0 + r) * p.G + gc + gn;
+            cn[r] = __ldg(p.codes + cb * 32 + lane);
+            sn[r] = __ldg(p.scales + cb * 8 + gid);
+          }
+        }
+        uint4 bq[MB][2];
+#pragma unroll
+        for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) bq[mb][h] = xs[((mb * ng + gl) * 2 + h) * 32 + lane];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const uint32_t w[4] = {c[r].x, c[r].y, c[r].z, c[r].w};
+          float d[MB][4];
+#pragma unroll
+          for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) d[mb][j] = 0.0f;
+#pragma unroll
+          for (int st = 0; st < 4; ++st) {
+            uint32_t a[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) a[j] = codes_to_bf16x2(w[st] >> (4 * j));
+#pragma unroll
+            for (int mb = 0; mb < MB; ++mb) {
+              const uint4& hb = bq[mb][st >> 1];
+              const uint32_t bb0 = (st & 1) ? hb.z : hb.x;
+              const uint32_t bb1 = (st & 1) ? hb.w : hb.y;
+              mma_bf16_16816(d[mb], a, bb0, bb1);
+            }
+          }
+#pragma unroll
+          for (int mb = 0; mb < MB; ++mb) {
+            acc[r][mb][0] = fmaf(s[r].x, d[mb][0], acc[r][mb][0]);
+            acc[r][mb][1] = fmaf(s[r].x, d[mb][1], acc[r][mb][1]);
+            acc[r][mb][2] = fmaf(s[r].y, d[mb][2], acc[r][mb][2]);
+            acc[r][mb][3] = fmaf(s[r].y, d[mb][3], acc[r][mb][3]);
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          c[r] = cn[r];
+          s[r] = sn[r];
+        }
+      }
     }
+
+    // Split-K sum over the warps in warp order, bias, bf16, store.  Accumulator j of lane l is
+    // weight row 16 b + l / 4 + 8 (j / 2) and X row 8 mb + 2 (l % 4) + j % 2.
+    constexpr int kPer = R * MB * 4 * 32;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) red[warp * kPer + ((r * MB + mb) * 4 + j) * 32 + lane] = acc[r][mb][j];
+    __syncthreads();
+    for (int e = threadIdx.x; e < kPer; e += kWThreads) {
+      float sum = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kWWarps; ++w) sum += red[w * kPer + e];
+      const int l = e & 31, j = (e >> 5) & 3, rm = e >> 7;
+      const int mb = rm % MB, r = rm / MB;
+      const int n = (b0 + r) * 16 + (l >> 2) + 8 * (j >> 1);
+      const int m = m0 + 8 * mb + 2 * (l & 3) + (j & 1);
+      if (n < p.N && m < p.M) {
+        const __nv_bfloat16 y = __float2bfloat16_rn(sum + p.bias[n]);
+        p.Y[static_cast<size_t>(m) * p.ldy + n] = *reinterpret_cast<const uint16_t*>(&y);
+      }
+    }
+    __syncthreads();  // red is rewritten by the next set
   }
 }
 
-template <int MT>
-static cudaError_t launch_w4a16_mt(const W4A16Params& p, int num_sms, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(MT) * p.K * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(w4a16_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+template <int R, int MB>
+static cudaError_t launch_w4a16_rm(const W4A16Params& p0, int num_sms, cudaStream_t stream) {
+  W4A16Params p = p0;
+  const int chunk_max = kWStageBytes / (1024 * MB);
+  p.chunk_g = p.G < chunk_max ? p.G : chunk_max;
+  const size_t smem = static_cast<size_t>(MB) * p.chunk_g * 1024 + sizeof(float) * kWWarps * R * MB * 4 * 32;
+  cudaError_t e = cudaFuncSetAttribute(w4a16_kernel<R, MB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  // Rows in launches of at most 65535 row tiles (the grid's y limit).
-  constexpr int kRowsPerLaunch = 65535 * MT;
-  for (int m = 0; m < p.M; m += kRowsPerLaunch) {
-    W4A16Params q = p;
-    q.M = p.M - m < kRowsPerLaunch ? p.M - m : kRowsPerLaunch;
-    q.X = p.X + static_cast<size_t>(m) * p.ldx;
-    q.Y = p.Y + static_cast<size_t>(m) * p.ldy;
-    const int mtiles = (q.M + MT - 1) / MT;
-    int bx = (q.N + 7) / 8;
-    const int cap = num_sms * 4 / (mtiles < 4 ? mtiles : 4);
-    if (bx > cap) bx = cap > 0 ? cap : 1;
-    w4a16_kernel<MT><<<dim3(static_cast<unsigned>(bx), static_cast<unsigned>(mtiles)), 256, smem, stream>>>(q);
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, w4a16_kernel<R, MB>, kWThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const int nsets = (p.N + 16 * R - 1) / (16 * R);
+  const int ctas = nsets < per_sm * num_sms ? nsets : per_sm * num_sms;
+  const int rows_per_pass = 8 * MB;
+  // grid.y is limited to 65535 passes: larger M runs in several launches
+  constexpr int kPassesPerLaunch = 65535;
+  const int passes = (p.M + rows_per_pass - 1) / rows_per_pass;
+  for (int q0 = 0; q0 < passes; q0 += kPassesPerLaunch) {
+    W4A16Params pq = p;
+    const int np = passes - q0 < kPassesPerLaunch ? passes - q0 : kPassesPerLaunch;
+    pq.X = p.X + static_cast<size_t>(q0) * rows_per_pass * p.ldx;
+    pq.Y = p.Y + static_cast<size_t>(q0) * rows_per_pass * p.ldy;
+    pq.M = p.M - q0 * rows_per_pass;
+    w4a16_kernel<R, MB><<<dim3(static_cast<unsigned>(ctas), static_cast<unsigned>(np)), kWThreads, smem, stream>>>(pq);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -142,15 +280,21 @@ cudaError_t launch_w4a16(const W4A16Args& a, int num_sms, cudaStream_t stream) {
   p.N = a.N;
   p.ldy = a.ldy;
   p.inv_lambda = a.inv_lambda;
-  p.codes = a.codes;
-  p.scales = a.scales;
+  p.codes = reinterpret_cast<const uint4*>(a.codes);
+  p.scales = reinterpret_cast<const float2*>(a.scales);
   p.bias = a.bias;
   p.Y = a.Y;
-  // Rows of x_hat staged per block: as many as the M x K fp32 tile allows in ~192 KB, up to 4.
-  const size_t budget = 192 * 1024;
-  if (a.M >= 4 && 4 * static_cast<size_t>(a.K) * 4 <= budget) return launch_w4a16_mt<4>(p, num_sms, stream);
-  if (a.M >= 2 && 2 * static_cast<size_t>(a.K) * 4 <= budget) return launch_w4a16_mt<2>(p, num_sms, stream);
-  return launch_w4a16_mt<1>(p, num_sms, stream);
+  p.G = a.K / 64;
+  p.chunk_g = 0;
+  // Rows of X per pass: 16 (two 8-column MMA tiles share each converted A fragment) once M > 8.
+  // Weight rows per task: 64 while that still gives two tasks per SM, else 32, else 16.
+  const bool two = a.M > 8;
+  const int blocks16 = (a.N + 15) / 16;
+  if (blocks16 >= 4 * 2 * num_sms * 9 / 10)
+    return two ? launch_w4a16_rm<4, 2>(p, num_sms, stream) : launch_w4a16_rm<4, 1>(p, num_sms, stream);
+  if (blocks16 >= 2 * 2 * num_sms * 9 / 10)
+    return two ? launch_w4a16_rm<2, 2>(p, num_sms, stream) : launch_w4a16_rm<2, 1>(p, num_sms, stream);
+  return two ? launch_w4a16_rm<1, 2>(p, num_sms, stream) : launch_w4a16_rm<1, 1>(p, num_sms, stream);
 }
 
 }  // namespace svdq
