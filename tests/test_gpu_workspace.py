@@ -1,10 +1,9 @@
-"""Kernel 1's K split: the per-tile arrival counters and the last-slice reduction of T.
+"""Kernel 1's workspace and determinism.
 
-When kernel 1 splits K, every slice writes an fp32 partial of T into the workspace and counts
-itself in a per-tile counter tagged with the launch; the last slice sums the partials in slice
-order.  These tests check that the result needs no initialised workspace (garbage counters),
-that reusing a workspace gives bit-identical results, and that a CUDA-graph replay of the same
-launches (the same launch tag every time) does too.
+Kernel 1 writes every byte of the activation codes, scales and T it leaves in the workspace (the
+padded rows included) and sums its warps' shares of T in a fixed order.  These tests check that
+the result needs no initialised workspace (filled with 0xFF first), that reusing a workspace gives
+bit-identical results, and that a CUDA-graph replay of the forward does too.
 """
 import numpy as np
 import pytest
@@ -27,8 +26,8 @@ def _bf16_dev(x_bits):
 
 
 def _layer(M=512, K=3072, N=512, r=32, seed=41):
-    # M = 512 rows -> 4 row tiles, K = 3072 -> 12 k-blocks: the split is 8 slices per tile on a B200
-    spec = synth.custom("ksplit", M=M, K=K, N=N, rank=r, seed=seed)
+    # M = 512 rows, K = 3072: 32 row blocks of kernel 1, 48 chunks of 64 columns each
+    spec = synth.custom("quant_down_ws", M=M, K=K, N=N, rank=r, seed=seed)
     X = synth.activations_bf16(spec)
     lin = S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(X), "nvfp4", r)
     return spec, X, lin
@@ -40,20 +39,20 @@ def _check_T(lin, X, act):
     assert np.array_equal(act["codes_x"], cx) and np.array_equal(act["scales_x"], sx)
     T_ref = O.bf16_to_f32(O.lowrank_down(xh, ops["L1"])).astype(np.float64)
     T_gpu = O.bf16_to_f32(act["T"]).astype(np.float64)
-    # fp32 accumulation in slice order vs the exact sum, both rounded to bf16: per-element bound
+    # fp32 accumulation vs the exact sum, both rounded to bf16: per-element bound
     assert_t_close(T_gpu, T_ref, O.bf16_to_f32(O.f32_to_bf16(xh)), O.bf16_to_f32(ops["L1"]))
 
 
-def test_split_reduction_needs_no_initialised_workspace_and_repeats_bit_exactly():
+def test_quant_down_needs_no_initialised_workspace_and_repeats_bit_exactly():
     spec, X, lin = _layer()
     Xd = _bf16_dev(X)
     ws = lin.new_workspace(spec.M)
-    ws.fill_(0xFF)  # every counter starts as garbage
+    ws.fill_(0xFF)  # garbage everywhere
     lin.svdq_quant_down(Xd, spec.M, spec.K, ws, ws.numel())
     S.svdq_get_device_error()
     first = lin.svdq_export_activations(ws, spec.M)
     _check_T(lin, X, first)
-    for _ in range(2):  # the counters were reset by the last slice; the next launches start clean
+    for _ in range(2):  # the same workspace again
         lin.svdq_quant_down(Xd, spec.M, spec.K, ws, ws.numel())
         S.svdq_get_device_error()
         again = lin.svdq_export_activations(ws, spec.M)
@@ -80,7 +79,7 @@ def test_graph_replay_of_the_forward_is_bit_identical_to_eager():
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         lin.svdq_linear_forward(Xd, spec.M, spec.K, Y, spec.N, ws, ws.numel())
-    for _ in range(3):  # the same launch tag on every replay
+    for _ in range(3):
         Y.fill_(float("nan"))
         g.replay()
         torch.cuda.synchronize()

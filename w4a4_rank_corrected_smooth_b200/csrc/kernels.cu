@@ -2,14 +2,12 @@
 // Design" (b): Down Projection fused with Quantize because they read the same input; Up
 // Projection fused with 4-Bit Compute because they write the same output), for sm_100a.
 //
-// Kernel 1, quant_down: one CTA per (128-row M tile, K slice).  A TMA warp streams X (and the
-// stage's 1/lambda) into a ring of shared-memory stages; sixteen worker warps apply the smoothing
-// factor and quantize every K-group (NVFP4: UE4M3 scale per 16; INT4: fp32 scale per 64) into
-// the tiled layouts kernel 2 copies verbatim, and write bf16(x_hat) back into the stage; one warp
-// feeds it with L1 to tcgen05 bf16 MMAs that accumulate T = x_hat L1 in tensor memory.  When K
-// is split over several CTAs, each writes its fp32 partial of T and counts itself in the tile's
-// counter; the last to arrive adds the partials in slice order (so the result is deterministic)
-// and writes bf16 T once.
+// Kernel 1, quant_down: one CTA of eight warps per 16 rows of X, each warp streaming its share of
+// the rows' 64-column chunks straight into registers.  It applies the smoothing factor, quantizes
+// every K-group (NVFP4: UE4M3 scale per 16; INT4: fp32 scale per 64) into the tiled layouts
+// kernel 2 copies verbatim, and feeds bf16(x_hat) from the same registers to warp-level bf16 MMAs
+// that accumulate T = x_hat L1; the warps' shares of T are added through shared memory in a fixed
+// order and written once as bf16.
 //
 // Kernel 2, gemm (NVFP4): persistent, warp specialised, on pairs of CTAs (cta_group::2 MMAs on
 // 256 x 256 tiles).  Two producer threads stream each k-block stage (operand tiles and scale
@@ -30,48 +28,42 @@
 namespace svdq {
 
 // ============================================================================ kernel 1
+//
+// Smoothing, 4-bit activation quantization and the bf16 down projection T = bf16(x_hat) L1, with
+// X read from HBM once.  One CTA of kQdWarps warps per block of 16 rows; warp w takes the 64-column
+// chunks w, w + kQdWarps, ... of K, so the CTA sweeps its rows front to back.  Lane l (g = l / 4,
+// j = l % 4) holds rows g and g + 8 of the block and, of every chunk, the columns 8j .. 8j + 7 and
+// 32 + 8j .. 32 + 8j + 7: two 16-byte loads per row, issued one chunk ahead of their use.  Each row
+// of a warp's chunk is read by 4 lanes as 64 contiguous bytes twice.
+//
+// NVFP4: the 16-element group 2h + j / 2 of half h of a chunk lies in lanes j and j ^ 1 (one
+// shuffle for its maximum); INT4: the 64-element group is the whole chunk row (two shuffles).
+// The codes come from the same exactly bracketed quantizer as before (see quant_rows below).
+//
+// Down projection on warp-level bf16 MMAs (m16n8k16) straight from the registers that hold x_hat:
+// the MMA's sum over k does not depend on the order of k, as long as A and B share it, so MMA s of
+// half h reads, in lane j, the physical columns 32h + 8j + 4s .. + 3 where the fragment layout
+// names the logical columns 2j, 2j + 1, 2j + 8, 2j + 9.  The matching B fragment of rank column n is
+// then 8 contiguous bytes of L1's K-major layout: one 16-byte load serves both MMAs of a half.
+// Each warp accumulates its chunks' share of T for its 16 rows in fp32; at the end the warps' shares
+// are summed through shared memory in warp order (deterministic) and rounded to bf16 once.
 
-constexpr int kQdMaxStages = 8;
-constexpr int kQdWorkerWarps = 16;
-constexpr int kQdMmaWarp = kQdWorkerWarps;        // tcgen05 MMA issuer (+ TMEM owner)
-constexpr int kQdTmaWarp = kQdWorkerWarps + 1;    // TMA producer
-constexpr int kQdThreads = (kQdWorkerWarps + 2) * 32;
-constexpr uint32_t kXsBytes = kBM * 128;  // one stage of X: 128 rows x 64 bf16, 128-byte swizzle
-constexpr uint32_t kIlBytes = 64 * 4;     // the stage's 64 values of 1/lambda
-constexpr size_t kQdSmemBudget = 220 * 1024;
-// Relative nudges that bracket a correctly rounded quotient (see the worker loop).
+constexpr int kQdWarps = 8;
+constexpr int kQdThreads = kQdWarps * 32;
+constexpr int kQdRows = 16;  // rows per CTA (the MMA's M)
+// Relative nudges that bracket a correctly rounded quotient (see quant_rows).
 constexpr float kNudgeLo = 1.0f - 0x1p-20f;
 constexpr float kNudgeHi = 1.0f + 0x1p-20f;
 
 struct QdParams {
-  int M, K, rank, KB, splits, stages;
+  const uint16_t* X;
+  int ldx, M, K, KB, rank;
   const float* inv_lambda;
   const uint8_t* l1;
   uint8_t* codes;
   uint8_t* sf;
   uint8_t* t;
-  float* part;              // [m-tile][split][128][rank] fp32 partials of T (splits > 1)
-  unsigned long long* cnt;  // per m-tile: (launch epoch << 8) | slices arrived
-  unsigned long long epoch; // distinct per launch, never 0
 };
-
-// Counts this CTA's slice in the tile's counter and returns whether it was the last of `splits`.
-// The counter holds (epoch << 8) | count; a value from another launch (or uninitialised memory)
-// restarts the count, and the last CTA resets it to 0, so a replay of the same launch also starts
-// from 0.  Lock-free (a failed CAS means another slice succeeded); bounded all the same.
-__device__ __forceinline__ bool arrive_slice_counter(unsigned long long* cnt, unsigned long long epoch, int splits,
-                                                     bool* ok) {
-  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(cnt);
-  for (int it = 0; it < (1 << 20); ++it) {
-    const unsigned long long nxt = (cur >> 8) == epoch ? cur + 1 : ((epoch << 8) | 1ull);
-    const unsigned long long prev = atomicCAS(cnt, cur, nxt);
-    if (prev == cur) return static_cast<int>(nxt & 0xFFull) == splits;
-    cur = prev;
-  }
-  atomicOr(&g_device_error, kErrWaitQuantDown);
-  *ok = false;
-  return false;
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -168,386 +160,263 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-template <int PREC>
-__global__ void __launch_bounds__(kQdThreads, 1)
-    quant_down_kernel(const __grid_constant__ CUtensorMap tmap_x, const QdParams p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ float rcp_tbl[128];  // RN(1 / UE4M3 value) for every finite scale code
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int r = p.rank;
-  const int NS = p.stages;
-  const bool has_lr = r > 0;
-  const uint32_t l1_bytes = static_cast<uint32_t>(r) * 128u;
-  const uint32_t l1_stride = static_cast<uint32_t>(align_up(l1_bytes, 1024));
-  uint8_t* xs = smem;                       // NS x 16 KB (X, then bf16 x_hat in place)
-  uint8_t* l1s = smem + NS * kXsBytes;      // NS x r*128 (L1 chunk)
-  const float* ils = reinterpret_cast<const float*>(l1s + NS * l1_stride);  // NS x 64 fp32 (1/lambda chunk)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(l1s + NS * l1_stride + NS * kIlBytes);
-  uint64_t* full = bars;                    // TMA landed: X tile (+ L1 chunk)
-  uint64_t* xready = bars + NS;             // workers wrote x_hat (one arrive per worker warp)
-  uint64_t* empty = bars + 2 * NS;          // stage free again
-  uint64_t* done = bars + 3 * NS;           // all MMAs of this CTA complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+// Streaming 16-byte load of X (read once: no L1 allocation).
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* ptr) {
+  uint4 r;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(ptr));
+  return r;
+}
 
+// fp32 (>= 0) -> E4M3 byte, round to nearest even, saturating at 448 (no ordering constraint).
+__device__ __forceinline__ uint32_t cvt_e4m3_rn(float x) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(x));
+  return static_cast<uint32_t>(out) & 0xFFu;
+}
+
+// Warp-level D += A B (m16n8k16, bf16 inputs, fp32 accumulation), free to be scheduled.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// x_hat = fp32(x) * (1/lambda) of 8 bf16 values (one rounding each), as 4 fp32 pairs.
+__device__ __forceinline__ void smooth8(const uint4& w, const float4& i0, const float4& i1, uint64_t (&xp)[4]) {
+  xp[0] = f2mul(f2pack(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u)), f2pack(i0.x, i0.y));
+  xp[1] = f2mul(f2pack(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u)), f2pack(i0.z, i0.w));
+  xp[2] = f2mul(f2pack(__uint_as_float(w.z << 16), __uint_as_float(w.z & 0xFFFF0000u)), f2pack(i1.x, i1.y));
+  xp[3] = f2mul(f2pack(__uint_as_float(w.w << 16), __uint_as_float(w.w & 0xFFFF0000u)), f2pack(i1.z, i1.w));
+}
+
+__device__ __forceinline__ float absmax8(const uint64_t (&xp)[4]) {
+  float v[8];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) f2unpack(xp[t], v[2 * t], v[2 * t + 1]);
+  return fmaxf(fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))),
+               fmaxf(fmaxf(fabsf(v[4]), fabsf(v[5])), fmaxf(fabsf(v[6]), fabsf(v[7]))));
+}
+
+template <int PREC, int NTM>
+__global__ void __launch_bounds__(kQdThreads, 2) quant_down_kernel(const QdParams p) {
+  extern __shared__ float shares[];  // [kQdWarps][16][rank]: each warp's fp32 share of T
+  __shared__ float rcp_tbl[128];     // NVFP4: 1 / value of each UE4M3 code (0 for code 0)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = blockIdx.x / p.splits;
-  const int split = blockIdx.x % p.splits;
-  const int kb0 = split * p.KB / p.splits, kb1 = (split + 1) * p.KB / p.splits;
-  const int c0 = kb0 * 4, nch = (kb1 - kb0) * 4;
-  const uint32_t tmem_cols = r <= 32 ? 32u : (r <= 64 ? 64u : 128u);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&xready[s], kQdWorkerWarps);
-      mbar_init(&empty[s], has_lr ? 1 : kQdWorkerWarps);
-    }
-    mbar_init(done, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
+  const int g = lane >> 2, j = lane & 3;
+  const int r = p.rank, nt = r >> 3;
   if (PREC == 0 && threadIdx.x < 128) rcp_tbl[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __frcp_rn(e4m3_to_f32(threadIdx.x));
-  if (has_lr && warp == kQdMmaWarp) {
-    tmem_alloc(tmem_slot, tmem_cols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = has_lr ? *tmem_slot : 0u;
-  // Kernel 2 may be scheduled once every block of this grid has got here (it waits for this
-  // grid's completion before reading anything this kernel writes).
+  // Kernel 2 may be scheduled now (it waits for this grid's completion before reading anything).
   pdl_launch_dependents();
 
-  if (warp < kQdWorkerWarps) {
-    // ------------------------------------------------------------ workers
-    // Quantization is exact (codes = E2M1_rne(RN(x / s)), resp. rint(RN(x / s)) for INT4): the
-    // quotient is bracketed between x * RN(RN(1/s)(1 -+ 2^-20)); both roundings are monotonic, so
-    // when the two bracketing codes agree they are the exact codes, and otherwise (x/s within
-    // ~2^-20 of a threshold) the IEEE division decides.
+  const int m0 = blockIdx.x * kQdRows;
+  int row[2], rin[2];
+  bool live[2];
+  const uint16_t* xrow[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    row[i] = m0 + g + 8 * i;
+    rin[i] = row[i] & (kBM - 1);
+    live[i] = row[i] < p.M;  // rows past M (up to the workspace's padded end) quantize zeros
+    xrow[i] = p.X + static_cast<size_t>(live[i] ? row[i] : 0) * p.ldx + 8 * j;
+  }
+  const int mt = m0 / kBM;
+  const int nch = p.K >> 6;
+  uint8_t* const codes_t = p.codes + codes_chunk_offset(mt, 0, p.KB, kBM);
+  uint8_t* const sf_t = p.sf + sf_chunk_offset(mt, 0, p.KB, kBM);
+  const float kInv6 = __frcp_rn(6.0f);
+
+  float d[NTM > 0 ? NTM : 1][4];
+#pragma unroll
+  for (int ni = 0; ni < (NTM > 0 ? NTM : 1); ++ni) d[ni][0] = d[ni][1] = d[ni][2] = d[ni][3] = 0.0f;
+
+  uint4 cur[2][2], nxt[2][2];
+  auto load = [&](int c, uint4 (&b)[2][2]) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        b[i][h] = live[i] ? ldg_stream_v4(xrow[i] + 64 * c + 32 * h) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  if (warp < nch) load(warp, cur);
+  for (int c = warp; c < nch; c += kQdWarps) {
+    if (c + kQdWarps < nch) load(c + kQdWarps, nxt);
+    const int k0 = c << 6;
+    const int kb = k0 >> 8, kin = k0 & 255;
+    uint64_t xp[2][2][4];  // x_hat of [row][half] as fp32 pairs
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float4 i0 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + k0 + 32 * h + 8 * j));
+      const float4 i1 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + k0 + 32 * h + 8 * j + 4));
+#pragma unroll
+      for (int i = 0; i < 2; ++i) smooth8(cur[i][h], i0, i1, xp[i][h]);
+    }
+    uint8_t* const codes_kb = codes_t + static_cast<size_t>(kb) * (kBM * kRowBytes);
+    uint8_t* const sf_kb = sf_t + static_cast<size_t>(kb) * (kBM * kSfBytesPerRowKb);
     if (PREC == 0) {
-      // NVFP4: thread t of the 512 handles one 16-element group per 64-column chunk: row t / 4,
-      // group t % 4 (two swizzled 16-byte units; the quarter-warps' loads hit distinct banks).
-      const int row = warp * 8 + (lane >> 2), g = lane & 3;
-      const float kInv6 = __frcp_rn(6.0f);
-      // Per-thread constants: the two swizzled 16-byte units of the group inside a stage, and
-      // this row's code/scale positions inside a (tile, k-block) chunk.
-      const uint32_t off0 = swz128(row, g * 32), off1 = swz128(row, g * 32 + 16);
-      uint8_t* const codes_tile = p.codes + codes_chunk_offset(mt, 0, p.KB, kBM);
-      uint8_t* const sf_tile = p.sf + sf_chunk_offset(mt, 0, p.KB, kBM) + (row & 31) * 16 + (row >> 5) * 4 + g;
-      int st = 0;
-      uint32_t ph = 0;
-      for (int c = 0; c < nch; ++c) {
-        const bool ok = !*abort_flag && wait_parity_bounded(&full[st], ph, kErrWaitQuantDown);
-        if (!__all_sync(0xffffffffu, ok)) {
-          *abort_flag = 1;
-          break;
-        }
-        const int gc = c0 + c;
-        const int kb = gc >> 2, cc = gc & 3;
-        const float4* ilv = reinterpret_cast<const float4*>(ils + st * 64 + g * 16);
-        uint8_t* xt = xs + st * kXsBytes;
-        uint4* cell0 = reinterpret_cast<uint4*>(xt + off0);
-        uint4* cell1 = reinterpret_cast<uint4*>(xt + off1);
-        const uint4 xa = *cell0, xb = *cell1;
-        const uint32_t w[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-        uint64_t xp[2][4];  // x_hat as fp32 pairs: element 2t, 2t + 1 of half h in xp[h][t]
-        float pm[8];        // per-pair maxima of |x_hat|, reduced as a tree (max is exact)
+      // NVFP4: the 16-element group of half h held by lanes j and j ^ 1
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const float4 i0 = ilv[2 * h], i1 = ilv[2 * h + 1];
-          const float il[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            // bf16 -> fp32 is exact; x_hat = fp32(x) * (1/lambda), one rounding per element
-            const uint32_t ww = w[4 * h + t];
-            xp[h][t] = f2mul(f2pack(__uint_as_float(ww << 16), __uint_as_float(ww & 0xFFFF0000u)),
-                             f2pack(il[2 * t], il[2 * t + 1]));
-            float lo, hi;
-            f2unpack(xp[h][t], lo, hi);
-            pm[4 * h + t] = fmaxf(fabsf(lo), fabsf(hi));
+          float amax = absmax8(xp[i][h]);
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+          // scale code UE4M3_rne(RN(amax / 6)) and codes E2M1_rne(RN(x / s)), each bracketed
+          // between two products whose codes agree exactly when the quotient is not within ~2^-20
+          // of a rounding threshold; otherwise the IEEE divisions decide
+          const float s_est = __fmul_rn(amax, kInv6);
+          uint32_t sbits = cvt_e4m3_rn(__fmul_rn(s_est, kNudgeLo));
+          bool slow = sbits != cvt_e4m3_rn(__fmul_rn(s_est, kNudgeHi));
+          uint32_t code = 0u;
+          if (!slow && sbits != 0u) {
+            const float rr = rcp_tbl[sbits];
+            code = e2m1x8_scaled(xp[i][h], __fmul_rn(rr, kNudgeLo));
+            slow = code != e2m1x8_scaled(xp[i][h], __fmul_rn(rr, kNudgeHi));
           }
-        }
-        const float amax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-        // scale code: UE4M3_rne(RN(amax / 6)), bracketed the same way
-        const float s_est = __fmul_rn(amax, kInv6);
-        uint32_t sbits = cvt_e4m3(__fmul_rn(s_est, kNudgeLo));
-        const uint32_t sc_hi = cvt_e4m3(__fmul_rn(s_est, kNudgeHi));
-        uint2 code = make_uint2(0u, 0u);
-        bool slow = sbits != sc_hi;
-        if (!slow && sbits != 0) {
-          const float rr = rcp_tbl[sbits];
-          const float mlo = __fmul_rn(rr, kNudgeLo), mhi = __fmul_rn(rr, kNudgeHi);
-          code.x = e2m1x8_scaled(xp[0], mlo);
-          code.y = e2m1x8_scaled(xp[1], mlo);
-          slow = (code.x != e2m1x8_scaled(xp[0], mhi)) | (code.y != e2m1x8_scaled(xp[1], mhi));
-        }
-        if (slow) {  // rare: the exact quotients decide
-          float xh[2][8];
+          if (slow) {
+            float v[8];
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int t = 0; t < 4; ++t) f2unpack(xp[h][t], xh[h][2 * t], xh[h][2 * t + 1]);
-          sbits = cvt_e4m3(__fdiv_rn(amax, 6.0f));
-          const float sd = e4m3_to_f32(sbits);
-          code.x = sd != 0.0f ? e2m1x8_div(xh[0], sd) : 0u;
-          code.y = sd != 0.0f ? e2m1x8_div(xh[1], sd) : 0u;
+            for (int t = 0; t < 4; ++t) f2unpack(xp[i][h][t], v[2 * t], v[2 * t + 1]);
+            sbits = cvt_e4m3_rn(__fdiv_rn(amax, 6.0f));
+            const float sd = e4m3_to_f32(sbits);
+            code = sd != 0.0f ? e2m1x8_div(v, sd) : 0u;
+          }
+          *reinterpret_cast<uint32_t*>(codes_kb + swz128(rin[i], (kin + 32 * h + 8 * j) >> 1)) = code;
+          if ((j & 1) == 0) sf_kb[sf_nvfp4_offset(rin[i], ((kin + 32 * h) >> 4) + (j >> 1), kBM)] = static_cast<uint8_t>(sbits);
         }
-        *reinterpret_cast<uint2*>(codes_tile + static_cast<size_t>(kb) * (kBM * kRowBytes) + swz128(row, cc * 32 + g * 8)) = code;
-        sf_tile[static_cast<size_t>(kb) * (kBM * kSfBytesPerRowKb) + cc * 512] = static_cast<uint8_t>(sbits);
-        if (has_lr) {
-          uint32_t hv[8];
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              float lo, hi;
-              f2unpack(xp[h][t], lo, hi);
-              hv[4 * h + t] = pack_bf16x2(lo, hi);
-            }
-          *cell0 = make_uint4(hv[0], hv[1], hv[2], hv[3]);  // bf16(x_hat) in place: the MMA's A operand
-          *cell1 = make_uint4(hv[4], hv[5], hv[6], hv[7]);
-          fence_proxy_async_smem();
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(has_lr ? &xready[st] : &empty[st]);
-        if (++st == NS) {
-          st = 0;
-          ph ^= 1u;
-        }
-      }
     } else {
-      // INT4: lane (sub, kg) of warp w handles 8 consecutive columns (16-byte unit kg) of rows
-      // 8w + sub and 8w + 4 + sub; the 64-element group spans the 8 lanes of a row.
-      const int sub = lane >> 3, kg = lane & 7;
-      for (int c = 0; c < nch; ++c) {
-        const int st = c % NS;
-        const bool ok = !*abort_flag && wait_parity_bounded(&full[st], (c / NS) & 1, kErrWaitQuantDown);
-        if (!__all_sync(0xffffffffu, ok)) {
-          *abort_flag = 1;
-          break;
-        }
-        const int gc = c0 + c;
-        const float4 il0 = *reinterpret_cast<const float4*>(ils + st * 64 + kg * 8);
-        const float4 il1 = *reinterpret_cast<const float4*>(ils + st * 64 + kg * 8 + 4);
-        const float il[8] = {il0.x, il0.y, il0.z, il0.w, il1.x, il1.y, il1.z, il1.w};
-        const int kb = gc >> 2, cc = gc & 3;
-        uint8_t* codes_chunk = p.codes + codes_chunk_offset(mt, kb, p.KB, kBM);
-        uint8_t* sf_chunk = p.sf + sf_chunk_offset(mt, kb, p.KB, kBM);
-        uint8_t* xt = xs + st * kXsBytes;
-        int row[2];
-        uint4* cell[2];
-        float xh[2][8];
-        float amax[2];
-        uint64_t ilp[4];
+      // INT4: the 64-element group is the chunk row, spread over the four lanes j
 #pragma unroll
-        for (int t = 0; t < 4; ++t) ilp[t] = f2pack(il[2 * t], il[2 * t + 1]);
+      for (int i = 0; i < 2; ++i) {
+        float amax = fmaxf(absmax8(xp[i][0]), absmax8(xp[i][1]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const float sc = __fdiv_rn(amax, 7.0f);
+        float v[2][8];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          row[i] = warp * 8 + i * 4 + sub;
-          cell[i] = reinterpret_cast<uint4*>(xt + swz128(row[i], kg * 16));
-          const uint4 xv = *cell[i];
-          const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const uint64_t xp = f2mul(f2pack(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xFFFF0000u)), ilp[t]);
-            f2unpack(xp, xh[i][2 * t], xh[i][2 * t + 1]);
-          }
-          amax[i] = fmaxf(fmaxf(fmaxf(fabsf(xh[i][0]), fabsf(xh[i][1])), fmaxf(fabsf(xh[i][2]), fabsf(xh[i][3]))),
-                          fmaxf(fmaxf(fabsf(xh[i][4]), fabsf(xh[i][5])), fmaxf(fabsf(xh[i][6]), fabsf(xh[i][7]))));
-          amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 1));
-          amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 2));
-          amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 4));
-        }
-        uint32_t codes[2], sbits[2];
+          for (int t = 0; t < 4; ++t) f2unpack(xp[i][h][t], v[h][2 * t], v[h][2 * t + 1]);
+        uint32_t code[2] = {0u, 0u};
         bool slow = false;
-        float sc[2];
+        if (sc != 0.0f) {
+          const float rr = __frcp_rn(sc);
+          if (rr < 1e30f) {
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          sc[i] = __fdiv_rn(amax[i], 7.0f);
-          sbits[i] = __float_as_uint(sc[i]);
-          codes[i] = 0;
-          if (sc[i] != 0.0f) {
-            const float rr = __frcp_rn(sc[i]);
-            if (rr < 1e30f) {
-              const uint32_t lo = int4x8(xh[i], __fmul_rn(rr, kNudgeLo));
-              const uint32_t hi = int4x8(xh[i], __fmul_rn(rr, kNudgeHi));
-              codes[i] = lo;
-              slow |= lo != hi;
-            } else {
-              slow = true;  // tiny scale: reciprocal out of range
+            for (int h = 0; h < 2; ++h) {
+              code[h] = int4x8(v[h], __fmul_rn(rr, kNudgeLo));
+              slow |= code[h] != int4x8(v[h], __fmul_rn(rr, kNudgeHi));
             }
+          } else {
+            slow = true;  // tiny scale: its reciprocal is out of range
           }
         }
         if (slow) {
 #pragma unroll
-          for (int i = 0; i < 2; ++i) codes[i] = sc[i] != 0.0f ? int4x8_div(xh[i], sc[i]) : 0u;
+          for (int h = 0; h < 2; ++h) code[h] = int4x8_div(v[h], sc);
         }
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          *reinterpret_cast<uint32_t*>(codes_chunk + swz128(row[i], cc * 32 + kg * 4)) = codes[i];
-          if (kg == 0) reinterpret_cast<uint32_t*>(sf_chunk)[sf_int4_a_index(row[i], cc)] = sbits[i];
-          if (has_lr) {
-            uint4 hv;
-            hv.x = pack_bf16x2(xh[i][0], xh[i][1]);
-            hv.y = pack_bf16x2(xh[i][2], xh[i][3]);
-            hv.z = pack_bf16x2(xh[i][4], xh[i][5]);
-            hv.w = pack_bf16x2(xh[i][6], xh[i][7]);
-            *cell[i] = hv;  // bf16(x_hat) in place: the tile becomes the MMA's A operand
+        for (int h = 0; h < 2; ++h)
+          *reinterpret_cast<uint32_t*>(codes_kb + swz128(rin[i], (kin + 32 * h + 8 * j) >> 1)) = code[h];
+        if (j == 0) reinterpret_cast<float*>(sf_kb)[sf_int4_a_index(rin[i], kin >> 6)] = sc;
+      }
+    }
+    if (NTM > 0) {
+      __syncwarp();  // the slow paths above are divergent; the MMAs are warp-collective
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t a[2][4];
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          float v0[4], v1[4];
+          f2unpack(xp[0][h][2 * s], v0[0], v0[1]);
+          f2unpack(xp[0][h][2 * s + 1], v0[2], v0[3]);
+          f2unpack(xp[1][h][2 * s], v1[0], v1[1]);
+          f2unpack(xp[1][h][2 * s + 1], v1[2], v1[3]);
+          a[s][0] = pack_bf16x2(v0[0], v0[1]);  // row g, logical k 2j, 2j + 1
+          a[s][1] = pack_bf16x2(v1[0], v1[1]);  // row g + 8
+          a[s][2] = pack_bf16x2(v0[2], v0[3]);  // row g, logical k 2j + 8, 2j + 9
+          a[s][3] = pack_bf16x2(v1[2], v1[3]);  // row g + 8
+        }
+#pragma unroll
+        for (int ni = 0; ni < NTM; ++ni)
+          if (ni < nt) {
+            const uint4 b = __ldg(reinterpret_cast<const uint4*>(
+                p.l1 + l1_offset(static_cast<uint32_t>(k0 + 32 * h + 8 * j), static_cast<uint32_t>(8 * ni + g), r)));
+            mma_16816(d[ni], a[0], b.x, b.y);
+            mma_16816(d[ni], a[1], b.z, b.w);
           }
-        }
-        if (has_lr) fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(has_lr ? &xready[st] : &empty[st]);
       }
     }
-  } else if (warp == kQdTmaWarp) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ TMA producer
-      int issued = 0;
-      for (int c = 0; c < nch; ++c) {
-        const int st = c % NS;
-        if (c >= NS && (*abort_flag || !wait_parity_bounded(&empty[st], ((c / NS) - 1) & 1, kErrWaitQuantDown))) {
-          *abort_flag = 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&full[st], kXsBytes + kIlBytes + (has_lr ? l1_bytes : 0u));
-        tma_load_2d(xs + st * kXsBytes, &tmap_x, (c0 + c) * 64, mt * kBM, &full[st]);
-        bulk_g2s(const_cast<float*>(ils) + st * 64, p.inv_lambda + static_cast<size_t>(c0 + c) * 64, kIlBytes, &full[st]);
-        if (has_lr)
-          bulk_g2s(l1s + st * l1_stride, p.l1 + static_cast<size_t>(c0 + c) * l1_bytes, l1_bytes, &full[st]);
-        ++issued;
-      }
-      if (*abort_flag) {
-        // Let every issued copy land before the CTA can retire.
-        for (int q = (issued > NS ? issued - NS : 0); q < issued; ++q)
-          wait_parity_bounded(&full[q % NS], (q / NS) & 1, kErrWaitQuantDown);
-      }
-    }
-  } else if (has_lr && lane == 0) {
-    // ------------------------------------------------------------ MMA issuer
-    const uint32_t idesc = idesc_bf16(128, r);
-    for (int c = 0; c < nch; ++c) {
-      const int st = c % NS;
-      const uint32_t par = (c / NS) & 1;
-      if (*abort_flag || !wait_parity_bounded(&full[st], par, kErrWaitQuantDown) ||
-          !wait_parity_bounded(&xready[st], par, kErrWaitQuantDown)) {
-        *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
-      const uint64_t ad = smem_desc(smem_u32(xs + st * kXsBytes), 16, 1024, kLayoutSw128);
-      const uint64_t bd = smem_desc(smem_u32(l1s + st * l1_stride), 16, 1024, kLayoutSw128);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem_base, ad + 2 * ks, bd + 2 * ks, idesc, (c | ks) != 0 ? 1u : 0u);
-      tc_commit(&empty[st]);
-    }
-    tc_commit(done);
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) cur[i][h] = nxt[i][h];
   }
 
-  // ---------------------------------------------------------------- T epilogue
-  __syncthreads();
-  const bool aborted = *abort_flag != 0;
-  if (has_lr && warp < 4) {
-    bool ok = !aborted && wait_parity_bounded(done, 0, kErrWaitQuantDown);
-    ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-collective
-    tc_fence_after();
-    if (ok) {
-      const int row = warp * 32 + lane;
-      float* prow = p.splits > 1 ? p.part + ((static_cast<size_t>(mt) * p.splits + split) * kBM + row) * r : nullptr;
-      for (int j = 0; j < r; j += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + j, v);
-        tmem_wait_ld();
-        if (p.splits == 1) {
-          uint8_t* tt = p.t + static_cast<size_t>(mt) * kBM * r * 2;
+  if (NTM > 0) {
+    // Each warp's share of T, then the sum over warps in warp order, rounded to bf16 once.
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(v[8 * h + 0]), __uint_as_float(v[8 * h + 1]));
-            o.y = pack_bf16x2(__uint_as_float(v[8 * h + 2]), __uint_as_float(v[8 * h + 3]));
-            o.z = pack_bf16x2(__uint_as_float(v[8 * h + 4]), __uint_as_float(v[8 * h + 5]));
-            o.w = pack_bf16x2(__uint_as_float(v[8 * h + 6]), __uint_as_float(v[8 * h + 7]));
-            *reinterpret_cast<uint4*>(tt + lr_offset(row, j + 8 * h, kBM, r)) = o;
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 16; q += 4)
-            *reinterpret_cast<float4*>(prow + j + q) = make_float4(__uint_as_float(v[q]), __uint_as_float(v[q + 1]),
-                                                                   __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]));
-        }
+    for (int ni = 0; ni < NTM; ++ni)
+      if (ni < nt) {
+        float* s0 = shares + (warp * kQdRows + g) * r + 8 * ni + 2 * j;
+        *reinterpret_cast<float2*>(s0) = make_float2(d[ni][0], d[ni][1]);
+        *reinterpret_cast<float2*>(s0 + 8 * r) = make_float2(d[ni][2], d[ni][3]);
       }
-    }
-  }
-  if (has_lr && p.splits > 1) {
-    // The last slice of the tile to finish sums all slices' partials in slice order
-    // (deterministic) and writes bf16 T.  Publication: the CTA barrier orders every thread's
-    // partial stores before thread 0's GPU-scope fence, which is cumulative, and that fence
-    // before the counter update; the last slice fences again before reading.
-    __shared__ int s_last;
     __syncthreads();
-    if (threadIdx.x == 0) {
-      bool ok = !aborted;
-      __threadfence();
-      const bool last = ok && arrive_slice_counter(p.cnt + mt, p.epoch, p.splits, &ok);
-      if (last) __threadfence();
-      if (!ok) *abort_flag = 1;
-      s_last = last ? 1 : 0;
-    }
-    __syncthreads();
-    if (s_last) {
-      uint8_t* tt = p.t + static_cast<size_t>(mt) * kBM * r * 2;
-      const float* pt = p.part + static_cast<size_t>(mt) * p.splits * kBM * r;
-      const size_t slice = static_cast<size_t>(kBM) * r;
-      const int units = kBM * r / 4;
-      // Two 4-column units per thread per round, all of a round's loads issued before the sums.
-      for (int u0 = threadIdx.x; u0 < units; u0 += 2 * blockDim.x) {
-        const int u1 = u0 + blockDim.x;
-        const bool has1 = u1 < units;
-        const int o0 = u0 * 4, o1 = (has1 ? u1 : u0) * 4;
-        float4 a0 = __ldcg(reinterpret_cast<const float4*>(pt + o0));
-        float4 a1 = __ldcg(reinterpret_cast<const float4*>(pt + o1));
-        float4 x0[7], x1[7];
+    uint8_t* const tt = p.t + static_cast<size_t>(mt) * kBM * r * 2;
+    for (int e = threadIdx.x; e < kQdRows * r / 2; e += kQdThreads) {
+      const int rw = (2 * e) / r, col = (2 * e) % r;
+      float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-        for (int q = 1; q < 8; ++q)
-          if (q < p.splits) {
-            x0[q - 1] = __ldcg(reinterpret_cast<const float4*>(pt + q * slice + o0));
-            x1[q - 1] = __ldcg(reinterpret_cast<const float4*>(pt + q * slice + o1));
-          }
-#pragma unroll
-        for (int q = 1; q < 8; ++q)
-          if (q < p.splits) {
-            a0.x += x0[q - 1].x; a0.y += x0[q - 1].y; a0.z += x0[q - 1].z; a0.w += x0[q - 1].w;
-            a1.x += x1[q - 1].x; a1.y += x1[q - 1].y; a1.z += x1[q - 1].z; a1.w += x1[q - 1].w;
-          }
-        *reinterpret_cast<uint2*>(tt + lr_offset(o0 / r, o0 % r, kBM, r)) =
-            make_uint2(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w));
-        if (has1)
-          *reinterpret_cast<uint2*>(tt + lr_offset(o1 / r, o1 % r, kBM, r)) =
-              make_uint2(pack_bf16x2(a1.x, a1.y), pack_bf16x2(a1.z, a1.w));
+      for (int w = 0; w < kQdWarps; ++w) {
+        const float2 v = *reinterpret_cast<const float2*>(shares + (w * kQdRows + rw) * r + col);
+        a0 += v.x;
+        a1 += v.y;
       }
-      if (threadIdx.x == 0) atomicExch(p.cnt + mt, 0ull);
+      *reinterpret_cast<uint32_t*>(tt + lr_offset(static_cast<uint32_t>((m0 + rw) & (kBM - 1)), col, kBM, r)) =
+          pack_bf16x2(a0, a1);
     }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (has_lr && warp == kQdMmaWarp) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, tmem_cols);
   }
 }
 
-static int quant_down_stages(int r) {
-  const size_t per = kXsBytes + align_up(static_cast<size_t>(r) * 128, 1024) + kIlBytes;
-  const int ns = static_cast<int>((kQdSmemBudget - 2048) / per);
-  return ns < kQdMaxStages ? ns : kQdMaxStages;
-}
+static int quant_down_ntm(int r) { return r == 0 ? 0 : (r <= 32 ? 4 : (r <= 64 ? 8 : 16)); }
 
-static size_t quant_down_smem_bytes(int r) {
-  const int ns = quant_down_stages(r);
-  return 1024 + ns * (kXsBytes + align_up(static_cast<size_t>(r) * 128, 1024) + kIlBytes) + 256;
+cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t stream) {
+  (void)num_sms;
+  QdParams p;
+  p.X = a.X;
+  p.ldx = a.ldx;
+  p.M = a.M;
+  p.K = a.K;
+  p.KB = a.K / kBK;
+  p.rank = a.rank;
+  p.inv_lambda = a.inv_lambda;
+  p.l1 = a.l1;
+  p.codes = a.codes;
+  p.sf = a.sf;
+  p.t = a.t;
+  // Every row of the workspace's padded tiles (kernel 2 consumes rows in pairs of 128-row tiles).
+  const int mpad = 2 * kBM * ((a.M + 2 * kBM - 1) / (2 * kBM));
+  const unsigned grid = static_cast<unsigned>(mpad / kQdRows);
+  const size_t smem = static_cast<size_t>(kQdWarps) * kQdRows * a.rank * sizeof(float);
+  void (*kern)(const QdParams) = nullptr;
+  const int ntm = quant_down_ntm(a.rank);
+  if (a.precision == 0)
+    kern = ntm == 0 ? quant_down_kernel<0, 0> : ntm == 4 ? quant_down_kernel<0, 4> : ntm == 8 ? quant_down_kernel<0, 8>
+                                                                                          : quant_down_kernel<0, 16>;
+  else
+    kern = ntm == 0 ? quant_down_kernel<1, 0> : ntm == 4 ? quant_down_kernel<1, 4> : ntm == 8 ? quant_down_kernel<1, 8>
+                                                                                          : quant_down_kernel<1, 16>;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<grid, kQdThreads, smem, stream>>>(p);
+  return cudaGetLastError();
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link dependency).
@@ -567,52 +436,6 @@ static EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
-cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t stream) {
-  QdParams p;
-  p.M = a.M;
-  p.K = a.K;
-  p.rank = a.rank;
-  p.KB = a.K / kBK;
-  p.stages = quant_down_stages(a.rank);
-  p.inv_lambda = a.inv_lambda;
-  p.l1 = a.l1;
-  p.codes = a.codes;
-  p.sf = a.sf;
-  p.t = a.t;
-  EncodeTiledFn enc = encode_tiled_fn();
-  if (!enc) return cudaErrorNotSupported;
-  CUtensorMap tmap;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.M)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.ldx) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBM)};
-  const cuuint32_t estr[2] = {1, 1};
-  if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.X), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  const int mt = 2 * ((a.M + 2 * kBM - 1) / (2 * kBM));  // pairs of 128-row tiles (kernel 2 works on 256 rows)
-  const size_t smem = quant_down_smem_bytes(a.rank);
-  void (*kern)(const CUtensorMap, const QdParams) = a.precision == 0 ? quant_down_kernel<0> : quant_down_kernel<1>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  // One CTA per SM (shared memory), one wave: as many K slices per tile as the SMs allow, within
-  // what the workspace's partials have room for.
-  int splits = num_sms / mt;
-  if (splits > a.split_cap) splits = a.split_cap;
-  if (splits < 1) splits = 1;
-  if (a.rank > 0 && splits > 1 && (!a.part || !a.cnt)) splits = 1;
-  p.splits = splits;
-  p.part = a.part;
-  p.cnt = a.cnt;
-  static std::atomic<unsigned long long> epoch_counter{0};
-  p.epoch = (epoch_counter.fetch_add(1) + 1) & ((1ull << 56) - 1);
-  if (p.epoch == 0) p.epoch = 1;
-  if (a.precision == 0)
-    quant_down_kernel<0><<<mt * splits, kQdThreads, smem, stream>>>(tmap, p);
-  else
-    quant_down_kernel<1><<<mt * splits, kQdThreads, smem, stream>>>(tmap, p);
-  return cudaGetLastError();
-}
 
 
 // A byte buffer seen as a 2-D tensor of 256-byte rows, copied in boxes of `box_rows` rows (the

@@ -14,9 +14,6 @@ struct QuantDownArgs {
   uint8_t* codes;          // workspace: tiled activation codes
   uint8_t* sf;             // workspace: tiled activation scales
   uint8_t* t;              // workspace: tiled bf16 T
-  float* part;             // workspace: fp32 partials of T per K slice (split_cap > 1 and rank > 0)
-  unsigned long long* cnt; // workspace: one arrival counter per 128-row tile (same condition)
-  int split_cap;           // largest K split the partials have room for
 };
 
 struct GemmArgs {

@@ -26,13 +26,14 @@ namespace svdq {
 // CTA in shared memory in fragment order: bf16(fp32(x) * (1/lambda)).
 //
 // Work split: a CTA owns R blocks of 16 weight rows and all of K; its 8 warps take the 64-wide
-// groups in turn (split K), each keeping the next group's codes and scales in flight while it
-// computes the current one; the warps' partial sums are added in warp order in shared memory
-// (deterministic), the bias added, and Y written.  grid.y runs over passes of 8 MB rows of X.
+// groups in turn (split K), each keeping the codes and scales of its next kWAhead groups in flight
+// while it computes the current one; the warps' partial sums are added in warp order in shared
+// memory (deterministic), the bias added, and Y written.  grid.y runs over passes of 8 MB rows of X.
 
 constexpr int kWThreads = 256;
 constexpr int kWWarps = kWThreads / 32;
 constexpr int kWStageBytes = 96 * 1024;  // activation fragments staged per pass over K
+constexpr int kWAhead = 3;               // groups of codes and scales in flight per warp
 
 struct W4A16Params {
   const uint16_t* X;
@@ -136,40 +137,26 @@ __global__ void __launch_bounds__(kWThreads) w4a16_kernel(const W4A16Params p) {
         stage(gc, ng);
         __syncthreads();
       }
+      // The warp's groups gl = warp, warp + 8, ...: codes and scales of the next kWAhead groups are
+      // in flight while one group's math runs (a window of registers shifted by one group a step).
       int gl = warp;
-      uint4 c[R];
-      float2 s[R];
+      uint4 c[kWAhead][R];
+      float2 s[kWAhead][R];
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        c[r] = make_uint4(0u, 0u, 0u, 0u);
-        s[r] = make_float2(0.0f, 0.0f);
-      }
-      if (gl < ng) {
+      for (int q = 0; q < kWAhead; ++q) {
+        const int gq = gl + q * kWWarps;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          const size_t cb = static_cast<size_t>(b0 + r) * p.G + gc + gl;
-          c[r] = __ldg(p.codes + cb * 32 + lane);
-          s[r] = __ldg(p.scales + cb * 8 + gid);
+          c[q][r] = make_uint4(0u, 0u, 0u, 0u);
+          s[q][r] = make_float2(0.0f, 0.0f);
+          if (gq < ng) {
+            const size_t cb = static_cast<size_t>(b0 + r) * p.G + gc + gq;
+            c[q][r] = __ldg(p.codes + cb * 32 + lane);
+            s[q][r] = __ldg(p.scales + cb * 8 + gid);
+          }
         }
       }
       for (; gl < ng; gl += kWWarps) {
-        // the next group's codes and scales go in flight before this group's math
-        uint4 cn[R];
-        float2 sn[R];
-        const int gn = gl + kWWarps;
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          cn[r] = make_uint4(0u, 0u, 0u, 0u);
-          sn[r] = make_float2(0.0f, 0.0f);
-        }
-        if (gn < ng) {
-#pragma unroll
-          for (int r = 0; r < R; ++r) {
-            const size_t cb = static_cast<size_t>(b0 + r) * p.G + gc + gn;
-            cn[r] = __ldg(p.codes + cb * 32 + lane);
-            sn[r] = __ldg(p.scales + cb * 8 + gid);
-          }
-        }
         uint4 bq[MB][2];
 #pragma unroll
         for (int mb = 0; mb < MB; ++mb)
@@ -177,7 +164,7 @@ __global__ void __launch_bounds__(kWThreads) w4a16_kernel(const W4A16Params p) {
           for (int h = 0; h < 2; ++h) bq[mb][h] = xs[((mb * ng + gl) * 2 + h) * 32 + lane];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          const uint32_t w[4] = {c[r].x, c[r].y, c[r].z, c[r].w};
+          const uint32_t w[4] = {c[0][r].x, c[0][r].y, c[0][r].z, c[0][r].w};
           float d[MB][4];
 #pragma unroll
           for (int mb = 0; mb < MB; ++mb)
@@ -198,16 +185,27 @@ __global__ void __launch_bounds__(kWThreads) w4a16_kernel(const W4A16Params p) {
           }
 #pragma unroll
           for (int mb = 0; mb < MB; ++mb) {
-            acc[r][mb][0] = fmaf(s[r].x, d[mb][0], acc[r][mb][0]);
-            acc[r][mb][1] = fmaf(s[r].x, d[mb][1], acc[r][mb][1]);
-            acc[r][mb][2] = fmaf(s[r].y, d[mb][2], acc[r][mb][2]);
-            acc[r][mb][3] = fmaf(s[r].y, d[mb][3], acc[r][mb][3]);
+            acc[r][mb][0] = fmaf(s[0][r].x, d[mb][0], acc[r][mb][0]);
+            acc[r][mb][1] = fmaf(s[0][r].x, d[mb][1], acc[r][mb][1]);
+            acc[r][mb][2] = fmaf(s[0][r].y, d[mb][2], acc[r][mb][2]);
+            acc[r][mb][3] = fmaf(s[0][r].y, d[mb][3], acc[r][mb][3]);
           }
         }
+        const int gn = gl + kWAhead * kWWarps;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          c[r] = cn[r];
-          s[r] = sn[r];
+#pragma unroll
+          for (int q = 0; q + 1 < kWAhead; ++q) {
+            c[q][r] = c[q + 1][r];
+            s[q][r] = s[q + 1][r];
+          }
+          c[kWAhead - 1][r] = make_uint4(0u, 0u, 0u, 0u);
+          s[kWAhead - 1][r] = make_float2(0.0f, 0.0f);
+          if (gn < ng) {
+            const size_t cb = static_cast<size_t>(b0 + r) * p.G + gc + gn;
+            c[kWAhead - 1][r] = __ldg(p.codes + cb * 32 + lane);
+            s[kWAhead - 1][r] = __ldg(p.scales + cb * 8 + gid);
+          }
         }
       }
     }
