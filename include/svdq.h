@@ -177,6 +177,19 @@ svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int
 svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
                                         void* stream);
 
+/* Bytes of the packed rotary table of M tokens (M rounded up to a multiple of 32 rows of
+ * head_dim fp32).  head_dim must be 128.  Errors: INVALID_ARG. */
+svdq_status svdq_rope_packed_size(int M, int head_dim, size_t* bytes);
+
+/* Packs a rotary table for svdq_linear_forward_qkv_norm_rope.  rope: device, M rows of head_dim/2
+ * (cos, sin) fp32 pairs (row stride head_dim floats), 16-byte aligned: row m holds the angles of
+ * token m.  packed: device, >= svdq_rope_packed_size(M) bytes, 16-byte aligned, caller-owned.  The
+ * packed layout puts the same 16 bytes of 32 consecutive rows side by side, so that the epilogue's
+ * warps (one row per lane) read whole 512-byte segments; rows past M repeat row M - 1.  Asynchronous
+ * on `stream`; no allocation.  A layout change only, not in the pages.  Errors: INVALID_ARG (head_dim
+ * other than 128, NULL or misaligned pointer, buffer too small), CUDA. */
+svdq_status svdq_pack_rope(const float* rope, int M, int head_dim, float* packed, size_t packed_bytes, void* stream);
+
 /* The grouped QKV projection with its Q/K normalization and rotary embedding in one operator
  * ([ND] "Quantizing models with structural rewrites": the fused operator consumes the QKV
  * projection, norm_q, norm_k and the rotary embedding; Q, K and V are concatenated along the
@@ -191,8 +204,8 @@ svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, in
  * row of one head; INT4: half of it, the two halves exchanging their sums of squares).  NVFP4 or
  * INT4 layer, head_dim = 128 and N a multiple of 3 * 128.
  * gamma_q, gamma_k: device, head_dim fp32 each, 16-byte aligned.
- * rope: device, M rows of head_dim/2 (cos, sin) fp32 pairs (row stride head_dim floats),
- *       16-byte aligned: row m holds the angles of token m.
+ * rope: device, the rotary table of the M tokens packed by svdq_pack_rope (for this M), 16-byte
+ *       aligned.  A model computes its table once per resolution and every QKV layer reuses it.
  * eps:  >= 0 and finite (FLUX uses 1e-6).
  * Other arguments, workspace rules and errors as svdq_linear_forward; INVALID_ARG also for a
  * W4A16 layer, another head_dim, N not a multiple of 3 * head_dim, or a bad pointer. */

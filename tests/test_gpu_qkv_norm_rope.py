@@ -34,12 +34,32 @@ def _y64(Y):
     return O.bf16_to_f32(Y.view(torch.int16).cpu().numpy().view(np.uint16)).astype(np.float64)
 
 
+def _pack(rope_d, M):
+    packed = torch.empty(S.svdq_rope_packed_size(M, D) // 4, dtype=torch.float32, device="cuda")
+    S.svdq_pack_rope(rope_d, M, D, packed, packed.numel() * 4)
+    return packed
+
+
 def _inputs(M, seed):
     cos, sin = synth.rope_tables(M, D, text_tokens=min(512, M // 4), grid_w=64)
     rope = np.stack([cos, sin], axis=-1).reshape(M, D).astype(np.float32)
     gq = synth.rms_norm_weight(D, seed)
     gk = synth.rms_norm_weight(D, seed + 1)
-    return cos, sin, gq, gk, torch.from_numpy(rope).cuda(), torch.from_numpy(gq).cuda(), torch.from_numpy(gk).cuda()
+    rope_d = _pack(torch.from_numpy(rope).cuda(), M)
+    return cos, sin, gq, gk, rope_d, torch.from_numpy(gq).cuda(), torch.from_numpy(gk).cuda()
+
+
+@pytest.mark.parametrize("M", [1, 31, 32, 33, 300])
+def test_rope_packing_layout(M):
+    """svdq_pack_rope moves every value to its place: the 16-byte half hf of the 4-pair unit u of row
+    m sits at float4 ((m // 32 * 16 + u) * 2 + hf) * 32 + m % 32; rows past M repeat row M - 1."""
+    rope = np.random.default_rng(M).standard_normal((M, D)).astype(np.float32)
+    packed = _pack(torch.from_numpy(rope).cuda(), M).cpu().numpy().reshape(-1, 4)
+    rows = (M + 31) // 32 * 32
+    assert packed.shape[0] == rows * D // 4
+    src = np.concatenate([rope, np.repeat(rope[-1:], rows - M, axis=0)]).reshape(rows, D // 8, 2, 4)
+    expect = src.reshape(rows // 32, 32, D // 8, 2, 4).transpose(0, 2, 3, 1, 4).reshape(-1, 4)
+    assert np.array_equal(packed, expect)
 
 
 def _run(lin, Xd, M, gq_d, gk_d, rope_d, eps=EPS):
@@ -131,7 +151,7 @@ def test_argument_checks():
     Xd = _bf16_dev(X)
     Y = torch.empty((256, 3 * D), dtype=torch.bfloat16, device="cuda")
     for prec, hd, rp, eps in (("w4a16", D, rope_d, EPS), ("nvfp4", 64, rope_d, EPS),
-                              ("nvfp4", D, rope_d[:, 1:], EPS), ("nvfp4", D, rope_d, -1.0),
+                              ("nvfp4", D, rope_d[1:], EPS), ("nvfp4", D, rope_d, -1.0),
                               ("nvfp4", D, rope_d, float("nan"))):
         lin = S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(X), prec,
                            0 if prec == "w4a16" else 16)

@@ -70,6 +70,8 @@ def _load() -> ctypes.CDLL:
         "svdq_prepare_host": ([vp, i, i, vp, vp, ctypes.POINTER(PrepareParams), vp, vp, vp, vp, vp, vp, vp], i),
         "svdq_selftest_wait_timeout": ([i, vp], i),
         "svdq_selftest_gelu_bf16": ([vp, vp, i, vp], i),
+        "svdq_rope_packed_size": ([i, i, ctypes.POINTER(sz)], i),
+        "svdq_pack_rope": ([vp, i, i, vp, sz, vp], i),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -84,7 +86,7 @@ DECLARED_SYMBOLS = tuple(sorted([
     "svdq_free_weights", "svdq_clone_weights", "svdq_get_weights_info", "svdq_export_weights", "svdq_workspace_size", "svdq_linear_forward", "svdq_linear_forward_noalloc",
     "svdq_linear_forward_qkv_norm_rope", "svdq_mlp_workspace_size", "svdq_mlp_forward",
     "svdq_quant_down", "svdq_gemm_up", "svdq_export_activations", "svdq_quantize_rows_host", "svdq_prepare_host",
-    "svdq_selftest_wait_timeout", "svdq_selftest_gelu_bf16"]))
+    "svdq_selftest_wait_timeout", "svdq_selftest_gelu_bf16", "svdq_rope_packed_size", "svdq_pack_rope"]))
 
 
 def lib() -> ctypes.CDLL:
@@ -133,6 +135,19 @@ def svdq_get_device_error(stream=None) -> None:
 
 def svdq_selftest_wait_timeout(spin_limit: int, stream=None) -> None:
     _check(_lib.svdq_selftest_wait_timeout(spin_limit, _stream(stream)))
+
+
+def svdq_rope_packed_size(M: int, head_dim: int = 128) -> int:
+    """Bytes of the packed rotary table of M tokens (see include/svdq.h)."""
+    out = ctypes.c_size_t()
+    _check(_lib.svdq_rope_packed_size(M, head_dim, ctypes.byref(out)))
+    return out.value
+
+
+def svdq_pack_rope(rope, M: int, head_dim: int, packed, packed_bytes: int, stream=None) -> None:
+    """Packs a device rotary table (M rows of head_dim/2 (cos, sin) fp32 pairs) for the fused QKV
+    operator into the caller's device buffer ``packed``."""
+    _check(_lib.svdq_pack_rope(_ptr(rope), M, head_dim, _ptr(packed), packed_bytes, _stream(stream)))
 
 
 def svdq_selftest_gelu_bf16(inp, out, n: int, stream=None) -> None:
@@ -319,6 +334,6 @@ def svdq_mlp_forward(up: "SVDQLinear", down: "SVDQLinear", X, M: int, ldx: int, 
 
 
 __all__ = ["SVDQLinear", "SVDQError", "svdq_check_device", "svdq_get_device_error", "svdq_selftest_wait_timeout",
-           "svdq_selftest_gelu_bf16",
+           "svdq_selftest_gelu_bf16", "svdq_rope_packed_size", "svdq_pack_rope",
            "svdq_quantize_rows_host", "svdq_prepare_host", "svdq_mlp_workspace_size", "svdq_mlp_forward", "SVDQ_NVFP4",
            "SVDQ_INT4", "SVDQ_W4A16", "LIB_PATH", "lib", "DECLARED_SYMBOLS"]

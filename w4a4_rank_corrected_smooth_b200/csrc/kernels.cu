@@ -33,8 +33,10 @@ namespace svdq {
 // X read from HBM once.  One CTA of kQdWarps warps per block of 16 rows; warp w takes the 64-column
 // chunks w, w + kQdWarps, ... of K, so the CTA sweeps its rows front to back.  Lane l (g = l / 4,
 // j = l % 4) holds rows g and g + 8 of the block and, of every chunk, the columns 8j .. 8j + 7 and
-// 32 + 8j .. 32 + 8j + 7: two 16-byte loads per row, issued one chunk ahead of their use.  Each row
-// of a warp's chunk is read by 4 lanes as 64 contiguous bytes twice.
+// 32 + 8j .. 32 + 8j + 7: four 16-byte copies (each row of a warp's chunk is read by 4 lanes as 64
+// contiguous bytes twice).  The copies run kQdAhead chunks ahead of their use, asynchronously into
+// a per-warp ring in shared memory (so that a whole SM keeps ~100 KB of X in flight, which HBM's
+// latency under load needs), and each lane reads back only what it copied itself.
 //
 // NVFP4: the 16-element group 2h + j / 2 of half h of a chunk lies in lanes j and j ^ 1 (one
 // shuffle for its maximum); INT4: the 64-element group is the whole chunk row (two shuffles).
@@ -51,6 +53,11 @@ namespace svdq {
 constexpr int kQdWarps = 8;
 constexpr int kQdThreads = kQdWarps * 32;
 constexpr int kQdRows = 16;  // rows per CTA (the MMA's M)
+constexpr int kQdAhead = 4;  // chunks of X in flight per warp
+// Per-warp ring: kQdAhead + 1 slots of 4 x 32 lanes x 16 bytes; a slot is refilled one iteration
+// after its contents were read, so the read has long completed.
+constexpr uint32_t kQdSlotBytes = 4 * 32 * 16;
+constexpr uint32_t kQdRingBytes = kQdWarps * (kQdAhead + 1) * kQdSlotBytes;
 // Relative nudges that bracket a correctly rounded quotient (see quant_rows).
 constexpr float kNudgeLo = 1.0f - 0x1p-20f;
 constexpr float kNudgeHi = 1.0f + 0x1p-20f;
@@ -160,13 +167,19 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-// Streaming 16-byte load of X (read once: no L1 allocation).
-__device__ __forceinline__ uint4 ldg_stream_v4(const void* ptr) {
-  uint4 r;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-      : "l"(ptr));
-  return r;
+// 16-byte asynchronous copy global -> shared (L2 only); zero-filled when src_bytes is 0.
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* gptr, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(gptr), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+  return v;
 }
 
 // fp32 (>= 0) -> E4M3 byte, round to nearest even, saturating at 448 (no ordering constraint).
@@ -202,7 +215,9 @@ __device__ __forceinline__ float absmax8(const uint64_t (&xp)[4]) {
 
 template <int PREC, int NTM>
 __global__ void __launch_bounds__(kQdThreads, 2) quant_down_kernel(const QdParams p) {
-  extern __shared__ float shares[];  // [kQdWarps][16][rank]: each warp's fp32 share of T
+  // Dynamic shared memory: the warps' rings of X, later (after every chunk) reused for
+  // [kQdWarps][16][rank] fp32: each warp's share of T.
+  extern __shared__ __align__(16) float shares[];
   __shared__ float rcp_tbl[128];     // NVFP4: 1 / value of each UE4M3 code (0 for code 0)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, j = lane & 3;
@@ -233,17 +248,34 @@ __global__ void __launch_bounds__(kQdThreads, 2) quant_down_kernel(const QdParam
 #pragma unroll
   for (int ni = 0; ni < (NTM > 0 ? NTM : 1); ++ni) d[ni][0] = d[ni][1] = d[ni][2] = d[ni][3] = 0.0f;
 
-  uint4 cur[2][2], nxt[2][2];
-  auto load = [&](int c, uint4 (&b)[2][2]) {
+  const uint32_t ring = smem_u32(shares) + static_cast<uint32_t>(warp) * (kQdAhead + 1) * kQdSlotBytes +
+                        static_cast<uint32_t>(lane) * 16u;
+  // Chunk c into ring slot `slot` (one commit group per call, empty past the end, so that the
+  // group count stays in step with the chunks).
+  auto issue = [&](int c, int slot) {
+    if (c < nch) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          cp_async16(ring + static_cast<uint32_t>(slot) * kQdSlotBytes + (2 * i + h) * 512u, xrow[i] + 64 * c + 32 * h,
+                     live[i] ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int q = 0; q < kQdAhead; ++q) issue(warp + q * kQdWarps, q);
+  int slot = 0;
+  for (int c = warp; c < nch; c += kQdWarps) {
+    cp_async_wait<kQdAhead - 1>();  // this chunk's copies have landed
+    uint4 cur[2][2];
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-        b[i][h] = live[i] ? ldg_stream_v4(xrow[i] + 64 * c + 32 * h) : make_uint4(0u, 0u, 0u, 0u);
-  };
-  if (warp < nch) load(warp, cur);
-  for (int c = warp; c < nch; c += kQdWarps) {
-    if (c + kQdWarps < nch) load(c + kQdWarps, nxt);
+      for (int h = 0; h < 2; ++h) cur[i][h] = lds_v4(ring + static_cast<uint32_t>(slot) * kQdSlotBytes + (2 * i + h) * 512u);
+    // the slot read in the previous iteration takes the chunk kQdAhead ahead
+    issue(c + kQdAhead * kQdWarps, slot == 0 ? kQdAhead : slot - 1);
+    slot = slot == kQdAhead ? 0 : slot + 1;
     const int k0 = c << 6;
     const int kb = k0 >> 8, kin = k0 & 255;
     uint64_t xp[2][2][4];  // x_hat of [row][half] as fp32 pairs
@@ -351,14 +383,12 @@ __global__ void __launch_bounds__(kQdThreads, 2) quant_down_kernel(const QdParam
           }
       }
     }
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) cur[i][h] = nxt[i][h];
   }
+  cp_async_wait<0>();
 
   if (NTM > 0) {
     // Each warp's share of T, then the sum over warps in warp order, rounded to bf16 once.
+    __syncthreads();  // every warp is done with its ring, which the shares overwrite
 #pragma unroll
     for (int ni = 0; ni < NTM; ++ni)
       if (ni < nt) {
@@ -402,7 +432,8 @@ cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t 
   // Every row of the workspace's padded tiles (kernel 2 consumes rows in pairs of 128-row tiles).
   const int mpad = 2 * kBM * ((a.M + 2 * kBM - 1) / (2 * kBM));
   const unsigned grid = static_cast<unsigned>(mpad / kQdRows);
-  const size_t smem = static_cast<size_t>(kQdWarps) * kQdRows * a.rank * sizeof(float);
+  const size_t shares = static_cast<size_t>(kQdWarps) * kQdRows * a.rank * sizeof(float);
+  const size_t smem = shares > kQdRingBytes ? shares : kQdRingBytes;
   void (*kern)(const QdParams) = nullptr;
   const int ntm = quant_down_ntm(a.rank);
   if (a.precision == 0)
@@ -671,6 +702,12 @@ __device__ __forceinline__ float gelu_bf16(float y) {
   return __float_as_uint(lo) == __float_as_uint(hi) ? lo : gelu_bf16_slow(y);
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
@@ -806,88 +843,97 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
         const int grow = row0 + lane;
         const bool live = grow < p.M;
         const int gmt = grow >> 7, rin = grow & 127;
+        uint8_t* const cdst = p.codes_down + codes_chunk_offset(gmt, nt, p.N / kBK, kBM);
+        uint8_t* const sdst = p.sf_down + sf_chunk_offset(gmt, nt, p.N / kBK, kBM);
+        const float kInv6 = __frcp_rn(6.0f);
+        // D (mi, ni) of the T partial: rows 16 mi .. 16 mi + 15 of the warp's 32, T columns 8 ni ..
+        // 8 ni + 7 (rank <= 32)
+        const int nti = p.r_down >> 3, g8 = lane >> 2, t4 = lane & 3;
+        float d[2][4][4];
 #pragma unroll
-        for (int bx = 0; bx < 2; ++bx)
+        for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+          for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d[mi][ni][e] = 0.0f;
+#pragma unroll
+        for (int bx = 0; bx < 2; ++bx) {  // 64 columns at a time through the box
+          // the biased output rounded to bf16, into this thread's row of the box
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const int hh = u >> 2, c = 8 * (u & 3);
             const float4 b0 = ldg_f4_in_order(p.bias + n0 + 64 * bx + 8 * u);
             const float4 b1 = ldg_f4_in_order(p.bias + n0 + 64 * bx + 8 * u + 4);
-            const float4 i0 = ldg_f4_in_order(p.il_down + n0 + 64 * bx + 8 * u);
-            const float4 i1 = ldg_f4_in_order(p.il_down + n0 + 64 * bx + 8 * u + 4);
-            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            const float il[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+            st_shared_v4(srow_swz ^ (static_cast<uint32_t>(u) << 4),
+                         make_uint4(pack_bf16x2(__uint_as_float(v[bx][hh][c]) + b0.x, __uint_as_float(v[bx][hh][c + 1]) + b0.y),
+                                    pack_bf16x2(__uint_as_float(v[bx][hh][c + 2]) + b0.z, __uint_as_float(v[bx][hh][c + 3]) + b0.w),
+                                    pack_bf16x2(__uint_as_float(v[bx][hh][c + 4]) + b1.x, __uint_as_float(v[bx][hh][c + 5]) + b1.y),
+                                    pack_bf16x2(__uint_as_float(v[bx][hh][c + 6]) + b1.z, __uint_as_float(v[bx][hh][c + 7]) + b1.w)));
+          }
+          // Per 16-column group: GELU rounded to bf16, times the down layer's 1/lambda (its x_hat),
+          // quantized with kernel 1's exact rounding into the down layer's workspace; bf16(x_hat)
+          // goes back into the box for the T partial.  The loop is not unrolled, so that the GELU's
+          // temporaries stay few (only the other half's accumulator columns remain in registers).
+#pragma unroll 1
+          for (int jg = 0; jg < 4; ++jg) {
+            const uint32_t a0 = srow_swz ^ (static_cast<uint32_t>(2 * jg) << 4);
+            const uint32_t a1 = srow_swz ^ (static_cast<uint32_t>(2 * jg + 1) << 4);
+            const uint4 w0 = ld_shared_v4(a0), w1 = ld_shared_v4(a1);
+            const uint32_t wy[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            const float* ilp = p.il_down + n0 + 64 * bx + 16 * jg;
+            float il[16];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float y = __bfloat162float(__float2bfloat16_rn(__uint_as_float(v[bx][hh][c + j]) + bb[j]));
-              const float g = gelu_bf16(y);
-              v[bx][hh][c + j] = __float_as_uint(live ? __fmul_rn(g, il[j]) : 0.0f);
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const float4 t = __ldg(reinterpret_cast<const float4*>(ilp + 4 * q4));
+              il[4 * q4] = t.x;
+              il[4 * q4 + 1] = t.y;
+              il[4 * q4 + 2] = t.z;
+              il[4 * q4 + 3] = t.w;
             }
-          }
-        uint8_t* const cdst = p.codes_down + codes_chunk_offset(gmt, nt, p.N / kBK, kBM);
-        uint8_t* const sdst = p.sf_down + sf_chunk_offset(gmt, nt, p.N / kBK, kBM);
-        const float kInv6 = __frcp_rn(6.0f);
+            uint64_t xp[2][4];
+            float pm[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {  // group j: columns 16 j .. 16 j + 15
-          const int bx = j >> 2, hh = (j >> 1) & 1, e0 = 16 * (j & 1);
-          uint64_t xp[2][4];
-          float pm[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const float lo = __uint_as_float(v[bx][hh][e0 + 2 * t]), hi = __uint_as_float(v[bx][hh][e0 + 2 * t + 1]);
-            xp[t >> 2][t & 3] = f2pack(lo, hi);
-            pm[t] = fmaxf(fabsf(lo), fabsf(hi));
-          }
-          const float amax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                   fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-          const float s_est = __fmul_rn(amax, kInv6);
-          uint32_t sbits = cvt_e4m3(__fmul_rn(s_est, kNudgeLo));
-          const uint32_t sc_hi = cvt_e4m3(__fmul_rn(s_est, kNudgeHi));
-          uint2 code = make_uint2(0u, 0u);
-          bool slow = sbits != sc_hi;
-          if (!slow && sbits != 0) {
-            const float rr = __frcp_rn(e4m3_to_f32(sbits));
-            const float mlo = __fmul_rn(rr, kNudgeLo), mhi = __fmul_rn(rr, kNudgeHi);
-            code.x = e2m1x8_scaled(xp[0], mlo);
-            code.y = e2m1x8_scaled(xp[1], mlo);
-            slow = (code.x != e2m1x8_scaled(xp[0], mhi)) | (code.y != e2m1x8_scaled(xp[1], mhi));
-          }
-          if (slow) {  // rare: the exact quotients decide
+            for (int t = 0; t < 8; ++t) {
+              const float lo = live ? __fmul_rn(gelu_bf16(__uint_as_float(wy[t] << 16)), il[2 * t]) : 0.0f;
+              const float hi = live ? __fmul_rn(gelu_bf16(__uint_as_float(wy[t] & 0xFFFF0000u)), il[2 * t + 1]) : 0.0f;
+              xp[t >> 2][t & 3] = f2pack(lo, hi);
+              pm[t] = fmaxf(fabsf(lo), fabsf(hi));
+            }
+            const float amax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+            const float s_est = __fmul_rn(amax, kInv6);
+            uint32_t sbits = cvt_e4m3(__fmul_rn(s_est, kNudgeLo));
+            const uint32_t sc_hi = cvt_e4m3(__fmul_rn(s_est, kNudgeHi));
+            uint2 code = make_uint2(0u, 0u);
+            bool slow = sbits != sc_hi;
+            if (!slow && sbits != 0) {
+              const float rr = __frcp_rn(e4m3_to_f32(sbits));
+              const float mlo = __fmul_rn(rr, kNudgeLo), mhi = __fmul_rn(rr, kNudgeHi);
+              code.x = e2m1x8_scaled(xp[0], mlo);
+              code.y = e2m1x8_scaled(xp[1], mlo);
+              slow = (code.x != e2m1x8_scaled(xp[0], mhi)) | (code.y != e2m1x8_scaled(xp[1], mhi));
+            }
             float xh[2][8];
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
               for (int t = 0; t < 4; ++t) f2unpack(xp[hf][t], xh[hf][2 * t], xh[hf][2 * t + 1]);
-            sbits = cvt_e4m3(__fdiv_rn(amax, 6.0f));
-            const float sd = e4m3_to_f32(sbits);
-            code.x = sd != 0.0f ? e2m1x8_div(xh[0], sd) : 0u;
-            code.y = sd != 0.0f ? e2m1x8_div(xh[1], sd) : 0u;
-          }
-          *reinterpret_cast<uint2*>(cdst + swz128(rin, 64 * h + 8 * j)) = code;
-          sdst[sf_nvfp4_offset(rin, 8 * h + j, kBM)] = static_cast<uint8_t>(sbits);
-        }
-        if (p.r_down > 0) {
-          // D (mi, ni): rows 16 mi .. 16 mi + 15 of the warp's 32, T columns 8 ni .. 8 ni + 7 (rank <= 32)
-          const int nti = p.r_down >> 3, g8 = lane >> 2, t4 = lane & 3;
-          float d[2][4][4];
-#pragma unroll
-          for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-            for (int ni = 0; ni < 4; ++ni)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) d[mi][ni][e] = 0.0f;
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {  // 64 columns at a time through the box
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {  // unit u: columns 64 hf + 8 u .. + 7 as bf16(x_hat)
-              const int hh = u >> 2, c = 8 * (u & 3);
-              st_shared_v4(srow_swz ^ (static_cast<uint32_t>(u) << 4),
-                           make_uint4(pack_bf16x2(__uint_as_float(v[hf][hh][c]), __uint_as_float(v[hf][hh][c + 1])),
-                                      pack_bf16x2(__uint_as_float(v[hf][hh][c + 2]), __uint_as_float(v[hf][hh][c + 3])),
-                                      pack_bf16x2(__uint_as_float(v[hf][hh][c + 4]), __uint_as_float(v[hf][hh][c + 5])),
-                                      pack_bf16x2(__uint_as_float(v[hf][hh][c + 6]), __uint_as_float(v[hf][hh][c + 7]))));
+            if (slow) {  // rare: the exact quotients decide
+              sbits = cvt_e4m3(__fdiv_rn(amax, 6.0f));
+              const float sd = e4m3_to_f32(sbits);
+              code.x = sd != 0.0f ? e2m1x8_div(xh[0], sd) : 0u;
+              code.y = sd != 0.0f ? e2m1x8_div(xh[1], sd) : 0u;
             }
-            __syncwarp();
+            const int j = 4 * bx + jg;  // group j of the thread's 128 columns
+            *reinterpret_cast<uint2*>(cdst + swz128(rin, 64 * h + 8 * j)) = code;
+            sdst[sf_nvfp4_offset(rin, 8 * h + j, kBM)] = static_cast<uint8_t>(sbits);
+            st_shared_v4(a0, make_uint4(pack_bf16x2(xh[0][0], xh[0][1]), pack_bf16x2(xh[0][2], xh[0][3]),
+                                        pack_bf16x2(xh[0][4], xh[0][5]), pack_bf16x2(xh[0][6], xh[0][7])));
+            st_shared_v4(a1, make_uint4(pack_bf16x2(xh[1][0], xh[1][1]), pack_bf16x2(xh[1][2], xh[1][3]),
+                                        pack_bf16x2(xh[1][4], xh[1][5]), pack_bf16x2(xh[1][6], xh[1][7])));
+          }
+          if (p.r_down > 0) {
+            __syncwarp();  // every row of the box holds bf16(x_hat)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
               uint32_t a[2][4];
@@ -897,7 +943,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
                 const uint32_t un = 2u * ks + (lane >> 4);
                 ldmatrix_x4(a[mi], smem_u32(box) + rr * 128u + ((un ^ (rr & 7u)) << 4));
               }
-              const int kcol = n0 + 64 * hf + 16 * ks + 2 * t4;  // the down layer's k of b0
+              const int kcol = n0 + 64 * bx + 16 * ks + 2 * t4;  // the down layer's k of b0
 #pragma unroll
               for (int ni = 0; ni < 4; ++ni) {
                 if (ni < nti) {
@@ -910,8 +956,10 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
                 }
               }
             }
-            __syncwarp();  // the box is rewritten by the next half
           }
+          __syncwarp();  // the box is rewritten by the next half
+        }
+        if (p.r_down > 0) {
           // This pair's slot among the pairs whose tile ranges meet these rows (it owns the slot):
           // the first tile of the pair's run on these rows stores, the later ones add in tile order.
           const int p_first = static_cast<int>((static_cast<long long>(m2 * p.NT + 1) * npairs - 1) / tiles);
@@ -928,15 +976,15 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
                 for (int jh = 0; jh < 2; ++jh) {
                   const int rl = 16 * mi + g8 + 8 * jh;
                   float2* dst = reinterpret_cast<float2*>(tp + static_cast<size_t>(rl) * nslots * p.r_down + 8 * ni + 2 * t4);
-                  float2 v = make_float2(d[mi][ni][2 * jh], d[mi][ni][2 * jh + 1]);
+                  float2 pv = make_float2(d[mi][ni][2 * jh], d[mi][ni][2 * jh + 1]);
                   if (!seg_start) {
                     const float2 o = *dst;
-                    v = make_float2(o.x + v.x, o.y + v.y);
+                    pv = make_float2(o.x + pv.x, o.y + pv.y);
                   }
-                  *dst = v;
+                  *dst = pv;
                 }
-          fence_proxy_async_smem();  // the box's generic reads precede the next tile's bulk copies into staging
         }
+        fence_proxy_async_smem();  // the box's generic accesses precede the next tile's bulk copies into staging
       } else {
         // Fused Q/K path: the thread's 128 columns are one head of its row.  Bias first, and the
         // head's mean square; the rows past M (never stored) read the last row's angles.
@@ -967,13 +1015,13 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
             nrm = rsqrtf(fmaf(ss, 1.0f / kQkvHeadDim, p.eps));
             gam = gamma_sm + (n0 < p.qk_cols / 2 ? 0 : kQkvHeadDim);
             const int m = row0 + lane < p.M ? row0 + lane : p.M - 1;
-            rp = p.rope + static_cast<size_t>(m) * kQkvHeadDim;
-            // Each lane reads its own row of the table from L2: the loads run kRopeAhead units ahead
-            // of their use so that their latency overlaps the arithmetic of the units before.
+            // The packed table (rope_packed_index) puts the 32 rows of a warp side by side, so each
+            // of these loads reads 512 contiguous bytes; they run kRopeAhead units ahead of their use.
+            rp = p.rope + rope_packed_index(m, 0, 0);
 #pragma unroll
             for (int k = 0; k < kRopeAhead; ++k) {
-              rq[k][0] = __ldg(reinterpret_cast<const float4*>(rp + 8 * k));
-              rq[k][1] = __ldg(reinterpret_cast<const float4*>(rp + 8 * k + 4));
+              rq[k][0] = __ldg(reinterpret_cast<const float4*>(rp + rope_packed_index(0, k, 0)));
+              rq[k][1] = __ldg(reinterpret_cast<const float4*>(rp + rope_packed_index(0, k, 1)));
             }
           }
         }
@@ -993,8 +1041,8 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
               const float4 r0 = rq[slot][0];  // (cos, sin) of pairs 0, 1
               const float4 r1 = rq[slot][1];  // pairs 2, 3
               if (k + kRopeAhead < 16) {
-                rq[slot][0] = __ldg(reinterpret_cast<const float4*>(rp + 8 * (k + kRopeAhead)));
-                rq[slot][1] = __ldg(reinterpret_cast<const float4*>(rp + 8 * (k + kRopeAhead) + 4));
+                rq[slot][0] = __ldg(reinterpret_cast<const float4*>(rp + rope_packed_index(0, k + kRopeAhead, 0)));
+                rq[slot][1] = __ldg(reinterpret_cast<const float4*>(rp + rope_packed_index(0, k + kRopeAhead, 1)));
               }
               const float x0 = __uint_as_float(v[bx][hh][c + 0]) * nrm * g0.x;
               const float x1 = __uint_as_float(v[bx][hh][c + 1]) * nrm * g0.y;
@@ -1243,22 +1291,23 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
 
 // ============================================================================ kernel 2, INT4
 //
-// INT4 codes with one fp32 scale per 64 elements cannot use block-scaled MMAs, so every 64-element
-// group is its own MMA: converter warps turn the packed nibbles of a group into f16 values (exact:
-// one LOP3 puts two sign-flipped codes into the mantissas of 1024, one f16x2 subtract of 1032
-// leaves the signed values), and kind::f16 MMAs accumulate the group's partial sum -- an integer
-// of magnitude <= 4096, exact in fp32 -- in one of four TMEM buffers (the bf16 up projection T L2
-// first).  Within a group, the MMA's k order is free as long as A and B share it: a 32-bit word of
-// codes (elements e0..e7) becomes the f16 pairs (e0, e4), (e1, e5), (e2, e6), (e3, e7) on both
-// sides, with no byte shuffles.  The epilogue warps keep the fp32 accumulator in registers and add
-// each partial times RN(s_x[m,g] s_w[n,g]) with packed f32x2 arithmetic.  The k-block's scales
-// arrive by bulk copy in a ring of their own, released by the epilogue once it has applied them.
+// INT4 codes with one fp32 scale per 64 elements cannot use block-scaled MMAs.  Converter warps
+// therefore dequantize each 64-element group into bf16 operand tiles in shared memory: one LOP3
+// puts two sign-flipped codes into the mantissas of 128, a bf16x2 subtract of 136 leaves the
+// signed values (exact), and a bf16x2 multiply by the group's scale gives bf16(q s) -- the scale
+// taken to bf16 first.  bf16 MMAs (kind::f16) then accumulate the whole tile, the up projection
+// T L2 included, in one fp32 accumulator in tensor memory, double buffered so that the next tile's
+// MMAs run while the epilogue drains this one; the epilogue only adds the bias (and applies the
+// fused Q/K normalization and rotary turn).  Within a group, the MMA's k order is free as long as
+// A and B share it: a 32-bit word of codes (elements e0..e7) becomes the bf16 pairs (e0, e4),
+// (e1, e5), (e2, e6), (e3, e7) on both sides, with no byte shuffles.  Rounding each operand to
+// bf16 keeps Y within about 1e-3 (relative Frobenius) of the exact grouped sum.
 // Warp roles, four warpgroups: 0 = converters, 1 = producer, MMA issuer and two idle warps, 2 and 3
 // = epilogue; the converters and warpgroup 1 give registers to the epilogue (setmaxnreg).
 
 constexpr int kIStages = 3;                                   // packed stages
-constexpr int kIGroups = 2;                                   // f16 group buffers
-constexpr int kISlots = 4;                                    // TMEM partial buffers (128 columns each)
+constexpr int kIGroups = 2;                                   // bf16 group buffers
+constexpr int kIAcc = 2;                                      // TMEM accumulators (128 columns each)
 constexpr int kISfStages = 4;                                 // scale stages (one k-block each)
 constexpr uint32_t kISfA = kBM * 4 * 4;                       // 2 KB: fp32 [128 rows][4 groups]
 constexpr uint32_t kISfB = 4 * kBN * 4;                       // 4 KB: fp32 [4 groups][256 rows]
@@ -1304,16 +1353,19 @@ __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Eight packed int4 codes (element j in bits 4j..4j+3) -> four f16x2 registers holding the pairs
-// (e0, e4), (e1, e5), (e2, e6), (e3, e7), exactly: (w >> 4s) & 0x000F000F puts e_s and e_s+4 in the
-// low mantissa bits of two f16 halves; XOR 0x6408 sets each half to 1024 + (v ^ 8) = 1032 + q.
-__device__ __forceinline__ uint4 int4x8_to_f16_pairs(uint32_t w) {
+
+// Eight packed int4 codes (element j in bits 4j..4j+3) -> four bf16x2 registers holding the pairs
+// (e0, e4), (e1, e5), (e2, e6), (e3, e7) times the bf16 pair s2: (w >> 4s) & 0x000F000F puts e_s and
+// e_s+4 in the low mantissa bits of two bf16 halves; XOR 0x4308 makes each half 128 + (v ^ 8) =
+// 136 + q, the subtract of 136 leaves q exactly, and the multiply rounds q s once.
+__device__ __forceinline__ uint4 int4x8_to_bf16_scaled(uint32_t w, uint32_t s2) {
   uint32_t r[4];
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
-    uint32_t t;
-    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w >> (4 * s)), "r"(0x000F000Fu), "r"(0x64086408u));
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r[s]) : "r"(t), "r"(0x64086408u));
+    uint32_t t, q;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w >> (4 * s)), "r"(0x000F000Fu), "r"(0x43084308u));
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(t), "r"(0x43084308u));
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r[s]) : "r"(q), "r"(s2));
   }
   return make_uint4(r[0], r[1], r[2], r[3]);
 }
@@ -1322,7 +1374,7 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* packed = smem;                                  // kIStages x 32 KB
-  uint8_t* groups = packed + kIStages * kIPack;            // kIGroups x 32 KB
+  uint8_t* groups = packed + kIStages * kIPack;            // kIGroups x 32 KB (bf16 A, B)
   uint8_t* sfring = groups + kIGroups * kIGrp;              // kISfStages x 6 KB
   uint8_t* staging = sfring + kISfStages * (kISfA + kISfB);
   uint64_t* pfull = reinterpret_cast<uint64_t*>(staging + kIStaging);
@@ -1330,8 +1382,8 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
   uint64_t* gfull = pempty + kIStages;
   uint64_t* gempty = gfull + kIGroups;
   uint64_t* tfull = gempty + kIGroups;
-  uint64_t* tempty = tfull + kISlots;
-  uint64_t* sfull = tempty + kISlots;
+  uint64_t* tempty = tfull + kIAcc;
+  uint64_t* sfull = tempty + kIAcc;
   uint64_t* sempty = sfull + kISfStages;
   uint64_t* sspair = sempty + kISfStages;  // (fused Q/K) both column halves' sums of squares written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sspair + 4);
@@ -1353,20 +1405,20 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
       mbar_init(&gfull[s], kIConvWarps);
       mbar_init(&gempty[s], 1);
     }
-    for (int b = 0; b < kISlots; ++b) {
+    for (int b = 0; b < kIAcc; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], kIEpiWarps);
     }
     for (int b = 0; b < kISfStages; ++b) {
       mbar_init(&sfull[b], 1);
-      mbar_init(&sempty[b], kIEpiWarps);
+      mbar_init(&sempty[b], kIConvWarps);
     }
     for (int q = 0; q < 4; ++q) mbar_init(&sspair[q], 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == kIMmaWarp) {
-    tmem_alloc(tmem_slot, kISlots * kIBN);
+    tmem_alloc(tmem_slot, kIAcc * kIBN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -1376,36 +1428,27 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
 
   if (warp >= kIFirstEpiWarp) {
     setmaxnreg_inc<kIRegsEpi>();
-    // ------------------------------------------------------------ rescale + epilogue (8 warps)
+    // ------------------------------------------------------------ epilogue (8 warps)
     const int ew = warp - kIFirstEpiWarp;
     const int q = warp & 3, cg = ew >> 2;  // TMEM lane quadrant this warp may access (warp % 4), column group
     const int rloc = q * 32 + lane;
     uint8_t* srow = staging + rloc * kIStagePitch + cg * kIEpiCols * 2;
-    int slot = 0, ss = 0, qkn = 0;
-    uint32_t sph = 0;
+    int local = 0, qkn = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-      const int mt = tile / p.NT, n128 = tile % p.NT, nh = n128 & 1;
-      uint64_t acc[kIEpiCols / 2];  // this thread's fp32 accumulators as pairs
-#pragma unroll
-      for (int c = 0; c < kIEpiCols / 2; ++c) acc[c] = 0ull;
-      const int nslots = (nlr > 0 ? 1 : 0) + ngrp;
-      for (int si = 0; si < nslots; ++si) {
-        const uint32_t b = slot % kISlots;
-        const bool lr = nlr > 0 && si == 0;
-        const int g = lr ? 0 : si - (nlr > 0 ? 1 : 0);
-        const int gi = g & 3;
-        bool w = true;
-        if (lane == 0) {
-          w = !*abort_flag && wait_parity_bounded(&tfull[b], (slot / kISlots) & 1, kErrWaitGemm);
-          if (w && !lr && gi == 0) w = wait_parity_bounded(&sfull[ss], sph, kErrWaitGemm);
-        }
-        if (!__shfl_sync(0xffffffffu, w, 0)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // the slot's 64 fp32 partials of this thread's row; then the slot goes back to the MMA
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++local) {
+      const int mt = tile / p.NT, n128 = tile % p.NT;
+      const uint32_t b = static_cast<uint32_t>(local) & 1u;  // accumulator of this tile
+      bool w = true;
+      if (lane == 0)
+        w = !*abort_flag && wait_parity_bounded(&tfull[b], (static_cast<uint32_t>(local) >> 1) & 1u, kErrWaitGemm);
+      if (!__shfl_sync(0xffffffffu, w, 0)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // this thread's 64 accumulator columns of its row; then the accumulator goes back to the MMA
+      uint64_t acc[kIEpiCols / 2];  // fp32 pairs
+      {
         uint32_t v0[32], v1[32];
         const uint32_t ta = tmem + b * kIBN + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(cg * kIEpiCols);
         tmem_ld32(ta, v0);
@@ -1414,42 +1457,12 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[b]);
-        if (lr) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            acc[c] = f2pack(__uint_as_float(v0[2 * c]), __uint_as_float(v0[2 * c + 1]));
-            acc[16 + c] = f2pack(__uint_as_float(v1[2 * c]), __uint_as_float(v1[2 * c + 1]));
-          }
-        } else {
-          const uint8_t* sfb = sfring + ss * (kISfA + kISfB);
-          const float sx = reinterpret_cast<const float*>(sfb)[rloc * 4 + gi];
-          const float* swp = reinterpret_cast<const float*>(sfb + kISfA) + gi * kBN + nh * kIBN + cg * kIEpiCols;
-          const uint64_t sx2 = f2pack(sx, sx);
-#pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            const float4 sw0 = *reinterpret_cast<const float4*>(swp + c);  // same for all lanes
-            const float4 sw1 = *reinterpret_cast<const float4*>(swp + 32 + c);
-            acc[c / 2] = f2fma(f2pack(__uint_as_float(v0[c]), __uint_as_float(v0[c + 1])),
-                               f2mul(sx2, f2pack(sw0.x, sw0.y)), acc[c / 2]);
-            acc[c / 2 + 1] = f2fma(f2pack(__uint_as_float(v0[c + 2]), __uint_as_float(v0[c + 3])),
-                                   f2mul(sx2, f2pack(sw0.z, sw0.w)), acc[c / 2 + 1]);
-            acc[16 + c / 2] = f2fma(f2pack(__uint_as_float(v1[c]), __uint_as_float(v1[c + 1])),
-                                    f2mul(sx2, f2pack(sw1.x, sw1.y)), acc[16 + c / 2]);
-            acc[16 + c / 2 + 1] = f2fma(f2pack(__uint_as_float(v1[c + 2]), __uint_as_float(v1[c + 3])),
-                                        f2mul(sx2, f2pack(sw1.z, sw1.w)), acc[16 + c / 2 + 1]);
-          }
-          if (gi == 3) {  // the k-block's scales are applied
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sempty[ss]);
-            if (++ss == kISfStages) {
-              ss = 0;
-              sph ^= 1u;
-            }
-          }
+        for (int c = 0; c < 16; ++c) {
+          acc[c] = f2pack(__uint_as_float(v0[2 * c]), __uint_as_float(v0[2 * c + 1]));
+          acc[16 + c] = f2pack(__uint_as_float(v1[2 * c]), __uint_as_float(v1[2 * c + 1]));
         }
-        ++slot;
       }
-      if (!ok) break;
       // bias, bf16, stage, one bulk store per row segment
       const int row = mt * kBM + rloc;
       const int n0 = n128 * kIBN + cg * kIEpiCols;
@@ -1507,8 +1520,8 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
           const int hc = cg * kIEpiCols + u * 8;  // the head's channel of a[0]
           const float4 g0 = __ldg(reinterpret_cast<const float4*>(gam + hc));
           const float4 g1 = __ldg(reinterpret_cast<const float4*>(gam + hc + 4));
-          const float4 r0 = __ldg(reinterpret_cast<const float4*>(p.rope + static_cast<size_t>(mrope) * 128 + hc));
-          const float4 r1 = __ldg(reinterpret_cast<const float4*>(p.rope + static_cast<size_t>(mrope) * 128 + hc + 4));
+          const float4 r0 = __ldg(reinterpret_cast<const float4*>(p.rope + rope_packed_index(mrope, hc >> 3, 0)));
+          const float4 r1 = __ldg(reinterpret_cast<const float4*>(p.rope + rope_packed_index(mrope, hc >> 3, 1)));
           const float x0 = a[0] * nrm * g0.x, x1 = a[1] * nrm * g0.y, x2 = a[2] * nrm * g0.z, x3 = a[3] * nrm * g0.w;
           const float x4 = a[4] * nrm * g1.x, x5 = a[5] * nrm * g1.y, x6 = a[6] * nrm * g1.z, x7 = a[7] * nrm * g1.w;
           o.x = pack_bf16x2(x0 * r0.x - x1 * r0.y, x0 * r0.y + x1 * r0.x);
@@ -1540,10 +1553,11 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
     // After an abort a warp skips its work but still passes every named barrier, so the four
     // converter warps always execute the same barrier sequence.
     const int t = threadIdx.x;  // 0..127: one row of A and one of B
-    int st = 0, gs = 0;
-    uint32_t ph = 0, gph = 0;
+    int st = 0, gs = 0, ss = 0;
+    uint32_t ph = 0, gph = 0, sph = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+      const int nh = (tile % p.NT) & 1;  // this CTA's half of the 256-row weight tile
       for (int j = 0; j < nst; ++j) {
         if (j < nlr) {  // low-rank stages go straight to the MMA
           if (++st == kIStages) {
@@ -1553,9 +1567,14 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
           continue;
         }
         bool w = ok;
-        if (lane == 0 && w) w = !*abort_flag && wait_parity_bounded(&pfull[st], ph, kErrWaitGemm);
+        if (lane == 0 && w) {
+          w = !*abort_flag && wait_parity_bounded(&pfull[st], ph, kErrWaitGemm);
+          if (w) w = wait_parity_bounded(&sfull[ss], sph, kErrWaitGemm);  // the k-block's scales
+        }
         ok = __shfl_sync(0xffffffffu, w, 0);
         const uint8_t* pk = packed + st * kIPack;
+        const float* sfa = reinterpret_cast<const float*>(sfring + ss * (kISfA + kISfB));
+        const float* sfb = sfa + kISfA / 4;
         for (int gi = 0; gi < 4; ++gi) {
           bool e = ok;
           if (lane == 0 && e) e = !*abort_flag && wait_parity_bounded(&gempty[gs], gph ^ 1u, kErrWaitGemm);
@@ -1566,17 +1585,19 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
             for (int op = 0; op < 2; ++op) {  // A then B: row t of each
               const uint8_t* src = pk + op * kIPackA;
               uint8_t* dst = gb + op * kIGrpA;
-              // row t of the group: eight 16-byte f16 units (one per packed 32-bit word), unit u
+              const float sc = op == 0 ? sfa[sf_int4_a_index(t, gi)] : sfb[sf_int4_b_index(nh * kIBN + t, gi)];
+              const uint32_t s2 = pack_bf16x2(sc, sc);
+              // row t of the group: eight 16-byte bf16 units (one per packed 32-bit word), unit u
               // at core matrix (t / 8, u) of the no-swizzle K-major layout (128 bytes between core
               // matrices along K, 1024 bytes per 8-row block)
               const uint32_t base = (t >> 3) * 1024u + (t & 7) * 16u;
 #pragma unroll
               for (int jj = 0; jj < 2; ++jj) {  // two packed 16-byte units = 64 codes of the group
                 const uint4 v = *reinterpret_cast<const uint4*>(src + swz128(t, (2 * gi + jj) * 16));
-                *reinterpret_cast<uint4*>(dst + base + (4 * jj + 0) * 128u) = int4x8_to_f16_pairs(v.x);
-                *reinterpret_cast<uint4*>(dst + base + (4 * jj + 1) * 128u) = int4x8_to_f16_pairs(v.y);
-                *reinterpret_cast<uint4*>(dst + base + (4 * jj + 2) * 128u) = int4x8_to_f16_pairs(v.z);
-                *reinterpret_cast<uint4*>(dst + base + (4 * jj + 3) * 128u) = int4x8_to_f16_pairs(v.w);
+                *reinterpret_cast<uint4*>(dst + base + (4 * jj + 0) * 128u) = int4x8_to_bf16_scaled(v.x, s2);
+                *reinterpret_cast<uint4*>(dst + base + (4 * jj + 1) * 128u) = int4x8_to_bf16_scaled(v.y, s2);
+                *reinterpret_cast<uint4*>(dst + base + (4 * jj + 2) * 128u) = int4x8_to_bf16_scaled(v.z, s2);
+                *reinterpret_cast<uint4*>(dst + base + (4 * jj + 3) * 128u) = int4x8_to_bf16_scaled(v.w, s2);
               }
             }
             fence_proxy_async_smem();
@@ -1587,6 +1608,12 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
             gs = 0;
             gph ^= 1u;
           }
+        }
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive(&sempty[ss]);  // this warp has read the k-block's scales
+        if (++ss == kISfStages) {
+          ss = 0;
+          sph ^= 1u;
         }
         named_bar(1, kIConvWarps * 32);  // every converter finished reading this packed stage
         if (t == 0 && ok) mbar_arrive(&pempty[st]);
@@ -1666,19 +1693,22 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
     } else if (warp == kIMmaWarp) {
       if (lane == 0) {
         // ------------------------------------------------------------ MMA issuer
-        const uint32_t id_lr = idesc_bf16(128, kIBN);
-        const uint32_t id_f16 = idesc_f16(128, kIBN);
-        int st = 0, gs = 0, slot = 0;
+        const uint32_t id_bf16 = idesc_bf16(128, kIBN);
+        int st = 0, gs = 0, local = 0;
         uint32_t ph = 0, gph = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-          // low-rank slot: T L2 in fp32 into TMEM buffer (slot % kISlots)
+        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++local) {
+          const uint32_t b = static_cast<uint32_t>(local) & 1u;
+          const uint32_t acc_t = tmem + b * kIBN;
+          if (*abort_flag ||
+              !wait_parity_bounded(&tempty[b], ((static_cast<uint32_t>(local) >> 1) & 1u) ^ 1u, kErrWaitGemm)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t accum = 0;
+          // the up projection T L2 first, then every 64-element group, all into this accumulator
           for (int j = 0; j < nlr && ok; ++j) {
-            const uint32_t b = slot % kISlots;
-            if (j == 0 && (*abort_flag || !wait_parity_bounded(&tempty[b], ((slot / kISlots) & 1) ^ 1u, kErrWaitGemm))) {
-              ok = false;
-              break;
-            }
             if (*abort_flag || !wait_parity_bounded(&pfull[st], ph, kErrWaitGemm)) {
               ok = false;
               break;
@@ -1688,23 +1718,18 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
             const uint32_t sb = smem_u32(packed + st * kIPack);
             const uint64_t ad = smem_desc(sb, 128, cw * 16, kLayoutNone);
             const uint64_t bd = smem_desc(sb + kIPackA, 128, cw * 16, kLayoutNone);
-            for (uint32_t ks = 0; ks < cw / 16; ++ks)
-              mma_bf16(tmem + b * kIBN, ad + 16 * ks, bd + 16 * ks, id_lr, (j | ks) != 0 ? 1u : 0u);
+            for (uint32_t ks = 0; ks < cw / 16; ++ks) {
+              mma_bf16(acc_t, ad + 16 * ks, bd + 16 * ks, id_bf16, accum);
+              accum = 1;
+            }
             tc_commit(&pempty[st]);
             if (++st == kIStages) {
               st = 0;
               ph ^= 1u;
             }
-            if (j == nlr - 1) {
-              tc_commit(&tfull[b]);
-              ++slot;
-            }
           }
-          // one slot per 64-element group
           for (int g = 0; g < ngrp && ok; ++g) {
-            const uint32_t b = slot % kISlots;
-            if (*abort_flag || !wait_parity_bounded(&tempty[b], ((slot / kISlots) & 1) ^ 1u, kErrWaitGemm) ||
-                !wait_parity_bounded(&gfull[gs], gph, kErrWaitGemm)) {
+            if (*abort_flag || !wait_parity_bounded(&gfull[gs], gph, kErrWaitGemm)) {
               ok = false;
               break;
             }
@@ -1713,16 +1738,17 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
             const uint64_t ad = smem_desc(gb, 128, 1024, kLayoutNone);
             const uint64_t bd = smem_desc(gb + kIGrpA, 128, 1024, kLayoutNone);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // 16 f16 of K per MMA: 2 core matrices (256 bytes) on
-              mma_bf16(tmem + b * kIBN, ad + 16 * ks, bd + 16 * ks, id_f16, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks) {  // 16 bf16 of K per MMA: 2 core matrices (256 bytes) on
+              mma_bf16(acc_t, ad + 16 * ks, bd + 16 * ks, id_bf16, accum);
+              accum = 1;
+            }
             tc_commit(&gempty[gs]);
-            tc_commit(&tfull[b]);
-            ++slot;
             if (++gs == kIGroups) {
               gs = 0;
               gph ^= 1u;
             }
           }
+          if (ok) tc_commit(&tfull[b]);
         }
         if (!ok) {
           *abort_flag = 1;
@@ -1741,7 +1767,7 @@ __global__ void __launch_bounds__(kIThreads, 1) gemm_int4_kernel(const GemmI4Par
     }
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kISlots * kIBN);
+    tmem_dealloc(tmem, kIAcc * kIBN);
   }
 }
 
@@ -1978,6 +2004,26 @@ __global__ void selftest_wait_kernel(int spin_limit) {
     for (int i = 0; i < spin_limit && !ok; ++i) ok = mbar_try_wait(&bar, 0);  // nothing ever arrives
     if (!ok) atomicOr(&g_device_error, kErrWaitSelftest);
   }
+}
+
+// The rotary table into the fused QKV epilogue's layout (rope_packed_index); rows past M, up to the
+// next multiple of 32, repeat row M - 1.
+__global__ void rope_pack_kernel(const float4* rope, int M, int rows, float4* packed) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;  // one float4 of the packed table
+  if (i >= rows * (kQkvHeadDim / 4)) return;
+  const int lane = i & 31, hf = (i >> 5) & 1, unit = (i >> 6) & (kQkvHeadDim / 8 - 1);
+  const int row = (i / (32 * kQkvHeadDim / 4)) * 32 + lane;
+  const int src = row < M ? row : M - 1;
+  packed[i] = rope[static_cast<size_t>(src) * (kQkvHeadDim / 4) + 2 * unit + hf];
+}
+
+cudaError_t launch_rope_pack(const float* rope, int M, float* packed, cudaStream_t stream) {
+  if (M <= 0) return cudaSuccess;
+  const int rows = (M + 31) / 32 * 32;
+  const int n = rows * (kQkvHeadDim / 4);
+  rope_pack_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(rope), M, rows, reinterpret_cast<float4*>(packed));
+  return cudaGetLastError();
 }
 
 // The fused MLP epilogue's bf16 GELU on a list of bf16 inputs (a test hook).

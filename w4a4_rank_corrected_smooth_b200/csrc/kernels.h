@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "layout.h"
+
 namespace svdq {
 
 struct QuantDownArgs {
@@ -53,6 +55,17 @@ cudaError_t launch_mlp_t_reduce(const float* part, int mpad, int smax, int r, in
 
 // Head size of the fused QKV operator: one epilogue thread holds one row of one head.
 constexpr int kQkvHeadDim = 128;
+
+// The fused QKV operator's rotary table: for each block of 32 rows, each 16-byte half (hf) of each
+// group of 4 (cos, sin) pairs (unit) of the 32 rows side by side, so that a warp whose lanes hold
+// the block's rows reads 512 contiguous bytes per unit half.  Index of the float4 in floats:
+SVDQ_HD constexpr size_t rope_packed_index(int row, int unit, int hf) {
+  return ((static_cast<size_t>(row >> 5) * (kQkvHeadDim / 8) + static_cast<size_t>(unit)) * 2 + hf) * 128 +
+         static_cast<size_t>(row & 31) * 4;
+}
+// Bytes of the packed table for M rows (rounded up to a multiple of 32).
+constexpr size_t rope_packed_bytes(int M) { return static_cast<size_t>((M + 31) / 32 * 32) * kQkvHeadDim * 4; }
+cudaError_t launch_rope_pack(const float* rope, int M, float* packed, cudaStream_t stream);
 
 // W4A16 layer (4-bit weights in canonical row-major layout, 16-bit activations).
 struct W4A16Args {

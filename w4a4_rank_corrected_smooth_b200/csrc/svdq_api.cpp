@@ -492,6 +492,30 @@ svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, in
   return svdq_linear_forward(w, X, M, ldx, Y, ldy, scratch, have, stream);
 }
 
+svdq_status svdq_rope_packed_size(int M, int head_dim, size_t* bytes) {
+  if (!bytes) return fail(SVDQ_ERR_INVALID_ARG, "NULL argument");
+  if (M < 0) return fail(SVDQ_ERR_INVALID_ARG, "M=%d is negative", M);
+  if (head_dim != svdq::kQkvHeadDim)
+    return fail(SVDQ_ERR_INVALID_ARG, "head_dim=%d: the fused QKV operator supports %d", head_dim, svdq::kQkvHeadDim);
+  *bytes = svdq::rope_packed_bytes(M);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_pack_rope(const float* rope, int M, int head_dim, float* packed, size_t packed_bytes, void* stream) {
+  size_t need = 0;
+  svdq_status s = svdq_rope_packed_size(M, head_dim, &need);
+  if (s != SVDQ_OK || M == 0) return s;
+  if (!rope || !packed) return fail(SVDQ_ERR_INVALID_ARG, "rope and packed must not be NULL");
+  if (!aligned(rope, 16) || !aligned(packed, 16))
+    return fail(SVDQ_ERR_INVALID_ARG, "rope and packed must be 16-byte aligned");
+  if (packed_bytes < need)
+    return fail(SVDQ_ERR_INVALID_ARG, "packed buffer of %zu bytes is smaller than the %zu bytes needed for M=%d",
+                packed_bytes, need, M);
+  cudaError_t e = svdq::launch_rope_pack(rope, M, packed, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the rotary-table packing kernel");
+  return SVDQ_OK;
+}
+
 svdq_status svdq_linear_forward_qkv_norm_rope(const svdq_weights* w, const void* X, int M, int ldx, void* Y,
                                               int ldy, const float* gamma_q, const float* gamma_k, float eps,
                                               const float* rope, int head_dim, void* workspace,
