@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per FLUX-shaped layer and per point of the M x rank sweep (not the driver's line)")
+    ap.add_argument("--leg", choices=["w4a16", "mlp_pair"], default=None,
+                    help="run one auxiliary leg alone and print its JSON line (not the driver's line; profiling)")
     return ap.parse_args()
 
 
@@ -899,6 +901,25 @@ def mlp_pair_leg(dev, stream, peaks, steps: int = 200):
     return out
 
 
+def run_leg(args):
+    """One auxiliary leg on GPU 0, alone (used to profile its kernel): the W4A16 modulation
+    projections or FLUX's MLP pair, fused against unfused."""
+    import torch
+
+    import w4a4_rank_corrected_smooth_b200 as S
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    S.svdq_check_device(0)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+    if args.leg == "w4a16":
+        out = w4a16_leg(dev, stream, peaks, peak_src, launches=max(3, args.steps))
+    else:
+        out = mlp_pair_leg(dev, stream, peaks, steps=max(3, args.steps))
+    print(json.dumps({"leg": args.leg, args.leg: out}), flush=True)
+
+
 def main():
     args = parse_args()
     world, _, _ = dist_info()
@@ -906,6 +927,8 @@ def main():
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args)
+    elif args.leg:
+        run_leg(args)
     elif args.sweep:
         run_sweep(args)
     else:
