@@ -170,6 +170,16 @@ class ClockSampler:
 # ---------------------------------------------------------------- helpers
 
 
+def hold_gpu(stream, us: float):
+    """Keeps the GPU busy for about ``us`` microseconds (a spin kernel on ``stream``), so that the
+    host can queue the launches of a timed region before the region starts: the timed region then
+    measures the GPU, not the host's launch latency."""
+    import torch
+
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(min(max(us, 20.0), 50000.0) * 2000))  # ~2 GHz SM clock
+
+
 def bf16_device(x_bits, device):
     import numpy as np
     import torch
@@ -335,6 +345,7 @@ def time_loop(layers, sets, steps, stream, sample_every: int = 8):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     samples = []
+    hold_gpu(stream, 40.0 * steps)
     start.record(stream)
     for i in range(steps):
         lin = layers[i % len(layers)]
@@ -373,6 +384,7 @@ def kernel_times(layers, sets, stream, launches: int = 200):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     evs = []
+    hold_gpu(stream, 40.0 * launches)
     start.record(stream)
     for i in range(launches):
         lin = layers[i % len(layers)]
@@ -429,6 +441,7 @@ def qkv_norm_rope_leg(layers, sets, spec, stream, steps):
         run(fused)  # warm-up of this variant
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
+        hold_gpu(stream, 40.0 * steps)
         a.record(stream)
         run(fused)
         b.record(stream)
@@ -538,6 +551,7 @@ def unfused_comparator(lin, layers, sets, layers0, sets0, steps, stream, k2_bare
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
+        hold_gpu(stream, 60.0 * steps)
         e0.record(stream)
         fn(steps)
         e1.record(stream)
@@ -591,6 +605,7 @@ def w4a16_leg(dev, stream, peaks, peak_src, launches: int = 200):
         ts = []
         for _ in range(launches):
             flush.sum()
+            hold_gpu(stream, 200.0)  # the launch is queued before the timed region starts
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
@@ -884,6 +899,7 @@ def mlp_pair_leg(dev, stream, peaks, steps: int = 200):
             fn(sets[i % 2])
         a = torch.cuda.Event(enable_timing=True)
         e = torch.cuda.Event(enable_timing=True)
+        hold_gpu(stream, 80.0 * steps)
         a.record(stream)
         for i in range(steps):
             fn(sets[i % 2])
