@@ -41,7 +41,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=30)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
@@ -51,7 +51,7 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per FLUX-shaped layer and per point of the M x rank sweep (not the driver's line)")
-    ap.add_argument("--leg", choices=["w4a16", "mlp_pair"], default=None,
+    ap.add_argument("--leg", choices=["w4a16", "mlp_pair", "qkv_norm_rope"], default=None,
                     help="run one auxiliary leg alone and print its JSON line (not the driver's line; profiling)")
     return ap.parse_args()
 
@@ -919,7 +919,7 @@ def mlp_pair_leg(dev, stream, peaks, steps: int = 200):
 
 def run_leg(args):
     """One auxiliary leg on GPU 0, alone (used to profile its kernel): the W4A16 modulation
-    projections or FLUX's MLP pair, fused against unfused."""
+    projections, FLUX's MLP pair (fused against unfused) or the fused QKV operator."""
     import torch
 
     import w4a4_rank_corrected_smooth_b200 as S
@@ -931,8 +931,19 @@ def run_leg(args):
     peaks, peak_src = load_peaks()
     if args.leg == "w4a16":
         out = w4a16_leg(dev, stream, peaks, peak_src, launches=max(3, args.steps))
-    else:
+    elif args.leg == "mlp_pair":
         out = mlp_pair_leg(dev, stream, peaks, steps=max(3, args.steps))
+    else:  # the fused QKV operator on the FLUX QKV layer, against the plain forward
+        import synth
+
+        spec = synth.get(DEFAULT_WORKLOAD)
+        X = synth.activations_bf16(spec)
+        lin = S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(X), "nvfp4", spec.rank,
+                           device=0)
+        Xd = bf16_device(X, dev)
+        sets = [(Xd, torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=dev), lin.new_workspace(spec.M))]
+        out = qkv_norm_rope_leg([lin], sets, spec, stream, max(3, args.steps))
+        lin.close()
     print(json.dumps({"leg": args.leg, args.leg: out}), flush=True)
 
 

@@ -148,9 +148,11 @@ svdq_status svdq_workspace_size(const svdq_weights* w, int M, size_t* bytes);
  *     writes Y = bf16_rn(acc) once.
  * X:  device, M rows of K bf16, row stride ldx elements.   Y: device, M x N bf16, stride ldy.
  * workspace: device, >= svdq_workspace_size(w, M) bytes, 256-byte aligned; holds the codes,
- *   scales and T between the two kernels (every row up to M rounded up to a multiple of 256);
- *   kernel 1 writes all of it, so its contents need no initialisation.  One workspace must not be
- *   used by two forwards whose kernels overlap on the GPU.
+ *   scales and T between the two kernels (every row up to M rounded up to a multiple of 256)
+ *   and, for large layers when kernel 1 splits K, the fp32 partials of T and one arrival counter
+ *   per 128-row tile; contents are scratch and need no initialisation (kernel 1 writes every byte
+ *   kernel 2 reads; a counter tagged with another launch restarts, the last slice resets it).  One
+ *   workspace must not be used by two forwards whose kernels overlap on the GPU.
  * No allocation, no synchronisation.  Errors: INVALID_ARG, CUDA (launch failure). */
 svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
                                 void* workspace, size_t workspace_bytes, void* stream);
@@ -171,7 +173,7 @@ svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int
  * workspaces.  Nothing in the array has to start at zero.  Shapes whose workspace
  * (svdq_workspace_size) exceeds 20 MiB are rejected with SVDQ_ERR_INVALID_ARG: the row limit is
  * the largest M whose svdq_workspace_size fits in 20 MiB (at K = 3072 and rank 32 today every M
- * up to 11520; it moves with the workspace layout, so query svdq_workspace_size rather than
+ * up to 9984; it moves with the workspace layout, so query svdq_workspace_size rather than
  * relying on that figure).  A W4A16 layer uses no scratch and has no such limit.
  * Other arguments and errors as svdq_linear_forward. */
 svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,

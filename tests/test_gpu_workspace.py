@@ -1,9 +1,12 @@
-"""Kernel 1's workspace and determinism.
+"""Kernel 1's workspace and determinism, for both of its forms.
 
-Kernel 1 writes every byte of the activation codes, scales and T it leaves in the workspace (the
-padded rows included) and sums its warps' shares of T in a fixed order.  These tests check that
-the result needs no initialised workspace (filled with 0xFF first), that reusing a workspace gives
-bit-identical results, and that a CUDA-graph replay of the forward does too.
+Kernel 1 writes every byte of the activation codes, scales and T that kernel 2 reads.  Its
+warp-level form (16-row blocks, rank <= 32, up to two waves of blocks) sums its warps' shares of T
+in a fixed order; its 128-row-tile form splits K over CTAs, each writing an fp32 partial of T and
+counting itself in a per-tile counter tagged with the launch, and the last slice sums the partials
+in slice order.  These tests check that the result needs no initialised workspace (0xFF
+everywhere: garbage counters), that reusing a workspace gives bit-identical results, and that a
+CUDA-graph replay of the forward (the same launch tag every time) does too.
 """
 import numpy as np
 import pytest
@@ -25,8 +28,11 @@ def _bf16_dev(x_bits):
     return torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
+# rank 32: the warp-level form (32 blocks of 16 rows); rank 64: the 128-row tiles, K split in 8
+FORMS = [32, 64]
+
+
 def _layer(M=512, K=3072, N=512, r=32, seed=41):
-    # M = 512 rows, K = 3072: 32 row blocks of kernel 1, 48 chunks of 64 columns each
     spec = synth.custom("quant_down_ws", M=M, K=K, N=N, rank=r, seed=seed)
     X = synth.activations_bf16(spec)
     lin = S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(X), "nvfp4", r)
@@ -43,8 +49,9 @@ def _check_T(lin, X, act):
     assert_t_close(T_gpu, T_ref, O.bf16_to_f32(O.f32_to_bf16(xh)), O.bf16_to_f32(ops["L1"]))
 
 
-def test_quant_down_needs_no_initialised_workspace_and_repeats_bit_exactly():
-    spec, X, lin = _layer()
+@pytest.mark.parametrize("r", FORMS)
+def test_quant_down_needs_no_initialised_workspace_and_repeats_bit_exactly(r):
+    spec, X, lin = _layer(r=r)
     Xd = _bf16_dev(X)
     ws = lin.new_workspace(spec.M)
     ws.fill_(0xFF)  # garbage everywhere
@@ -61,8 +68,9 @@ def test_quant_down_needs_no_initialised_workspace_and_repeats_bit_exactly():
     lin.close()
 
 
-def test_graph_replay_of_the_forward_is_bit_identical_to_eager():
-    spec, X, lin = _layer(M=1000, seed=43)
+@pytest.mark.parametrize("r", FORMS)
+def test_graph_replay_of_the_forward_is_bit_identical_to_eager(r):
+    spec, X, lin = _layer(M=1000, r=r, seed=43)
     Xd = _bf16_dev(X)
     ws = lin.new_workspace(spec.M)
     Y_eager = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device="cuda")

@@ -2,12 +2,14 @@
 // Design" (b): Down Projection fused with Quantize because they read the same input; Up
 // Projection fused with 4-Bit Compute because they write the same output), for sm_100a.
 //
-// Kernel 1, quant_down: one CTA of eight warps per 16 rows of X, each warp streaming its share of
-// the rows' 64-column chunks straight into registers.  It applies the smoothing factor, quantizes
-// every K-group (NVFP4: UE4M3 scale per 16; INT4: fp32 scale per 64) into the tiled layouts
-// kernel 2 copies verbatim, and feeds bf16(x_hat) from the same registers to warp-level bf16 MMAs
-// that accumulate T = x_hat L1; the warps' shares of T are added through shared memory in a fixed
-// order and written once as bf16.
+// Kernel 1, quant_down, in two forms.  Both apply the smoothing factor, quantize every K-group
+// (NVFP4: UE4M3 scale per 16; INT4: fp32 scale per 64) with the same exact rounding into the tiled
+// layouts kernel 2 copies verbatim, and compute T = bf16(x_hat) L1 deterministically.
+// quant_down_kernel: one CTA of eight warps per 16 rows, each warp streaming its share of the rows'
+// 64-column chunks into registers and feeding bf16(x_hat) from them to warp-level bf16 MMAs; the
+// warps' shares of T are added through shared memory (layers of up to two waves of 16-row blocks,
+// rank <= 32).  quant_down_tile_kernel: one CTA per (128-row tile, K slice), X by TMA, T by
+// tcgen05 MMAs in tensor memory, K slices reduced by the last to arrive (larger layers and ranks).
 //
 // Kernel 2, gemm (NVFP4): persistent, warp specialised, on pairs of CTAs (cta_group::2 MMAs on
 // 256 x 256 tiles).  Two producer threads stream each k-block stage (operand tiles and scale
@@ -413,41 +415,443 @@ __global__ void __launch_bounds__(kQdThreads, 2) quant_down_kernel(const QdParam
   }
 }
 
-static int quant_down_ntm(int r) { return r == 0 ? 0 : (r <= 32 ? 4 : (r <= 64 ? 8 : 16)); }
 
-cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t stream) {
-  (void)num_sms;
-  QdParams p;
-  p.X = a.X;
-  p.ldx = a.ldx;
-  p.M = a.M;
-  p.K = a.K;
-  p.KB = a.K / kBK;
-  p.rank = a.rank;
-  p.inv_lambda = a.inv_lambda;
-  p.l1 = a.l1;
-  p.codes = a.codes;
-  p.sf = a.sf;
-  p.t = a.t;
-  // Every row of the workspace's padded tiles (kernel 2 consumes rows in pairs of 128-row tiles).
-  const int mpad = 2 * kBM * ((a.M + 2 * kBM - 1) / (2 * kBM));
-  const unsigned grid = static_cast<unsigned>(mpad / kQdRows);
-  const size_t shares = static_cast<size_t>(kQdWarps) * kQdRows * a.rank * sizeof(float);
-  const size_t smem = shares > kQdRingBytes ? shares : kQdRingBytes;
-  void (*kern)(const QdParams) = nullptr;
-  const int ntm = quant_down_ntm(a.rank);
-  if (a.precision == 0)
-    kern = ntm == 0 ? quant_down_kernel<0, 0> : ntm == 4 ? quant_down_kernel<0, 4> : ntm == 8 ? quant_down_kernel<0, 8>
-                                                                                          : quant_down_kernel<0, 16>;
-  else
-    kern = ntm == 0 ? quant_down_kernel<1, 0> : ntm == 4 ? quant_down_kernel<1, 4> : ntm == 8 ? quant_down_kernel<1, 8>
-                                                                                          : quant_down_kernel<1, 16>;
-  if (smem > 48 * 1024) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
+// ---------------------------------------------------------------------------- kernel 1, large layers
+//
+// The same three steps on 128-row tiles, for layers whose rows exceed one wave of the warp-level
+// kernel or whose rank exceeds 32 (there its 16-row blocks re-read L1 r/16 times the bytes of X
+// from L2).  One CTA per (128-row tile, K slice): a TMA warp streams X (and the stage's 1/lambda
+// and L1 chunk) into a ring of shared-memory stages; sixteen worker warps apply the smoothing
+// factor and quantize (NVFP4: one 16-element group per thread; INT4: 8 lanes share a 64-element
+// group) with the same exact bracketed rounding, and write bf16(x_hat) back into the stage; one
+// warp feeds it with L1 to tcgen05 bf16 MMAs that accumulate T in tensor memory.  When K is split
+// over several CTAs, each writes its fp32 partial of T and counts itself in the tile's counter;
+// the last to arrive adds the partials in slice order (deterministic) and writes bf16 T once.
+
+constexpr int kQtMaxStages = 8;
+constexpr int kQtWorkerWarps = 16;
+constexpr int kQtMmaWarp = kQtWorkerWarps;        // tcgen05 MMA issuer (+ TMEM owner)
+constexpr int kQtTmaWarp = kQtWorkerWarps + 1;    // TMA producer
+constexpr int kQtThreads = (kQtWorkerWarps + 2) * 32;
+constexpr uint32_t kQtXsBytes = kBM * 128;  // one stage of X: 128 rows x 64 bf16, 128-byte swizzle
+constexpr uint32_t kQtIlBytes = 64 * 4;     // the stage's 64 values of 1/lambda
+constexpr size_t kQtSmemBudget = 220 * 1024;
+
+struct QtParams {
+  int M, K, rank, KB, splits, stages;
+  const float* inv_lambda;
+  const uint8_t* l1;
+  uint8_t* codes;
+  uint8_t* sf;
+  uint8_t* t;
+  float* part;              // [m-tile][split][128][rank] fp32 partials of T (splits > 1)
+  unsigned long long* cnt;  // per m-tile: (launch epoch << 8) | slices arrived
+  unsigned long long epoch; // distinct per launch, never 0
+};
+
+// Counts this CTA's slice in the tile's counter and returns whether it was the last of `splits`.
+// The counter holds (epoch << 8) | count; a value from another launch (or uninitialised memory)
+// restarts the count, and the last CTA resets it to 0, so a replay of the same launch also starts
+// from 0.  Lock-free (a failed CAS means another slice succeeded); bounded all the same.
+__device__ __forceinline__ bool arrive_slice_counter(unsigned long long* cnt, unsigned long long epoch, int splits,
+                                                     bool* ok) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(cnt);
+  for (int it = 0; it < (1 << 20); ++it) {
+    const unsigned long long nxt = (cur >> 8) == epoch ? cur + 1 : ((epoch << 8) | 1ull);
+    const unsigned long long prev = atomicCAS(cnt, cur, nxt);
+    if (prev == cur) return static_cast<int>(nxt & 0xFFull) == splits;
+    cur = prev;
   }
-  kern<<<grid, kQdThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  atomicOr(&g_device_error, kErrWaitQuantDown);
+  *ok = false;
+  return false;
+}
+
+template <int PREC>
+__global__ void __launch_bounds__(kQtThreads, 1)
+    quant_down_tile_kernel(const __grid_constant__ CUtensorMap tmap_x, const QtParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ float rcp_tbl[128];  // RN(1 / UE4M3 value) for every finite scale code
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int r = p.rank;
+  const int NS = p.stages;
+  const bool has_lr = r > 0;
+  const uint32_t l1_bytes = static_cast<uint32_t>(r) * 128u;
+  const uint32_t l1_stride = static_cast<uint32_t>(align_up(l1_bytes, 1024));
+  uint8_t* xs = smem;                       // NS x 16 KB (X, then bf16 x_hat in place)
+  uint8_t* l1s = smem + NS * kQtXsBytes;      // NS x r*128 (L1 chunk)
+  const float* ils = reinterpret_cast<const float*>(l1s + NS * l1_stride);  // NS x 64 fp32 (1/lambda chunk)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(l1s + NS * l1_stride + NS * kQtIlBytes);
+  uint64_t* full = bars;                    // TMA landed: X tile (+ L1 chunk)
+  uint64_t* xready = bars + NS;             // workers wrote x_hat (one arrive per worker warp)
+  uint64_t* empty = bars + 2 * NS;          // stage free again
+  uint64_t* done = bars + 3 * NS;           // all MMAs of this CTA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = blockIdx.x / p.splits;
+  const int split = blockIdx.x % p.splits;
+  const int kb0 = split * p.KB / p.splits, kb1 = (split + 1) * p.KB / p.splits;
+  const int c0 = kb0 * 4, nch = (kb1 - kb0) * 4;
+  const uint32_t tmem_cols = r <= 32 ? 32u : (r <= 64 ? 64u : 128u);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&xready[s], kQtWorkerWarps);
+      mbar_init(&empty[s], has_lr ? 1 : kQtWorkerWarps);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (PREC == 0 && threadIdx.x < 128) rcp_tbl[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __frcp_rn(e4m3_to_f32(threadIdx.x));
+  if (has_lr && warp == kQtMmaWarp) {
+    tmem_alloc(tmem_slot, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = has_lr ? *tmem_slot : 0u;
+  // Kernel 2 may be scheduled once every block of this grid has got here (it waits for this
+  // grid's completion before reading anything this kernel writes).
+  pdl_launch_dependents();
+
+  if (warp < kQtWorkerWarps) {
+    // ------------------------------------------------------------ workers
+    // Quantization is exact (codes = E2M1_rne(RN(x / s)), resp. rint(RN(x / s)) for INT4): the
+    // quotient is bracketed between x * RN(RN(1/s)(1 -+ 2^-20)); both roundings are monotonic, so
+    // when the two bracketing codes agree they are the exact codes, and otherwise (x/s within
+    // ~2^-20 of a threshold) the IEEE division decides.
+    if (PREC == 0) {
+      // NVFP4: thread t of the 512 handles one 16-element group per 64-column chunk: row t / 4,
+      // group t % 4 (two swizzled 16-byte units; the quarter-warps' loads hit distinct banks).
+      const int row = warp * 8 + (lane >> 2), g = lane & 3;
+      const float kInv6 = __frcp_rn(6.0f);
+      // Per-thread constants: the two swizzled 16-byte units of the group inside a stage, and
+      // this row's code/scale positions inside a (tile, k-block) chunk.
+      const uint32_t off0 = swz128(row, g * 32), off1 = swz128(row, g * 32 + 16);
+      uint8_t* const codes_tile = p.codes + codes_chunk_offset(mt, 0, p.KB, kBM);
+      uint8_t* const sf_tile = p.sf + sf_chunk_offset(mt, 0, p.KB, kBM) + (row & 31) * 16 + (row >> 5) * 4 + g;
+      int st = 0;
+      uint32_t ph = 0;
+      for (int c = 0; c < nch; ++c) {
+        const bool ok = !*abort_flag && wait_parity_bounded(&full[st], ph, kErrWaitQuantDown);
+        if (!__all_sync(0xffffffffu, ok)) {
+          *abort_flag = 1;
+          break;
+        }
+        const int gc = c0 + c;
+        const int kb = gc >> 2, cc = gc & 3;
+        const float4* ilv = reinterpret_cast<const float4*>(ils + st * 64 + g * 16);
+        uint8_t* xt = xs + st * kQtXsBytes;
+        uint4* cell0 = reinterpret_cast<uint4*>(xt + off0);
+        uint4* cell1 = reinterpret_cast<uint4*>(xt + off1);
+        const uint4 xa = *cell0, xb = *cell1;
+        const uint32_t w[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+        uint64_t xp[2][4];  // x_hat as fp32 pairs: element 2t, 2t + 1 of half h in xp[h][t]
+        float pm[8];        // per-pair maxima of |x_hat|, reduced as a tree (max is exact)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float4 i0 = ilv[2 * h], i1 = ilv[2 * h + 1];
+          const float il[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            // bf16 -> fp32 is exact; x_hat = fp32(x) * (1/lambda), one rounding per element
+            const uint32_t ww = w[4 * h + t];
+            xp[h][t] = f2mul(f2pack(__uint_as_float(ww << 16), __uint_as_float(ww & 0xFFFF0000u)),
+                             f2pack(il[2 * t], il[2 * t + 1]));
+            float lo, hi;
+            f2unpack(xp[h][t], lo, hi);
+            pm[4 * h + t] = fmaxf(fabsf(lo), fabsf(hi));
+          }
+        }
+        const float amax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        // scale code: UE4M3_rne(RN(amax / 6)), bracketed the same way
+        const float s_est = __fmul_rn(amax, kInv6);
+        uint32_t sbits = cvt_e4m3(__fmul_rn(s_est, kNudgeLo));
+        const uint32_t sc_hi = cvt_e4m3(__fmul_rn(s_est, kNudgeHi));
+        uint2 code = make_uint2(0u, 0u);
+        bool slow = sbits != sc_hi;
+        if (!slow && sbits != 0) {
+          const float rr = rcp_tbl[sbits];
+          const float mlo = __fmul_rn(rr, kNudgeLo), mhi = __fmul_rn(rr, kNudgeHi);
+          code.x = e2m1x8_scaled(xp[0], mlo);
+          code.y = e2m1x8_scaled(xp[1], mlo);
+          slow = (code.x != e2m1x8_scaled(xp[0], mhi)) | (code.y != e2m1x8_scaled(xp[1], mhi));
+        }
+        if (slow) {  // rare: the exact quotients decide
+          float xh[2][8];
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int t = 0; t < 4; ++t) f2unpack(xp[h][t], xh[h][2 * t], xh[h][2 * t + 1]);
+          sbits = cvt_e4m3(__fdiv_rn(amax, 6.0f));
+          const float sd = e4m3_to_f32(sbits);
+          code.x = sd != 0.0f ? e2m1x8_div(xh[0], sd) : 0u;
+          code.y = sd != 0.0f ? e2m1x8_div(xh[1], sd) : 0u;
+        }
+        *reinterpret_cast<uint2*>(codes_tile + static_cast<size_t>(kb) * (kBM * kRowBytes) + swz128(row, cc * 32 + g * 8)) = code;
+        sf_tile[static_cast<size_t>(kb) * (kBM * kSfBytesPerRowKb) + cc * 512] = static_cast<uint8_t>(sbits);
+        if (has_lr) {
+          uint32_t hv[8];
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              float lo, hi;
+              f2unpack(xp[h][t], lo, hi);
+              hv[4 * h + t] = pack_bf16x2(lo, hi);
+            }
+          *cell0 = make_uint4(hv[0], hv[1], hv[2], hv[3]);  // bf16(x_hat) in place: the MMA's A operand
+          *cell1 = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(has_lr ? &xready[st] : &empty[st]);
+        if (++st == NS) {
+          st = 0;
+          ph ^= 1u;
+        }
+      }
+    } else {
+      // INT4: lane (sub, kg) of warp w handles 8 consecutive columns (16-byte unit kg) of rows
+      // 8w + sub and 8w + 4 + sub; the 64-element group spans the 8 lanes of a row.
+      const int sub = lane >> 3, kg = lane & 7;
+      for (int c = 0; c < nch; ++c) {
+        const int st = c % NS;
+        const bool ok = !*abort_flag && wait_parity_bounded(&full[st], (c / NS) & 1, kErrWaitQuantDown);
+        if (!__all_sync(0xffffffffu, ok)) {
+          *abort_flag = 1;
+          break;
+        }
+        const int gc = c0 + c;
+        const float4 il0 = *reinterpret_cast<const float4*>(ils + st * 64 + kg * 8);
+        const float4 il1 = *reinterpret_cast<const float4*>(ils + st * 64 + kg * 8 + 4);
+        const float il[8] = {il0.x, il0.y, il0.z, il0.w, il1.x, il1.y, il1.z, il1.w};
+        const int kb = gc >> 2, cc = gc & 3;
+        uint8_t* codes_chunk = p.codes + codes_chunk_offset(mt, kb, p.KB, kBM);
+        uint8_t* sf_chunk = p.sf + sf_chunk_offset(mt, kb, p.KB, kBM);
+        uint8_t* xt = xs + st * kQtXsBytes;
+        int row[2];
+        uint4* cell[2];
+        float xh[2][8];
+        float amax[2];
+        uint64_t ilp[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) ilp[t] = f2pack(il[2 * t], il[2 * t + 1]);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          row[i] = warp * 8 + i * 4 + sub;
+          cell[i] = reinterpret_cast<uint4*>(xt + swz128(row[i], kg * 16));
+          const uint4 xv = *cell[i];
+          const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const uint64_t xp = f2mul(f2pack(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xFFFF0000u)), ilp[t]);
+            f2unpack(xp, xh[i][2 * t], xh[i][2 * t + 1]);
+          }
+          amax[i] = fmaxf(fmaxf(fmaxf(fabsf(xh[i][0]), fabsf(xh[i][1])), fmaxf(fabsf(xh[i][2]), fabsf(xh[i][3]))),
+                          fmaxf(fmaxf(fabsf(xh[i][4]), fabsf(xh[i][5])), fmaxf(fabsf(xh[i][6]), fabsf(xh[i][7]))));
+          amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 1));
+          amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 2));
+          amax[i] = fmaxf(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], 4));
+        }
+        uint32_t codes[2], sbits[2];
+        bool slow = false;
+        float sc[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          sc[i] = __fdiv_rn(amax[i], 7.0f);
+          sbits[i] = __float_as_uint(sc[i]);
+          codes[i] = 0;
+          if (sc[i] != 0.0f) {
+            const float rr = __frcp_rn(sc[i]);
+            if (rr < 1e30f) {
+              const uint32_t lo = int4x8(xh[i], __fmul_rn(rr, kNudgeLo));
+              const uint32_t hi = int4x8(xh[i], __fmul_rn(rr, kNudgeHi));
+              codes[i] = lo;
+              slow |= lo != hi;
+            } else {
+              slow = true;  // tiny scale: reciprocal out of range
+            }
+          }
+        }
+        if (slow) {
+#pragma unroll
+          for (int i = 0; i < 2; ++i) codes[i] = sc[i] != 0.0f ? int4x8_div(xh[i], sc[i]) : 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          *reinterpret_cast<uint32_t*>(codes_chunk + swz128(row[i], cc * 32 + kg * 4)) = codes[i];
+          if (kg == 0) reinterpret_cast<uint32_t*>(sf_chunk)[sf_int4_a_index(row[i], cc)] = sbits[i];
+          if (has_lr) {
+            uint4 hv;
+            hv.x = pack_bf16x2(xh[i][0], xh[i][1]);
+            hv.y = pack_bf16x2(xh[i][2], xh[i][3]);
+            hv.z = pack_bf16x2(xh[i][4], xh[i][5]);
+            hv.w = pack_bf16x2(xh[i][6], xh[i][7]);
+            *cell[i] = hv;  // bf16(x_hat) in place: the tile becomes the MMA's A operand
+          }
+        }
+        if (has_lr) fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(has_lr ? &xready[st] : &empty[st]);
+      }
+    }
+  } else if (warp == kQtTmaWarp) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      int issued = 0;
+      for (int c = 0; c < nch; ++c) {
+        const int st = c % NS;
+        if (c >= NS && (*abort_flag || !wait_parity_bounded(&empty[st], ((c / NS) - 1) & 1, kErrWaitQuantDown))) {
+          *abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[st], kQtXsBytes + kQtIlBytes + (has_lr ? l1_bytes : 0u));
+        tma_load_2d(xs + st * kQtXsBytes, &tmap_x, (c0 + c) * 64, mt * kBM, &full[st]);
+        bulk_g2s(const_cast<float*>(ils) + st * 64, p.inv_lambda + static_cast<size_t>(c0 + c) * 64, kQtIlBytes, &full[st]);
+        if (has_lr)
+          bulk_g2s(l1s + st * l1_stride, p.l1 + static_cast<size_t>(c0 + c) * l1_bytes, l1_bytes, &full[st]);
+        ++issued;
+      }
+      if (*abort_flag) {
+        // Let every issued copy land before the CTA can retire.
+        for (int q = (issued > NS ? issued - NS : 0); q < issued; ++q)
+          wait_parity_bounded(&full[q % NS], (q / NS) & 1, kErrWaitQuantDown);
+      }
+    }
+  } else if (has_lr && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = idesc_bf16(128, r);
+    for (int c = 0; c < nch; ++c) {
+      const int st = c % NS;
+      const uint32_t par = (c / NS) & 1;
+      if (*abort_flag || !wait_parity_bounded(&full[st], par, kErrWaitQuantDown) ||
+          !wait_parity_bounded(&xready[st], par, kErrWaitQuantDown)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint64_t ad = smem_desc(smem_u32(xs + st * kQtXsBytes), 16, 1024, kLayoutSw128);
+      const uint64_t bd = smem_desc(smem_u32(l1s + st * l1_stride), 16, 1024, kLayoutSw128);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem_base, ad + 2 * ks, bd + 2 * ks, idesc, (c | ks) != 0 ? 1u : 0u);
+      tc_commit(&empty[st]);
+    }
+    tc_commit(done);
+  }
+
+  // ---------------------------------------------------------------- T epilogue
+  __syncthreads();
+  const bool aborted = *abort_flag != 0;
+  if (has_lr && warp < 4) {
+    bool ok = !aborted && wait_parity_bounded(done, 0, kErrWaitQuantDown);
+    ok = __all_sync(0xffffffffu, ok);  // the TMEM loads below are warp-collective
+    tc_fence_after();
+    if (ok) {
+      const int row = warp * 32 + lane;
+      float* prow = p.splits > 1 ? p.part + ((static_cast<size_t>(mt) * p.splits + split) * kBM + row) * r : nullptr;
+      for (int j = 0; j < r; j += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + j, v);
+        tmem_wait_ld();
+        if (p.splits == 1) {
+          uint8_t* tt = p.t + static_cast<size_t>(mt) * kBM * r * 2;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(v[8 * h + 0]), __uint_as_float(v[8 * h + 1]));
+            o.y = pack_bf16x2(__uint_as_float(v[8 * h + 2]), __uint_as_float(v[8 * h + 3]));
+            o.z = pack_bf16x2(__uint_as_float(v[8 * h + 4]), __uint_as_float(v[8 * h + 5]));
+            o.w = pack_bf16x2(__uint_as_float(v[8 * h + 6]), __uint_as_float(v[8 * h + 7]));
+            *reinterpret_cast<uint4*>(tt + lr_offset(row, j + 8 * h, kBM, r)) = o;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 16; q += 4)
+            *reinterpret_cast<float4*>(prow + j + q) = make_float4(__uint_as_float(v[q]), __uint_as_float(v[q + 1]),
+                                                                   __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]));
+        }
+      }
+    }
+  }
+  if (has_lr && p.splits > 1) {
+    // The last slice of the tile to finish sums all slices' partials in slice order
+    // (deterministic) and writes bf16 T.  Publication: the CTA barrier orders every thread's
+    // partial stores before thread 0's GPU-scope fence, which is cumulative, and that fence
+    // before the counter update; the last slice fences again before reading.
+    __shared__ int s_last;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      bool ok = !aborted;
+      __threadfence();
+      const bool last = ok && arrive_slice_counter(p.cnt + mt, p.epoch, p.splits, &ok);
+      if (last) __threadfence();
+      if (!ok) {
+        // A slice that gave up resets the tile's count, so that a replay of this launch (a CUDA
+        // graph keeps its launch tag) does not resume a count this launch left incomplete.
+        *abort_flag = 1;
+        atomicExch(p.cnt + mt, 0ull);
+      }
+      s_last = last ? 1 : 0;
+    }
+    __syncthreads();
+    if (s_last) {
+      uint8_t* tt = p.t + static_cast<size_t>(mt) * kBM * r * 2;
+      const float* pt = p.part + static_cast<size_t>(mt) * p.splits * kBM * r;
+      const size_t slice = static_cast<size_t>(kBM) * r;
+      const int units = kBM * r / 4;
+      // Two 4-column units per thread per round, all of a round's loads issued before the sums.
+      for (int u0 = threadIdx.x; u0 < units; u0 += 2 * blockDim.x) {
+        const int u1 = u0 + blockDim.x;
+        const bool has1 = u1 < units;
+        const int o0 = u0 * 4, o1 = (has1 ? u1 : u0) * 4;
+        float4 a0 = __ldcg(reinterpret_cast<const float4*>(pt + o0));
+        float4 a1 = __ldcg(reinterpret_cast<const float4*>(pt + o1));
+        float4 x0[7], x1[7];
+#pragma unroll
+        for (int q = 1; q < 8; ++q)
+          if (q < p.splits) {
+            x0[q - 1] = __ldcg(reinterpret_cast<const float4*>(pt + q * slice + o0));
+            x1[q - 1] = __ldcg(reinterpret_cast<const float4*>(pt + q * slice + o1));
+          }
+#pragma unroll
+        for (int q = 1; q < 8; ++q)
+          if (q < p.splits) {
+            a0.x += x0[q - 1].x; a0.y += x0[q - 1].y; a0.z += x0[q - 1].z; a0.w += x0[q - 1].w;
+            a1.x += x1[q - 1].x; a1.y += x1[q - 1].y; a1.z += x1[q - 1].z; a1.w += x1[q - 1].w;
+          }
+        *reinterpret_cast<uint2*>(tt + lr_offset(o0 / r, o0 % r, kBM, r)) =
+            make_uint2(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w));
+        if (has1)
+          *reinterpret_cast<uint2*>(tt + lr_offset(o1 / r, o1 % r, kBM, r)) =
+              make_uint2(pack_bf16x2(a1.x, a1.y), pack_bf16x2(a1.z, a1.w));
+      }
+      if (threadIdx.x == 0) atomicExch(p.cnt + mt, 0ull);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (has_lr && warp == kQtMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+static int quant_down_tile_stages(int r) {
+  const size_t per = kQtXsBytes + align_up(static_cast<size_t>(r) * 128, 1024) + kQtIlBytes;
+  const int ns = static_cast<int>((kQtSmemBudget - 2048) / per);
+  return ns < kQtMaxStages ? ns : kQtMaxStages;
+}
+
+static size_t quant_down_tile_smem_bytes(int r) {
+  const int ns = quant_down_tile_stages(r);
+  return 1024 + ns * (kQtXsBytes + align_up(static_cast<size_t>(r) * 128, 1024) + kQtIlBytes) + 256;
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link dependency).
@@ -465,6 +869,92 @@ static EncodeTiledFn encode_tiled_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   }
   return fn;
+}
+
+static cudaError_t launch_quant_down_tile(const QuantDownArgs& a, int num_sms, cudaStream_t stream) {
+  QtParams p;
+  p.M = a.M;
+  p.K = a.K;
+  p.rank = a.rank;
+  p.KB = a.K / kBK;
+  p.stages = quant_down_tile_stages(a.rank);
+  p.inv_lambda = a.inv_lambda;
+  p.l1 = a.l1;
+  p.codes = a.codes;
+  p.sf = a.sf;
+  p.t = a.t;
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tmap;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.ldx) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBM)};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.X), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const int mt = 2 * ((a.M + 2 * kBM - 1) / (2 * kBM));  // pairs of 128-row tiles (kernel 2 works on 256 rows)
+  const size_t smem = quant_down_tile_smem_bytes(a.rank);
+  void (*kern)(const CUtensorMap, const QtParams) = a.precision == 0 ? quant_down_tile_kernel<0> : quant_down_tile_kernel<1>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  // One CTA per SM (shared memory), one wave: as many K slices per tile as the SMs allow, within
+  // what the workspace's partials have room for.
+  int splits = num_sms / mt;
+  if (splits > a.split_cap) splits = a.split_cap;
+  if (splits < 1) splits = 1;
+  if (a.rank > 0 && splits > 1 && (!a.part || !a.cnt)) splits = 1;
+  p.splits = splits;
+  p.part = a.part;
+  p.cnt = a.cnt;
+  static std::atomic<unsigned long long> epoch_counter{0};
+  p.epoch = (epoch_counter.fetch_add(1) + 1) & ((1ull << 56) - 1);
+  if (p.epoch == 0) p.epoch = 1;
+  if (a.precision == 0)
+    quant_down_tile_kernel<0><<<mt * splits, kQtThreads, smem, stream>>>(tmap, p);
+  else
+    quant_down_tile_kernel<1><<<mt * splits, kQtThreads, smem, stream>>>(tmap, p);
+  return cudaGetLastError();
+}
+
+
+static cudaError_t launch_quant_down_warps(const QuantDownArgs& a, cudaStream_t stream) {
+  QdParams p;
+  p.X = a.X;
+  p.ldx = a.ldx;
+  p.M = a.M;
+  p.K = a.K;
+  p.KB = a.K / kBK;
+  p.rank = a.rank;
+  p.inv_lambda = a.inv_lambda;
+  p.l1 = a.l1;
+  p.codes = a.codes;
+  p.sf = a.sf;
+  p.t = a.t;
+  // Every row of the workspace's padded tiles (kernel 2 consumes rows in pairs of 128-row tiles).
+  const int mpad = 2 * kBM * ((a.M + 2 * kBM - 1) / (2 * kBM));
+  const unsigned grid = static_cast<unsigned>(mpad / kQdRows);
+  const size_t shares = static_cast<size_t>(kQdWarps) * kQdRows * a.rank * sizeof(float);
+  const size_t smem = shares > kQdRingBytes ? shares : kQdRingBytes;
+  // rank 0 or at most 32 (the caller dispatches larger ranks to the 128-row tiles)
+  void (*kern)(const QdParams) = a.precision == 0 ? (a.rank == 0 ? quant_down_kernel<0, 0> : quant_down_kernel<0, 4>)
+                                                  : (a.rank == 0 ? quant_down_kernel<1, 0> : quant_down_kernel<1, 4>);
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<grid, kQdThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+// The warp-level kernel when its 16-row blocks fit in one wave (two per SM) and the rank is at most
+// 32 (the FLUX QKV and MLP-up layers: X streamed with the most parallelism); the 128-row tiles
+// otherwise, and whenever the caller's workspace has room for their K-split partials only.
+cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t stream) {
+  const int mpad = 2 * kBM * ((a.M + 2 * kBM - 1) / (2 * kBM));
+  if (a.rank <= 32 && mpad / kQdRows <= 2 * num_sms) return launch_quant_down_warps(a, stream);
+  return launch_quant_down_tile(a, num_sms, stream);
 }
 
 
@@ -702,6 +1192,53 @@ __device__ __forceinline__ float gelu_bf16(float y) {
   return __float_as_uint(lo) == __float_as_uint(hi) ? lo : gelu_bf16_slow(y);
 }
 
+// The fused MLP epilogue evaluates GELU for every hidden value, so its common range goes through a
+// table in shared memory: the exact bf16 GELU of every bf16 input with |y| in [2^-4, 8) (both
+// signs, 7 binades of 128 values), filled by gelu_bf16 itself at kernel start.  Below 2^-4 a short
+// series does it (bracketed like gelu_bf16), from 8 up GELU(y) rounds to y, and below -8 the full
+// evaluation runs.
+constexpr int kGeluTblE0 = 123;     // bf16 exponent field of 2^-4
+constexpr int kGeluTblBinades = 7;  // 2^-4 .. 2^3
+constexpr int kGeluTblSize = 2 * kGeluTblBinades * 128;
+
+__device__ __noinline__ void fill_gelu_table(uint16_t* tbl, int tid, int nthreads) {
+  for (int i = tid; i < kGeluTblSize; i += nthreads) {
+    const uint32_t sign = static_cast<uint32_t>(i / (kGeluTblBinades * 128));
+    const uint32_t rest = static_cast<uint32_t>(i % (kGeluTblBinades * 128));
+    const uint32_t b = (sign << 15) | ((kGeluTblE0 + rest / 128) << 7) | (rest % 128);
+    tbl[i] = static_cast<uint16_t>(__float_as_uint(gelu_bf16(__uint_as_float(b << 16))) >> 16);
+  }
+}
+
+// 2^-125 <= |y| < 2^-4: GELU(y) = y (1/2 + c1 (y - y^3/6 + y^5/40 - y^7/336) + O(y^9)) with
+// c1 = 1/sqrt(2 pi); the truncation is below 1e-14 relative, the fp32 Horner steps a few ulp, so
+// the result is bracketed by 2^-20 relative and the rare straddling case falls back to double.
+__device__ __forceinline__ float gelu_bf16_series(float y) {
+  const float c1 = 0.3989422804014327f, c3 = -0.06649038006690545f, c5 = 0.009973557010035818f,
+              c7 = -0.0011873282154803355f;
+  const float y2 = __fmul_rn(y, y);
+  const float p = __fmaf_rn(y2, __fmaf_rn(y2, __fmaf_rn(y2, c7, c5), c3), c1);
+  const float g = __fmul_rn(y, __fmaf_rn(y, p, 0.5f));
+  const float d = __fmaf_rn(fabsf(g), 0x1p-20f, 0x1p-140f);
+  const float lo = __bfloat162float(__float2bfloat16_rn(__fsub_rn(g, d)));
+  const float hi = __bfloat162float(__float2bfloat16_rn(__fadd_rn(g, d)));
+  return __float_as_uint(lo) == __float_as_uint(hi) ? lo : gelu_bf16_slow(y);
+}
+
+// The correctly rounded bf16 GELU of a bf16 y (as fp32), with the table `tbl` in shared memory.
+__device__ __forceinline__ float gelu_bf16_tab(float y, const uint16_t* tbl) {
+  const uint32_t b = __float_as_uint(y) >> 16;
+  const uint32_t e = ((b >> 7) & 0xFFu) - static_cast<uint32_t>(kGeluTblE0);
+  if (e < static_cast<uint32_t>(kGeluTblBinades))
+    return __uint_as_float(static_cast<uint32_t>(tbl[((b >> 15) * kGeluTblBinades + e) * 128u + (b & 127u)]) << 16);
+  if (y >= 8.0f) return y;  // y Phi(y) = y (1 - Q(y)) with Q(y) < 1e-15: rounds to y
+  if ((__float_as_uint(y) & 0x7FFFFFFFu) < 0x3D800000u) {  // |y| < 2^-4
+    if ((__float_as_uint(y) & 0x7FFFFFFFu) < 0x01000000u) return gelu_bf16_tiny(__float_as_uint(y));
+    return gelu_bf16_series(y);
+  }
+  return gelu_bf16(y);
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
@@ -730,6 +1267,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
   uint64_t* stg_free = lr_full + 1;         // (both) the epilogue's stores finished reading staging
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stg_free + 1);
   float* gamma_sm = reinterpret_cast<float*>(staging + kGStaging + 256);  // fused Q/K: gamma_q, gamma_k
+  uint16_t* gelu_tbl = reinterpret_cast<uint16_t*>(staging + kGStaging + 256);  // fused MLP: GELU table
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -770,6 +1308,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
     tmem_alloc2(tmem_slot, kTmemCols);
     tmem_relinquish2();
   }
+  if constexpr (kEpi == 2) fill_gelu_table(gelu_tbl, threadIdx.x, kGThreads);  // (before kernel 1 ends)
   tc_fence_before();
   cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
   tc_fence_after();
@@ -894,8 +1433,9 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
             float pm[8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
-              const float lo = live ? __fmul_rn(gelu_bf16(__uint_as_float(wy[t] << 16)), il[2 * t]) : 0.0f;
-              const float hi = live ? __fmul_rn(gelu_bf16(__uint_as_float(wy[t] & 0xFFFF0000u)), il[2 * t + 1]) : 0.0f;
+              const float lo = live ? __fmul_rn(gelu_bf16_tab(__uint_as_float(wy[t] << 16), gelu_tbl), il[2 * t]) : 0.0f;
+              const float hi =
+                  live ? __fmul_rn(gelu_bf16_tab(__uint_as_float(wy[t] & 0xFFFF0000u), gelu_tbl), il[2 * t + 1]) : 0.0f;
               xp[t >> 2][t & 3] = f2pack(lo, hi);
               pm[t] = fmaxf(fabsf(lo), fabsf(hi));
             }
@@ -1818,7 +2358,10 @@ static cudaError_t launch_gemm_int4(const GemmArgs& a, int num_sms, cudaStream_t
   return cudaGetLastError();
 }
 
-static size_t gemm_smem_bytes() { return 1024 + kGStages * kGStage + kGStaging + 256 + 2 * kQkvHeadDim * 4; }
+static size_t gemm_smem_bytes() {
+  constexpr size_t extra = 2 * kQkvHeadDim * 4 > kGeluTblSize * 2 ? 2 * kQkvHeadDim * 4 : kGeluTblSize * 2;
+  return 1024 + kGStages * kGStage + kGStaging + 256 + extra;
+}
 
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   if (a.precision != 0) return launch_gemm_int4(a, num_sms, stream);
@@ -2028,9 +2571,12 @@ cudaError_t launch_rope_pack(const float* rope, int M, float* packed, cudaStream
 
 // The fused MLP epilogue's bf16 GELU on a list of bf16 inputs (a test hook).
 __global__ void selftest_gelu_kernel(const uint16_t* in, uint16_t* out, int n) {
+  __shared__ uint16_t tbl[kGeluTblSize];
+  fill_gelu_table(tbl, threadIdx.x, blockDim.x);
+  __syncthreads();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) {
-    const float g = gelu_bf16(__uint_as_float(static_cast<uint32_t>(in[i]) << 16));
+    const float g = gelu_bf16_tab(__uint_as_float(static_cast<uint32_t>(in[i]) << 16), tbl);
     out[i] = static_cast<uint16_t>(__float_as_uint(g) >> 16);
   }
 }

@@ -16,6 +16,10 @@ struct QuantDownArgs {
   uint8_t* codes;          // workspace: tiled activation codes
   uint8_t* sf;             // workspace: tiled activation scales
   uint8_t* t;              // workspace: tiled bf16 T
+  // 128-row-tile kernel only (when it splits K and rank > 0):
+  float* part;             // workspace: fp32 partials of T per K slice
+  unsigned long long* cnt; // workspace: one arrival counter per 128-row tile
+  int split_cap;           // largest K split the partials have room for
 };
 
 struct GemmArgs {

@@ -73,15 +73,26 @@ SVDQ_HD constexpr size_t l1_offset(uint32_t k, uint32_t i, int r) {
   return static_cast<size_t>(k / 64u) * static_cast<size_t>(r) * 128u + swz128(i, (k % 64u) * 2u);
 }
 
+// Kernel 1's 128-row-tile form splits K into at most this many slices per tile: at most 8, at most
+// one per k-block, and at most 160 CTAs in all (one wave on a GPU of up to 160 SMs).
+SVDQ_HD constexpr int quant_down_split_cap(int m_tiles, int KB) {
+  const int by_grid = m_tiles > 0 ? 160 / m_tiles : 1;
+  const int cap = by_grid < 8 ? by_grid : 8;
+  return cap < 1 ? 1 : (cap < KB ? cap : KB);
+}
+
 struct WorkspaceLayout {
-  size_t codes = 0, sf = 0, t = 0, total = 0;
-  int m_tiles = 0;
+  size_t codes = 0, sf = 0, t = 0, part = 0, cnt = 0, total = 0;
+  int m_tiles = 0, split_cap = 1;
 };
 
-// Workspace: activation codes, scales and T (bf16) of every row of the padded tiles.
+// Workspace: activation codes, scales and T (bf16) of every row of the padded tiles and, for the
+// 128-row-tile form of kernel 1 when it splits K (rank > 0), the fp32 partials of T of every slice
+// plus one arrival counter per 128-row tile.
 inline WorkspaceLayout workspace_layout(int M, int K, int r) {
   WorkspaceLayout w;
   w.m_tiles = 2 * ((M + 2 * kBM - 1) / (2 * kBM));  // kernel 2 consumes rows in pairs of 128-row tiles
+  w.split_cap = quant_down_split_cap(w.m_tiles, K / kBK);
   const size_t mpad = static_cast<size_t>(w.m_tiles) * kBM;
   w.codes = 0;
   size_t end = mpad * static_cast<size_t>(K) / 2;
@@ -89,6 +100,12 @@ inline WorkspaceLayout workspace_layout(int M, int K, int r) {
   end = w.sf + mpad * static_cast<size_t>(K) / kBK * kSfBytesPerRowKb;
   w.t = align_up(end, 1024);
   end = w.t + mpad * static_cast<size_t>(r) * 2;
+  if (r > 0 && w.split_cap > 1) {
+    w.part = align_up(end, 1024);
+    end = w.part + mpad * static_cast<size_t>(w.split_cap) * static_cast<size_t>(r) * 4;
+    w.cnt = align_up(end, 256);
+    end = w.cnt + static_cast<size_t>(w.m_tiles) * 8;
+  }
   w.total = M > 0 ? align_up(end, 1024) : 0;
   return w;
 }

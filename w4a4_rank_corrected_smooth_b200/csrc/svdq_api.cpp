@@ -137,6 +137,9 @@ svdq_status do_quant_down(const svdq_weights* w, const void* X, int M, int ldx, 
   a.codes = base + L.codes;
   a.sf = base + L.sf;
   a.t = base + L.t;
+  a.part = L.part ? reinterpret_cast<float*>(base + L.part) : nullptr;
+  a.cnt = L.cnt ? reinterpret_cast<unsigned long long*>(base + L.cnt) : nullptr;
+  a.split_cap = L.split_cap;  // with rank 0 no partials are needed
   cudaError_t e = svdq::launch_quant_down(a, w->num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launch of the quantize/down-projection kernel");
   return SVDQ_OK;

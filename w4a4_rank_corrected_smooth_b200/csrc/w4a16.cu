@@ -137,74 +137,65 @@ __global__ void __launch_bounds__(kWThreads) w4a16_kernel(const W4A16Params p) {
         stage(gc, ng);
         __syncthreads();
       }
-      // The warp's groups gl = warp, warp + 8, ...: codes and scales of the next kWAhead groups are
-      // in flight while one group's math runs (a window of registers shifted by one group a step).
-      int gl = warp;
+      // The warp's groups gl = warp, warp + 8, ...: the codes and scales of its next kWAhead groups
+      // are in flight while one group's math runs.  Slot q holds the groups gb + q * 8 of the block
+      // gb; a slot is refilled with the group kWAhead steps later as soon as its math is done.
       uint4 c[kWAhead][R];
       float2 s[kWAhead][R];
-#pragma unroll
-      for (int q = 0; q < kWAhead; ++q) {
-        const int gq = gl + q * kWWarps;
+      auto fetch = [&](int q, int g) {
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           c[q][r] = make_uint4(0u, 0u, 0u, 0u);
           s[q][r] = make_float2(0.0f, 0.0f);
-          if (gq < ng) {
-            const size_t cb = static_cast<size_t>(b0 + r) * p.G + gc + gq;
+          if (g < ng) {
+            const size_t cb = static_cast<size_t>(b0 + r) * p.G + gc + g;
             c[q][r] = __ldg(p.codes + cb * 32 + lane);
             s[q][r] = __ldg(p.scales + cb * 8 + gid);
           }
         }
-      }
-      for (; gl < ng; gl += kWWarps) {
-        uint4 bq[MB][2];
+      };
 #pragma unroll
-        for (int mb = 0; mb < MB; ++mb)
+      for (int q = 0; q < kWAhead; ++q) fetch(q, warp + q * kWWarps);
+      for (int gb = warp; gb < ng; gb += kWAhead * kWWarps) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) bq[mb][h] = xs[((mb * ng + gl) * 2 + h) * 32 + lane];
+        for (int q = 0; q < kWAhead; ++q) {
+          const int gl = gb + q * kWWarps;
+          if (gl < ng) {
+            uint4 bq[MB][2];
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const uint32_t w[4] = {c[0][r].x, c[0][r].y, c[0][r].z, c[0][r].w};
-          float d[MB][4];
+            for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
-          for (int mb = 0; mb < MB; ++mb)
+              for (int h = 0; h < 2; ++h) bq[mb][h] = xs[((mb * ng + gl) * 2 + h) * 32 + lane];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) d[mb][j] = 0.0f;
+            for (int r = 0; r < R; ++r) {
+              const uint32_t w[4] = {c[q][r].x, c[q][r].y, c[q][r].z, c[q][r].w};
+              float d[MB][4];
 #pragma unroll
-          for (int st = 0; st < 4; ++st) {
-            uint32_t a[4];
+              for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) a[j] = codes_to_bf16x2(w[st] >> (4 * j));
+                for (int j = 0; j < 4; ++j) d[mb][j] = 0.0f;
 #pragma unroll
-            for (int mb = 0; mb < MB; ++mb) {
-              const uint4& hb = bq[mb][st >> 1];
-              const uint32_t bb0 = (st & 1) ? hb.z : hb.x;
-              const uint32_t bb1 = (st & 1) ? hb.w : hb.y;
-              mma_bf16_16816(d[mb], a, bb0, bb1);
+              for (int st = 0; st < 4; ++st) {
+                uint32_t a[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) a[j] = codes_to_bf16x2(w[st] >> (4 * j));
+#pragma unroll
+                for (int mb = 0; mb < MB; ++mb) {
+                  const uint4& hb = bq[mb][st >> 1];
+                  const uint32_t bb0 = (st & 1) ? hb.z : hb.x;
+                  const uint32_t bb1 = (st & 1) ? hb.w : hb.y;
+                  mma_bf16_16816(d[mb], a, bb0, bb1);
+                }
+              }
+#pragma unroll
+              for (int mb = 0; mb < MB; ++mb) {
+                acc[r][mb][0] = fmaf(s[q][r].x, d[mb][0], acc[r][mb][0]);
+                acc[r][mb][1] = fmaf(s[q][r].x, d[mb][1], acc[r][mb][1]);
+                acc[r][mb][2] = fmaf(s[q][r].y, d[mb][2], acc[r][mb][2]);
+                acc[r][mb][3] = fmaf(s[q][r].y, d[mb][3], acc[r][mb][3]);
+              }
             }
-          }
-#pragma unroll
-          for (int mb = 0; mb < MB; ++mb) {
-            acc[r][mb][0] = fmaf(s[0][r].x, d[mb][0], acc[r][mb][0]);
-            acc[r][mb][1] = fmaf(s[0][r].x, d[mb][1], acc[r][mb][1]);
-            acc[r][mb][2] = fmaf(s[0][r].y, d[mb][2], acc[r][mb][2]);
-            acc[r][mb][3] = fmaf(s[0][r].y, d[mb][3], acc[r][mb][3]);
-          }
-        }
-        const int gn = gl + kWAhead * kWWarps;
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-#pragma unroll
-          for (int q = 0; q + 1 < kWAhead; ++q) {
-            c[q][r] = c[q + 1][r];
-            s[q][r] = s[q + 1][r];
-          }
-          c[kWAhead - 1][r] = make_uint4(0u, 0u, 0u, 0u);
-          s[kWAhead - 1][r] = make_float2(0.0f, 0.0f);
-          if (gn < ng) {
-            const size_t cb = static_cast<size_t>(b0 + r) * p.G + gc + gn;
-            c[kWAhead - 1][r] = __ldg(p.codes + cb * 32 + lane);
-            s[kWAhead - 1][r] = __ldg(p.scales + cb * 8 + gid);
+            fetch(q, gl + kWAhead * kWWarps);
           }
         }
       }
