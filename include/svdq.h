@@ -171,10 +171,11 @@ svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int
  * whose kernels overlap on the GPU (different streams, no ordering between them) race and give
  * wrong results, so order them on one stream or use svdq_linear_forward with separate
  * workspaces.  Nothing in the array has to start at zero.  Shapes whose workspace
- * (svdq_workspace_size) exceeds 20 MiB are rejected with SVDQ_ERR_INVALID_ARG: the row limit is
- * the largest M whose svdq_workspace_size fits in 20 MiB (at K = 3072 and rank 32 today every M
- * up to 9984; it moves with the workspace layout, so query svdq_workspace_size rather than
- * relying on that figure).  A W4A16 layer uses no scratch and has no such limit.
+ * (svdq_workspace_size) exceeds 20 MiB are rejected with SVDQ_ERR_INVALID_ARG: a shape is
+ * accepted exactly when its svdq_workspace_size fits in 20 MiB (at K = 3072 and rank 32 today every
+ * M up to 9984 does; the size is not monotonic in M, since kernel 1's K-split partials vanish once
+ * a 128-row tile gets a single slice; it moves with the workspace layout, so query
+ * svdq_workspace_size rather than relying on that figure).  A W4A16 layer uses no scratch and has no such limit.
  * Other arguments and errors as svdq_linear_forward. */
 svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
                                         void* stream);

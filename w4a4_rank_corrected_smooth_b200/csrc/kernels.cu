@@ -1349,14 +1349,31 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
     if (lr_issuer && t_first < t_end) issue_lr(t_first);
     int local = 0;
     for (int tile = t_first; tile < t_end; tile += t_step, ++local) {
+      const int m2 = tile / p.NT, nt = tile % p.NT;
+      const int row0 = (2 * m2 + static_cast<int>(rank)) * kBM + q * 32;
+      const int n0 = nt * kBN + h * 128;
+      // Fused Q/K: this row's rotary table goes in flight before the wait for the accumulator.  The
+      // packed table (rope_packed_index) puts the 32 rows of a warp side by side, so each load reads
+      // 512 contiguous bytes; the loads run kRopeAhead units ahead of their use.  Rows past M (never
+      // stored) read the last row's angles.
+      const float* rp = nullptr;
+      float4 rq[kRopeAhead][2];
+      if constexpr (kEpi == 1) {
+        if (n0 < p.qk_cols) {
+          const int m = row0 + lane < p.M ? row0 + lane : p.M - 1;
+          rp = p.rope + rope_packed_index(m, 0, 0);
+#pragma unroll
+          for (int k = 0; k < kRopeAhead; ++k) {
+            rq[k][0] = __ldg(reinterpret_cast<const float4*>(rp + rope_packed_index(0, k, 0)));
+            rq[k][1] = __ldg(reinterpret_cast<const float4*>(rp + rope_packed_index(0, k, 1)));
+          }
+        }
+      }
       if (!warp_wait(acc_full, static_cast<uint32_t>(local) & 1u, abort_flag)) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const int m2 = tile / p.NT, nt = tile % p.NT;
-      const int row0 = (2 * m2 + static_cast<int>(rank)) * kBM + q * 32;
-      const int n0 = nt * kBN + h * 128;
       const uint32_t tacc = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * 128);
       // All 128 columns are read before the accumulator is released (the next tile's MMAs wait
       // for it), then biased, rounded and staged.
@@ -1527,12 +1544,10 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
         fence_proxy_async_smem();  // the box's generic accesses precede the next tile's bulk copies into staging
       } else {
         // Fused Q/K path: the thread's 128 columns are one head of its row.  Bias first, and the
-        // head's mean square; the rows past M (never stored) read the last row's angles.
+        // head's mean square.
         bool qk = false;
         float nrm = 0.0f;
         const float* gam = nullptr;
-        const float* rp = nullptr;
-        float4 rq[kRopeAhead][2];  // the row's (cos, sin) pairs, kRopeAhead 16-byte units ahead
         if constexpr (kEpi == 1) {
           qk = n0 < p.qk_cols;
           if (qk) {
@@ -1554,15 +1569,6 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
               }
             nrm = rsqrtf(fmaf(ss, 1.0f / kQkvHeadDim, p.eps));
             gam = gamma_sm + (n0 < p.qk_cols / 2 ? 0 : kQkvHeadDim);
-            const int m = row0 + lane < p.M ? row0 + lane : p.M - 1;
-            // The packed table (rope_packed_index) puts the 32 rows of a warp side by side, so each
-            // of these loads reads 512 contiguous bytes; they run kRopeAhead units ahead of their use.
-            rp = p.rope + rope_packed_index(m, 0, 0);
-#pragma unroll
-            for (int k = 0; k < kRopeAhead; ++k) {
-              rq[k][0] = __ldg(reinterpret_cast<const float4*>(rp + rope_packed_index(0, k, 0)));
-              rq[k][1] = __ldg(reinterpret_cast<const float4*>(rp + rope_packed_index(0, k, 1)));
-            }
           }
         }
 #pragma unroll
