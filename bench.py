@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per FLUX-shaped layer and per point of the M x rank sweep (not the driver's line)")
+    ap.add_argument("--sweep-filter", default=None,
+                    help="with --sweep: only the workloads whose name matches this regular expression, no legs")
     ap.add_argument("--leg", choices=["w4a16", "mlp_pair", "qkv_norm_rope"], default=None,
                     help="run one auxiliary leg alone and print its JSON line (not the driver's line; profiling)")
     return ap.parse_args()
@@ -574,8 +576,10 @@ W4A16_SHAPES = [(1, 3072, 18432), (2, 3072, 18432), (4, 3072, 18432), (1, 3072, 
 
 def w4a16_leg(dev, stream, peaks, peak_src, launches: int = 200):
     """The W4A16 layer on FLUX's modulation projections (one token per image: M rows of K = 3072
-    into N = 6*3072 or 3*3072): each launch timed alone with CUDA events on the launching stream,
-    L2 flushed (a 256 MiB read) before every launch, median over ``launches``.  Weight-only
+    into N = 6*3072 or 3*3072).  ``launches`` launches back to back on one stream, rotating over
+    enough copies of the layer's weights that their total exceeds twice the L2 cache (so every
+    launch streams its weights from HBM, with no flush kernel in between), CUDA events around the
+    whole run; the time per launch includes the gap between consecutive launches.  Weight-only
     4-bit layers of this size are bound by HBM, so the roofline is the measured copy bandwidth."""
     import numpy as np
     import torch
@@ -583,46 +587,47 @@ def w4a16_leg(dev, stream, peaks, peak_src, launches: int = 200):
     import synth
     import w4a4_rank_corrected_smooth_b200 as S
 
-    # L2 flush by reading 256 MiB: the lines it leaves in L2 are clean, so the timed launch does not
-    # pay for write-backs of a flush's dirty lines
-    flush = torch.ones(64 << 20, dtype=torch.int32, device=dev)
     out = {}
     prepared = {}
+    l2_bytes = 126 << 20
     for (M, K, N) in W4A16_SHAPES:
         if (K, N) not in prepared:
-            for lin_, _ in prepared.values():
-                lin_.close()
+            for lins_, _ in prepared.values():
+                for l_ in lins_:
+                    l_.close()
             prepared.clear()
             spec = synth.custom(f"flux_modulation_{K}x{N}", M=8, K=K, N=N, rank=0, seed=N)
             X8 = synth.activations_bf16(spec)
-            prepared[(K, N)] = (S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(X8),
-                                             "w4a16", 0, device=dev.index), X8)
-        lin, X8 = prepared[(K, N)]
+            lin = S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(X8), "w4a16", 0,
+                               device=dev.index)
+            wbytes = N * K // 2 + 4 * N * (K // 64)
+            ncopies = max(2, -(-2 * l2_bytes // wbytes))
+            prepared[(K, N)] = ([lin] + [lin.clone() for _ in range(ncopies - 1)], X8)
+        lins, X8 = prepared[(K, N)]
         Xd = bf16_device(np.ascontiguousarray(X8[:M]), dev)
-        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        for _ in range(5):
-            lin.svdq_linear_forward(Xd, M, K, Y, N, None, 0, stream)
-        ts = []
-        for _ in range(launches):
-            flush.sum()
-            hold_gpu(stream, 200.0)  # the launch is queued before the timed region starts
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            lin.svdq_linear_forward(Xd, M, K, Y, N, None, 0, stream)
-            e1.record(stream)
-            e1.synchronize()
-            ts.append(e0.elapsed_time(e1))
+        Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        for i in range(2 * len(lins)):
+            lins[i % len(lins)].svdq_linear_forward(Xd, M, K, Ys[i % 2], N, None, 0, stream)
+        hold_gpu(stream, 30.0 * launches)  # the launches are queued before the timed region starts
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(launches):
+            lins[i % len(lins)].svdq_linear_forward(Xd, M, K, Ys[i % 2], N, None, 0, stream)
+        e1.record(stream)
+        e1.synchronize()
         S.svdq_get_device_error(stream)
-        ms = float(np.median(ts))
+        ms = e0.elapsed_time(e1) / launches
         nbytes = N * K // 2 + 4 * N * (K // 64) + 2 * M * K + 2 * M * N + 4 * K + 4 * N
         gbs = nbytes / (ms / 1e3) / 1e9
         out[f"{M}x{K}x{N}"] = {"us": ms * 1e3, "algorithmic_bytes_per_launch": nbytes, "achieved_gbs": gbs,
-                               "frac": gbs / peaks["hbm_gbs"]}
-    for lin_, _ in prepared.values():
-        lin_.close()
+                               "frac": gbs / peaks["hbm_gbs"], "weight_copies": len(lins)}
+    for lins_, _ in prepared.values():
+        for l_ in lins_:
+            l_.close()
+    timing = f"{launches} launches back to back over rotating weight copies (> 2x L2), events around the run"
     return {"kernel": "w4a16_kernel", "bound": "hbm", "peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src,
-            "timing": f"median of {launches} launches, each alone, L2 flushed (256 MiB read) before each", "shapes": out}
+            "timing": timing, "shapes": out}
 
 
 def run_ours(args):
@@ -790,6 +795,9 @@ def run_sweep(args):
     names = ["flux_qkv_4608x3072x9216_r32", "flux_mlp_up_4608x3072x12288_r32", "flux_mlp_down_4608x12288x3072_r32",
              "dit_qkv_mlp_in_16896x3072x21504_r32", "dit_out_16896x15360x3072_r32"]
     names += [f"sweep_{M}x3072x3072_r{r}" for r in (0, 16, 32, 64, 128) for M in (256, 1024, 4096, 16384)]
+    if args.sweep_filter:
+        import re
+        names = [n for n in names if re.search(args.sweep_filter, n)]
     prepared = {}
     xcache = {}
     for name in names:
@@ -851,6 +859,8 @@ def run_sweep(args):
     for l, l0 in prepared.values():
         l.close()
         l0.close()
+    if args.sweep_filter:
+        return
     print(json.dumps({"sweep": True, "w4a16_modulation": w4a16_leg(dev, stream, peaks, peak_src)}), flush=True)
     print(json.dumps({"sweep": True, "mlp_pair": mlp_pair_leg(dev, stream, peaks)}), flush=True)
 

@@ -149,10 +149,10 @@ svdq_status svdq_workspace_size(const svdq_weights* w, int M, size_t* bytes);
  * X:  device, M rows of K bf16, row stride ldx elements.   Y: device, M x N bf16, stride ldy.
  * workspace: device, >= svdq_workspace_size(w, M) bytes, 256-byte aligned; holds the codes,
  *   scales and T between the two kernels (every row up to M rounded up to a multiple of 256)
- *   and, for large layers when kernel 1 splits K, the fp32 partials of T and one arrival counter
- *   per 128-row tile; contents are scratch and need no initialisation (kernel 1 writes every byte
- *   kernel 2 reads; a counter tagged with another launch restarts, the last slice resets it).  One
- *   workspace must not be used by two forwards whose kernels overlap on the GPU.
+ *   and, when kernel 1 splits K, the fp32 partials of T and one arrival counter per 16-row block;
+ *   contents are scratch and need no initialisation (kernel 1 writes every byte kernel 2 reads; a
+ *   counter tagged with another launch restarts, the last slice resets it).  One workspace must
+ *   not be used by two forwards whose kernels overlap on the GPU.
  * No allocation, no synchronisation.  Errors: INVALID_ARG, CUDA (launch failure). */
 svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
                                 void* workspace, size_t workspace_bytes, void* stream);

@@ -75,7 +75,7 @@ def _check(lin, X, rows, Y, Y_plain, ops, cos, sin, gq, gk, eps=EPS, prec="nvfp4
     N = lin.N
     qk = 2 * N // 3
     got = _y64(Y[torch.from_numpy(rows).cuda()])
-    # V: bit-identical to the plain forward
+    # V: bit-identical to the plain forward (the same MMAs in the same order)
     assert torch.equal(Y[:, qk:].view(torch.int16), Y_plain[:, qk:].view(torch.int16))
     exact = O.linear(X[rows], ops, prec)["Y"]
     ref = O.qkv_norm_rope(exact, D, gq, gk, cos[rows], sin[rows], eps)

@@ -2,9 +2,10 @@
 
 Kernel 1 writes every byte of the activation codes, scales and T that kernel 2 reads.  Its
 warp-level form (16-row blocks, rank <= 32, up to two waves of blocks) sums its warps' shares of T
-in a fixed order; its 128-row-tile form splits K over CTAs, each writing an fp32 partial of T and
-counting itself in a per-tile counter tagged with the launch, and the last slice sums the partials
-in slice order.  These tests check that the result needs no initialised workspace (0xFF
+in a fixed order, and on layers of fewer blocks than two per SM also splits K over CTAs; its
+128-row-tile form always splits K when the grid has room.  A split writes an fp32 partial of T per
+slice and counts itself in a counter (per 16-row block or 128-row tile) tagged with the launch,
+and the last slice sums the partials in slice order.  These tests check that the result needs no initialised workspace (0xFF
 everywhere: garbage counters), that reusing a workspace gives bit-identical results, and that a
 CUDA-graph replay of the forward (the same launch tag every time) does too.
 """
@@ -28,8 +29,9 @@ def _bf16_dev(x_bits):
     return torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-# rank 32: the warp-level form (32 blocks of 16 rows); rank 64: the 128-row tiles, K split in 8
-FORMS = [32, 64]
+# (rank, M): the warp-level form with K split over CTAs (M = 512: 32 blocks of 16 rows, 6 slices)
+# and without (M = 4608: 288 blocks); the 128-row tiles (rank 64), K split in 8
+FORMS = [(32, 512), (32, 4608), (64, 512)]
 
 
 def _layer(M=512, K=3072, N=512, r=32, seed=41):
@@ -49,9 +51,9 @@ def _check_T(lin, X, act):
     assert_t_close(T_gpu, T_ref, O.bf16_to_f32(O.f32_to_bf16(xh)), O.bf16_to_f32(ops["L1"]))
 
 
-@pytest.mark.parametrize("r", FORMS)
-def test_quant_down_needs_no_initialised_workspace_and_repeats_bit_exactly(r):
-    spec, X, lin = _layer(r=r)
+@pytest.mark.parametrize("r,M", FORMS)
+def test_quant_down_needs_no_initialised_workspace_and_repeats_bit_exactly(r, M):
+    spec, X, lin = _layer(M=M, r=r)
     Xd = _bf16_dev(X)
     ws = lin.new_workspace(spec.M)
     ws.fill_(0xFF)  # garbage everywhere
@@ -68,9 +70,9 @@ def test_quant_down_needs_no_initialised_workspace_and_repeats_bit_exactly(r):
     lin.close()
 
 
-@pytest.mark.parametrize("r", FORMS)
-def test_graph_replay_of_the_forward_is_bit_identical_to_eager(r):
-    spec, X, lin = _layer(M=1000, r=r, seed=43)
+@pytest.mark.parametrize("r,M", [(r, 1000 if M == 512 else M) for r, M in FORMS])
+def test_graph_replay_of_the_forward_is_bit_identical_to_eager(r, M):
+    spec, X, lin = _layer(M=M, r=r, seed=43)
     Xd = _bf16_dev(X)
     ws = lin.new_workspace(spec.M)
     Y_eager = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device="cuda")

@@ -72,7 +72,29 @@ struct QdParams {
   uint8_t* codes;
   uint8_t* sf;
   uint8_t* t;
+  int splits;               // K slices per 16-row block (layers of fewer blocks than SMs)
+  float* part;              // [block][slice][16][rank] fp32 partials of T (splits > 1, rank > 0)
+  unsigned long long* cnt;  // per 16-row block: (launch epoch << 8) | slices arrived
+  unsigned long long epoch; // distinct per launch, never 0
 };
+
+// Counts this CTA's slice in the counter of its rows and returns whether it was the last of
+// `splits`.  The counter holds (epoch << 8) | count; a value from another launch (or uninitialised
+// memory) restarts the count, and the last CTA resets it to 0, so a replay of the same launch also
+// starts from 0.  Lock-free (a failed CAS means another slice succeeded); bounded all the same.
+__device__ __forceinline__ bool arrive_slice_counter(unsigned long long* cnt, unsigned long long epoch, int splits,
+                                                     bool* ok) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(cnt);
+  for (int it = 0; it < (1 << 20); ++it) {
+    const unsigned long long nxt = (cur >> 8) == epoch ? cur + 1 : ((epoch << 8) | 1ull);
+    const unsigned long long prev = atomicCAS(cnt, cur, nxt);
+    if (prev == cur) return static_cast<int>(nxt & 0xFFull) == splits;
+    cur = prev;
+  }
+  atomicOr(&g_device_error, kErrWaitQuantDown);
+  *ok = false;
+  return false;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -229,7 +251,8 @@ __global__ void __launch_bounds__(kQdThreads, 2) quant_down_kernel(const QdParam
   // Kernel 2 may be scheduled now (it waits for this grid's completion before reading anything).
   pdl_launch_dependents();
 
-  const int m0 = blockIdx.x * kQdRows;
+  const int blk = blockIdx.x / p.splits, split = blockIdx.x % p.splits;
+  const int m0 = blk * kQdRows;
   int row[2], rin[2];
   bool live[2];
   const uint16_t* xrow[2];
@@ -242,6 +265,7 @@ __global__ void __launch_bounds__(kQdThreads, 2) quant_down_kernel(const QdParam
   }
   const int mt = m0 / kBM;
   const int nch = p.K >> 6;
+  const int c0 = split * nch / p.splits, c1 = (split + 1) * nch / p.splits;  // this CTA's chunks of K
   uint8_t* const codes_t = p.codes + codes_chunk_offset(mt, 0, p.KB, kBM);
   uint8_t* const sf_t = p.sf + sf_chunk_offset(mt, 0, p.KB, kBM);
   const float kInv6 = __frcp_rn(6.0f);
@@ -255,7 +279,7 @@ __global__ void __launch_bounds__(kQdThreads, 2) quant_down_kernel(const QdParam
   // Chunk c into ring slot `slot` (one commit group per call, empty past the end, so that the
   // group count stays in step with the chunks).
   auto issue = [&](int c, int slot) {
-    if (c < nch) {
+    if (c < c1) {
 #pragma unroll
       for (int i = 0; i < 2; ++i)
 #pragma unroll
@@ -266,9 +290,9 @@ __global__ void __launch_bounds__(kQdThreads, 2) quant_down_kernel(const QdParam
     cp_async_commit();
   };
 #pragma unroll
-  for (int q = 0; q < kQdAhead; ++q) issue(warp + q * kQdWarps, q);
+  for (int q = 0; q < kQdAhead; ++q) issue(c0 + warp + q * kQdWarps, q);
   int slot = 0;
-  for (int c = warp; c < nch; c += kQdWarps) {
+  for (int c = c0 + warp; c < c1; c += kQdWarps) {
     cp_async_wait<kQdAhead - 1>();  // this chunk's copies have landed
     uint4 cur[2][2];
 #pragma unroll
@@ -400,6 +424,7 @@ __global__ void __launch_bounds__(kQdThreads, 2) quant_down_kernel(const QdParam
       }
     __syncthreads();
     uint8_t* const tt = p.t + static_cast<size_t>(mt) * kBM * r * 2;
+    float* const pb = p.part + static_cast<size_t>(blk) * p.splits * kQdRows * r;  // this block's partials
     for (int e = threadIdx.x; e < kQdRows * r / 2; e += kQdThreads) {
       const int rw = (2 * e) / r, col = (2 * e) % r;
       float a0 = 0.0f, a1 = 0.0f;
@@ -409,8 +434,42 @@ __global__ void __launch_bounds__(kQdThreads, 2) quant_down_kernel(const QdParam
         a0 += v.x;
         a1 += v.y;
       }
-      *reinterpret_cast<uint32_t*>(tt + lr_offset(static_cast<uint32_t>((m0 + rw) & (kBM - 1)), col, kBM, r)) =
-          pack_bf16x2(a0, a1);
+      if (p.splits == 1)
+        *reinterpret_cast<uint32_t*>(tt + lr_offset(static_cast<uint32_t>((m0 + rw) & (kBM - 1)), col, kBM, r)) =
+            pack_bf16x2(a0, a1);
+      else
+        *reinterpret_cast<float2*>(pb + (static_cast<size_t>(split) * kQdRows + rw) * r + col) = make_float2(a0, a1);
+    }
+    if (p.splits > 1) {
+      // The last slice of the block to finish adds all slices' partials in slice order
+      // (deterministic) and writes bf16 T.  Publication: the CTA barrier orders every thread's
+      // partial stores before thread 0's GPU-scope fence, which is cumulative, and that fence
+      // before the counter update; the last slice fences again before reading.
+      __shared__ int s_last;
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        bool ok = true;
+        __threadfence();
+        const bool last = arrive_slice_counter(p.cnt + blk, p.epoch, p.splits, &ok);
+        if (last) __threadfence();
+        if (!ok) atomicExch(p.cnt + blk, 0ull);  // a replay of this launch starts the count afresh
+        s_last = last ? 1 : 0;
+      }
+      __syncthreads();
+      if (s_last) {
+        for (int e = threadIdx.x; e < kQdRows * r / 2; e += kQdThreads) {
+          const int rw = (2 * e) / r, col = (2 * e) % r;
+          float2 a = __ldcg(reinterpret_cast<const float2*>(pb + static_cast<size_t>(rw) * r + col));
+          for (int q = 1; q < p.splits; ++q) {
+            const float2 v = __ldcg(reinterpret_cast<const float2*>(pb + (static_cast<size_t>(q) * kQdRows + rw) * r + col));
+            a.x += v.x;
+            a.y += v.y;
+          }
+          *reinterpret_cast<uint32_t*>(tt + lr_offset(static_cast<uint32_t>((m0 + rw) & (kBM - 1)), col, kBM, r)) =
+              pack_bf16x2(a.x, a.y);
+        }
+        if (threadIdx.x == 0) atomicExch(p.cnt + blk, 0ull);
+      }
     }
   }
 }
@@ -449,23 +508,6 @@ struct QtParams {
   unsigned long long epoch; // distinct per launch, never 0
 };
 
-// Counts this CTA's slice in the tile's counter and returns whether it was the last of `splits`.
-// The counter holds (epoch << 8) | count; a value from another launch (or uninitialised memory)
-// restarts the count, and the last CTA resets it to 0, so a replay of the same launch also starts
-// from 0.  Lock-free (a failed CAS means another slice succeeded); bounded all the same.
-__device__ __forceinline__ bool arrive_slice_counter(unsigned long long* cnt, unsigned long long epoch, int splits,
-                                                     bool* ok) {
-  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(cnt);
-  for (int it = 0; it < (1 << 20); ++it) {
-    const unsigned long long nxt = (cur >> 8) == epoch ? cur + 1 : ((epoch << 8) | 1ull);
-    const unsigned long long prev = atomicCAS(cnt, cur, nxt);
-    if (prev == cur) return static_cast<int>(nxt & 0xFFull) == splits;
-    cur = prev;
-  }
-  atomicOr(&g_device_error, kErrWaitQuantDown);
-  *ok = false;
-  return false;
-}
 
 template <int PREC>
 __global__ void __launch_bounds__(kQtThreads, 1)
@@ -871,6 +913,13 @@ static EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
+// A tag that differs between launches (56 bits, never 0) for the K-split arrival counters.
+static unsigned long long next_launch_epoch() {
+  static std::atomic<unsigned long long> counter{0};
+  const unsigned long long e = (counter.fetch_add(1) + 1) & ((1ull << 56) - 1);
+  return e == 0 ? 1 : e;
+}
+
 static cudaError_t launch_quant_down_tile(const QuantDownArgs& a, int num_sms, cudaStream_t stream) {
   QtParams p;
   p.M = a.M;
@@ -908,9 +957,7 @@ static cudaError_t launch_quant_down_tile(const QuantDownArgs& a, int num_sms, c
   p.splits = splits;
   p.part = a.part;
   p.cnt = a.cnt;
-  static std::atomic<unsigned long long> epoch_counter{0};
-  p.epoch = (epoch_counter.fetch_add(1) + 1) & ((1ull << 56) - 1);
-  if (p.epoch == 0) p.epoch = 1;
+  p.epoch = next_launch_epoch();
   if (a.precision == 0)
     quant_down_tile_kernel<0><<<mt * splits, kQtThreads, smem, stream>>>(tmap, p);
   else
@@ -919,7 +966,7 @@ static cudaError_t launch_quant_down_tile(const QuantDownArgs& a, int num_sms, c
 }
 
 
-static cudaError_t launch_quant_down_warps(const QuantDownArgs& a, cudaStream_t stream) {
+static cudaError_t launch_quant_down_warps(const QuantDownArgs& a, int num_sms, cudaStream_t stream) {
   QdParams p;
   p.X = a.X;
   p.ldx = a.ldx;
@@ -934,7 +981,21 @@ static cudaError_t launch_quant_down_warps(const QuantDownArgs& a, cudaStream_t 
   p.t = a.t;
   // Every row of the workspace's padded tiles (kernel 2 consumes rows in pairs of 128-row tiles).
   const int mpad = 2 * kBM * ((a.M + 2 * kBM - 1) / (2 * kBM));
-  const unsigned grid = static_cast<unsigned>(mpad / kQdRows);
+  const int blocks = mpad / kQdRows;
+  // Layers of fewer 16-row blocks than two per SM split K over up to 8 CTAs per block (each warp
+  // keeping at least one chunk), within what the workspace's partials of T have room for.
+  int splits = (2 * num_sms) / blocks;
+  const int by_chunks = (a.K / 64) / kQdWarps;
+  if (splits > by_chunks) splits = by_chunks;
+  if (splits > 8) splits = 8;
+  if (a.rank > 0 && splits > a.split_cap) splits = a.split_cap;
+  if (a.rank > 0 && (!a.part || !a.cnt)) splits = 1;
+  if (splits < 1) splits = 1;
+  p.splits = splits;
+  p.part = a.part;
+  p.cnt = a.cnt;
+  p.epoch = next_launch_epoch();
+  const unsigned grid = static_cast<unsigned>(blocks * splits);
   const size_t shares = static_cast<size_t>(kQdWarps) * kQdRows * a.rank * sizeof(float);
   const size_t smem = shares > kQdRingBytes ? shares : kQdRingBytes;
   // rank 0 or at most 32 (the caller dispatches larger ranks to the 128-row tiles)
@@ -953,7 +1014,7 @@ static cudaError_t launch_quant_down_warps(const QuantDownArgs& a, cudaStream_t 
 // otherwise, and whenever the caller's workspace has room for their K-split partials only.
 cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t stream) {
   const int mpad = 2 * kBM * ((a.M + 2 * kBM - 1) / (2 * kBM));
-  if (a.rank <= 32 && mpad / kQdRows <= 2 * num_sms) return launch_quant_down_warps(a, stream);
+  if (a.rank <= 32 && mpad / kQdRows <= 2 * num_sms) return launch_quant_down_warps(a, num_sms, stream);
   return launch_quant_down_tile(a, num_sms, stream);
 }
 
@@ -1000,6 +1061,9 @@ static cudaError_t make_rows_map(CUtensorMap* map, const void* base, uint64_t by
 // stages before the k-blocks.  Kernel 2 is launched as a programmatic dependent of kernel 1.
 
 constexpr int kGStages = 5;
+// The fused MLP epilogue outlasts the k-loop, which then needs fewer stages in flight; its fourth
+// stage's shared memory holds the epilogue's GELU table instead.
+__host__ __device__ constexpr int gemm_stages(int epi) { return epi == 2 ? 4 : kGStages; }
 // Warp roles, four warpgroups: 0 = the scale warps (warp w writes TMEM lane quadrant w); 1 = the
 // operand producer, the MMA issuer, the scale producer and one idle warp; 2 and 3 = the epilogue.
 constexpr int kGSfWarps = 4;
@@ -1192,13 +1256,12 @@ __device__ __forceinline__ float gelu_bf16(float y) {
   return __float_as_uint(lo) == __float_as_uint(hi) ? lo : gelu_bf16_slow(y);
 }
 
-// The fused MLP epilogue evaluates GELU for every hidden value, so its common range goes through a
-// table in shared memory: the exact bf16 GELU of every bf16 input with |y| in [2^-4, 8) (both
-// signs, 7 binades of 128 values), filled by gelu_bf16 itself at kernel start.  Below 2^-4 a short
-// series does it (bracketed like gelu_bf16), from 8 up GELU(y) rounds to y, and below -8 the full
-// evaluation runs.
-constexpr int kGeluTblE0 = 123;     // bf16 exponent field of 2^-4
-constexpr int kGeluTblBinades = 7;  // 2^-4 .. 2^3
+// The fused MLP epilogue evaluates GELU for every hidden value, so the range that holds nearly all
+// of them goes through a table in shared memory: the exact bf16 GELU of every bf16 input with |y|
+// in [2^-10, 16) (both signs, 14 binades of 128 values, 7 KB), filled by gelu_bf16 itself at kernel
+// start.  Outside that range the rounded value has a closed form (gelu_bf16_outside_table).
+constexpr int kGeluTblE0 = 117;      // bf16 exponent field of 2^-10
+constexpr int kGeluTblBinades = 14;  // 2^-10 .. 2^3
 constexpr int kGeluTblSize = 2 * kGeluTblBinades * 128;
 
 __device__ __noinline__ void fill_gelu_table(uint16_t* tbl, int tid, int nthreads) {
@@ -1210,19 +1273,22 @@ __device__ __noinline__ void fill_gelu_table(uint16_t* tbl, int tid, int nthread
   }
 }
 
-// 2^-125 <= |y| < 2^-4: GELU(y) = y (1/2 + c1 (y - y^3/6 + y^5/40 - y^7/336) + O(y^9)) with
-// c1 = 1/sqrt(2 pi); the truncation is below 1e-14 relative, the fp32 Horner steps a few ulp, so
-// the result is bracketed by 2^-20 relative and the rare straddling case falls back to double.
-__device__ __forceinline__ float gelu_bf16_series(float y) {
-  const float c1 = 0.3989422804014327f, c3 = -0.06649038006690545f, c5 = 0.009973557010035818f,
-              c7 = -0.0011873282154803355f;
-  const float y2 = __fmul_rn(y, y);
-  const float p = __fmaf_rn(y2, __fmaf_rn(y2, __fmaf_rn(y2, c7, c5), c3), c1);
-  const float g = __fmul_rn(y, __fmaf_rn(y, p, 0.5f));
-  const float d = __fmaf_rn(fabsf(g), 0x1p-20f, 0x1p-140f);
-  const float lo = __bfloat162float(__float2bfloat16_rn(__fsub_rn(g, d)));
-  const float hi = __bfloat162float(__float2bfloat16_rn(__fadd_rn(g, d)));
-  return __float_as_uint(lo) == __float_as_uint(hi) ? lo : gelu_bf16_slow(y);
+// The bf16 inputs outside the table, where GELU(y) = y/2 + y^2/sqrt(2 pi) + O(y^4) near zero and
+// y (1 - Q(|y|)) or |y| Q(|y|) in the tails (Q the normal upper tail):
+// - |y| < 2^-125: the tiny-input integer path (y/2 may be a bf16 subnormal with a tie);
+// - 2^-125 <= |y| < 2^-10: y/2, a normal bf16 number; the correction, below 0.8 |y| |y/2| <
+//   2^-10 |y/2|, stays under half the bf16 spacing next to y/2 on either side (at least 2^-9 |y/2|,
+//   the side toward zero of a power of two included), so it cannot move the rounding;
+// - y >= 16: y, since Q(16) < 1e-57;
+// - y <= -16: -0, since |y| Q(|y|) < 1e-56 is below half the smallest bf16 subnormal (2^-134) and
+//   the exact value is negative;
+// - NaN: itself.
+__device__ __forceinline__ float gelu_bf16_outside_table(float y) {
+  const uint32_t a = __float_as_uint(y) & 0x7FFFFFFFu;
+  if (a < 0x01000000u) return gelu_bf16_tiny(__float_as_uint(y));
+  if (a < 0x3A800000u) return __fmul_rn(0.5f, y);
+  if (y <= -16.0f) return -0.0f;
+  return y;
 }
 
 // The correctly rounded bf16 GELU of a bf16 y (as fp32), with the table `tbl` in shared memory.
@@ -1231,12 +1297,7 @@ __device__ __forceinline__ float gelu_bf16_tab(float y, const uint16_t* tbl) {
   const uint32_t e = ((b >> 7) & 0xFFu) - static_cast<uint32_t>(kGeluTblE0);
   if (e < static_cast<uint32_t>(kGeluTblBinades))
     return __uint_as_float(static_cast<uint32_t>(tbl[((b >> 15) * kGeluTblBinades + e) * 128u + (b & 127u)]) << 16);
-  if (y >= 8.0f) return y;  // y Phi(y) = y (1 - Q(y)) with Q(y) < 1e-15: rounds to y
-  if ((__float_as_uint(y) & 0x7FFFFFFFu) < 0x3D800000u) {  // |y| < 2^-4
-    if ((__float_as_uint(y) & 0x7FFFFFFFu) < 0x01000000u) return gelu_bf16_tiny(__float_as_uint(y));
-    return gelu_bf16_series(y);
-  }
-  return gelu_bf16(y);
+  return gelu_bf16_outside_table(y);
 }
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
@@ -1255,13 +1316,14 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
 template <int kEpi>
 __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_constant__ GemmMaps maps,
                                                                     const GemmParams p) {
+  constexpr int kNS = gemm_stages(kEpi);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* staging = smem + kGStages * kGStage;
+  uint8_t* staging = smem + kNS * kGStage;
   uint64_t* full = reinterpret_cast<uint64_t*>(staging + kGStaging);  // (both) this CTA's tiles landed
-  uint64_t* empty = full + kGStages;        // (both) MMAs done with the stage
-  uint64_t* ready = empty + kGStages;       // (leader) both CTAs' tiles landed and scales written
-  uint64_t* acc_full = ready + kGStages;    // (both) accumulator ready
+  uint64_t* empty = full + kNS;        // (both) MMAs done with the stage
+  uint64_t* ready = empty + kNS;       // (leader) both CTAs' tiles landed and scales written
+  uint64_t* acc_full = ready + kNS;    // (both) accumulator ready
   uint64_t* acc_empty = acc_full + 1;       // (leader) both CTAs drained the accumulator
   uint64_t* lr_full = acc_empty + 1;        // (leader) both CTAs' low-rank operands landed in staging
   uint64_t* stg_free = lr_full + 1;         // (both) the epilogue's stores finished reading staging
@@ -1279,11 +1341,13 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
   const int tiles = p.MT2 * p.NT;
   // Up to rank 64 the low-rank operands (T and this CTA's half of L2: 512 r bytes) fit in the
   // epilogue's staging, which is idle during a tile's k-loop: they are loaded there once the
-  // previous tile's stores have read it, and their MMAs close the tile.  Larger ranks take
-  // ring stages before the k-blocks.
-  const bool lr_in_staging = r > 0 && r <= 64;
+  // previous tile's stores have read it, and their MMAs close the tile.  Larger ranks, and the
+  // fused epilogues (which can outlast a k-loop: the MMAs would wait for them), take ring stages
+  // after the k-blocks; either way the tile's MMAs run in the same order (k-blocks, then the up
+  // projection), so every epilogue mode sees the same accumulator.
+  const bool lr_in_staging = kEpi == 0 && r > 0 && r <= 64;
   const int nlr_ring = lr_in_staging ? 0 : nlr;
-  const int nstages_tile = nlr_ring + p.KB;
+  const int nstages_tile = p.KB + nlr_ring;  // k-blocks, then (ring) low-rank chunks
   // Tiles of this pair: interleaved (pair, pair + npairs, ...), except in the fused MLP mode, which
   // walks a contiguous m-major range so that consecutive tiles share rows and their partials of the
   // down layer's T accumulate in one slot.
@@ -1292,7 +1356,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
   const int t_step = kEpi == 2 ? 1 : npairs;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kGStages; ++s) {
+    for (int s = 0; s < kNS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&ready[s], 2 * kGSfWarps);
@@ -1653,7 +1717,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
           ok = false;
           break;
         }
-        if (j >= nlr_ring) {
+        if (j < p.KB) {
           tc_fence_after();  // the MMAs that last read this buffer completed before the stage refilled
           const uint8_t* src = smem + st * kGStage + kGA + kGB + 16 * lane;
           uint32_t v[3][16];
@@ -1674,7 +1738,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(ready_leader + 8u * st);
-        if (++st == kGStages) {
+        if (++st == kNS) {
           st = 0;
           ph ^= 1u;
         }
@@ -1698,22 +1762,23 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
               break;
             }
             uint8_t* sb = smem + st * kGStage;
-            if (j < nlr_ring) {
-              const uint32_t cw = lr_chunk_width(r, j);
+            if (j >= p.KB) {  // low-rank chunk j - KB
+              const int lc = j - p.KB;
+              const uint32_t cw = lr_chunk_width(r, lc);
               const uint32_t tb = kBM * cw * 2, lb = (kBN / 2) * cw * 2;
               mbar_arrive_expect_tx(&full[st], tb + lb);
-              const int trow = static_cast<int>((static_cast<size_t>(mt) * kBM * r * 2 + static_cast<size_t>(kBM) * kLrChunk * 2 * j) / 256);
-              const int lrow = static_cast<int>((static_cast<size_t>(nt) * kBN * r * 2 + static_cast<size_t>(kBN) * kLrChunk * 2 * j + rank * lb) / 256);
+              const int trow = static_cast<int>((static_cast<size_t>(mt) * kBM * r * 2 + static_cast<size_t>(kBM) * kLrChunk * 2 * lc) / 256);
+              const int lrow = static_cast<int>((static_cast<size_t>(nt) * kBN * r * 2 + static_cast<size_t>(kBN) * kLrChunk * 2 * lc + rank * lb) / 256);
               for (uint32_t q = 0; q < tb / 4096; ++q) tma_load_2d(sb + 4096 * q, &maps.t, 0, trow + 16 * q, &full[st]);
               for (uint32_t q = 0; q < lb / 4096; ++q) tma_load_2d(sb + kGA + 4096 * q, &maps.l2, 0, lrow + 16 * q, &full[st]);
             } else {
-              const int kb = j - nlr_ring;
+              const int kb = j;
               mbar_arrive_expect_tx(&full[st], kGStage);
               tma_load_2d(sb, &maps.a, 0, static_cast<int>(codes_chunk_offset(mt, kb, p.KB, kBM) / 256), &full[st]);
               tma_load_2d(sb + kGA, &maps.b, 0, static_cast<int>((codes_chunk_offset(nt, kb, p.KB, kBN) + rank * kGB) / 256),
                           &full[st]);
             }
-            if (++st == kGStages) {
+            if (++st == kNS) {
               st = 0;
               ph ^= 1u;
             }
@@ -1733,18 +1798,18 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
           const int m2 = tile / p.NT, nt = tile % p.NT;
           const int mt = 2 * m2 + static_cast<int>(rank);
           for (int j = 0; j < nstages_tile; ++j) {
-            if (j >= nlr_ring) {
+            if (j < p.KB) {
               if (*abort_flag || !wait_parity_bounded(&empty[st], ph ^ 1u, kErrWaitGemm)) {
                 ok = false;
                 break;
               }
-              const int kb = j - nlr_ring;
+              const int kb = j;
               uint8_t* sb = smem + st * kGStage;
               tma_load_2d(sb + kGA + kGB, &maps.sfa, 0, static_cast<int>(sf_chunk_offset(mt, kb, p.KB, kBM) / 256), &full[st]);
               tma_load_2d(sb + kGA + kGB + kGSfa, &maps.sfb, 0, static_cast<int>(sf_chunk_offset(nt, kb, p.KB, kBN) / 256),
                           &full[st]);
             }
-            if (++st == kGStages) {
+            if (++st == kNS) {
               st = 0;
               ph ^= 1u;
             }
@@ -1775,8 +1840,8 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
             }
             tc_fence_after();
             const uint32_t sb = smem_u32(smem + st * kGStage);
-            if (j < nlr_ring) {
-              const uint32_t cw = lr_chunk_width(r, j);
+            if (j >= p.KB) {  // low-rank chunk j - KB
+              const uint32_t cw = lr_chunk_width(r, j - p.KB);
               const uint64_t ad = smem_desc(sb, 128, cw * 16, kLayoutNone);
               const uint64_t bd = smem_desc(sb + kGA, 128, cw * 16, kLayoutNone);
               for (uint32_t ks = 0; ks < cw / 16; ++ks) {
@@ -1794,7 +1859,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
               }
             }
             tc_commit2_both(smem_u32(&empty[st]));
-            if (++st == kGStages) {
+            if (++st == kNS) {
               st = 0;
               ph ^= 1u;
             }
@@ -2364,9 +2429,9 @@ static cudaError_t launch_gemm_int4(const GemmArgs& a, int num_sms, cudaStream_t
   return cudaGetLastError();
 }
 
-static size_t gemm_smem_bytes() {
-  constexpr size_t extra = 2 * kQkvHeadDim * 4 > kGeluTblSize * 2 ? 2 * kQkvHeadDim * 4 : kGeluTblSize * 2;
-  return 1024 + kGStages * kGStage + kGStaging + 256 + extra;
+static size_t gemm_smem_bytes(int mode) {
+  const size_t extra = mode == 2 ? kGeluTblSize * 2 : (mode == 1 ? 2 * kQkvHeadDim * 4 : 0);
+  return 1024 + static_cast<size_t>(gemm_stages(mode)) * kGStage + kGStaging + 256 + extra;
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
@@ -2416,8 +2481,8 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const size_t smem = gemm_smem_bytes();
   const int mode = a.mlp ? 2 : (a.qk_cols > 0 ? 1 : 0);
+  const size_t smem = gemm_smem_bytes(mode);
   auto kernel = mode == 2 ? gemm_nvfp4_kernel<2> : (mode == 1 ? gemm_nvfp4_kernel<1> : gemm_nvfp4_kernel<0>);
   // The epilogue warpgroups' setmaxnreg.inc waits until the block's pool holds their share, and
   // the pool is the launch's registers a thread x threads: refuse to launch a build whose count

@@ -91,6 +91,7 @@ constexpr int kW4A16MaxK = 49152;
 cudaError_t launch_selftest_wait(int spin_limit, cudaStream_t stream);
 cudaError_t launch_selftest_gelu(const uint16_t* in, uint16_t* out, int n, cudaStream_t stream);
 cudaError_t read_and_clear_device_error(unsigned int* value, cudaStream_t stream);
+cudaError_t read_and_clear_w4a16_error(unsigned int* value, cudaStream_t stream);
 
 // Fixed-size scratch in the library's device module (for the allocation-free forward).
 size_t noalloc_scratch_bytes();

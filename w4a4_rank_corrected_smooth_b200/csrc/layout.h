@@ -86,9 +86,9 @@ struct WorkspaceLayout {
   int m_tiles = 0, split_cap = 1;
 };
 
-// Workspace: activation codes, scales and T (bf16) of every row of the padded tiles and, for the
-// 128-row-tile form of kernel 1 when it splits K (rank > 0), the fp32 partials of T of every slice
-// plus one arrival counter per 128-row tile.
+// Workspace: activation codes, scales and T (bf16) of every row of the padded tiles and, for kernel 1
+// when it splits K (rank > 0), the fp32 partials of T of every slice plus one arrival counter per
+// 16-row block (the 128-row-tile form uses the first one per 128-row tile).
 inline WorkspaceLayout workspace_layout(int M, int K, int r) {
   WorkspaceLayout w;
   w.m_tiles = 2 * ((M + 2 * kBM - 1) / (2 * kBM));  // kernel 2 consumes rows in pairs of 128-row tiles
@@ -104,7 +104,7 @@ inline WorkspaceLayout workspace_layout(int M, int K, int r) {
     w.part = align_up(end, 1024);
     end = w.part + mpad * static_cast<size_t>(w.split_cap) * static_cast<size_t>(r) * 4;
     w.cnt = align_up(end, 256);
-    end = w.cnt + static_cast<size_t>(w.m_tiles) * 8;
+    end = w.cnt + mpad / 16 * 8;
   }
   w.total = M > 0 ? align_up(end, 1024) : 0;
   return w;

@@ -10,8 +10,9 @@
 
 namespace svdq {
 
-// Device error word (one per device context), read and cleared by svdq_get_device_error().
-// Defined by the one translation unit that holds the kernels (it includes this header once).
+// Device error word (one per device context and translation unit), read and cleared by
+// svdq_get_device_error().  Defined here for the translation unit of the W4A4 kernels; the W4A16
+// kernel's unit defines its own before including this header.
 #ifndef SVDQ_DEVICE_ERROR_DEFINED
 #define SVDQ_DEVICE_ERROR_DEFINED
 __device__ unsigned int g_device_error = 0;
@@ -22,6 +23,7 @@ enum : unsigned int {
   kErrWaitGemm = 2u,
   kErrWaitSelftest = 4u,
   kErrLaunchShape = 8u,
+  kErrWaitW4A16 = 16u,
 };
 
 // Time limit of one bounded wait (nanoseconds of %globaltimer).

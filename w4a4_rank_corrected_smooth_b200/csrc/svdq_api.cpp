@@ -105,17 +105,23 @@ void free_device(svdq_weights* w) {
   w->d_bias = nullptr;
 }
 
+// Workspace bytes of a forward (kernel 1's region: codes, scales, T and its K-split partials).
+size_t forward_workspace_bytes(const svdq_weights* w, int M) {
+  if (w->precision == SVDQ_W4A16 || M <= 0) return 0;
+  return svdq::workspace_layout(M, w->K, w->rank).total;
+}
+
 svdq_status check_forward_common(const svdq_weights* w, int M, const void* ws, size_t ws_bytes) {
   if (!w) return fail(SVDQ_ERR_INVALID_ARG, "weights handle is NULL");
   if (M < 0) return fail(SVDQ_ERR_INVALID_ARG, "M=%d is negative", M);
   if (M == 0) return SVDQ_OK;
   if (w->precision == SVDQ_W4A16) return SVDQ_OK;  // no workspace: one kernel, nothing in between
-  const svdq::WorkspaceLayout L = svdq::workspace_layout(M, w->K, w->rank);
+  const size_t need = forward_workspace_bytes(w, M);
   if (!ws) return fail(SVDQ_ERR_INVALID_ARG, "workspace is NULL");
   if (!aligned(ws, 256)) return fail(SVDQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  if (ws_bytes < L.total)
+  if (ws_bytes < need)
     return fail(SVDQ_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu bytes needed for M=%d", ws_bytes,
-                L.total, M);
+                need, M);
   return SVDQ_OK;
 }
 
@@ -286,9 +292,12 @@ svdq_status svdq_check_device(int device) {
 }
 
 svdq_status svdq_get_device_error(void* stream) {
-  unsigned int v = 0;
+  unsigned int v = 0, vw = 0;
   cudaError_t e = svdq::read_and_clear_device_error(&v, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  e = svdq::read_and_clear_w4a16_error(&vw, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the W4A16 kernel's device error word");
+  v |= vw;
   if (v != 0) return fail(SVDQ_ERR_TIMEOUT, "a kernel's bounded wait gave up (device error bits 0x%x)", v);
   return SVDQ_OK;
 }
@@ -471,7 +480,7 @@ svdq_status svdq_export_weights(const svdq_weights* w, float* inv_lambda, uint8_
 svdq_status svdq_workspace_size(const svdq_weights* w, int M, size_t* bytes) {
   if (!w || !bytes) return fail(SVDQ_ERR_INVALID_ARG, "NULL argument");
   if (M < 0) return fail(SVDQ_ERR_INVALID_ARG, "M=%d is negative", M);
-  *bytes = w->precision == SVDQ_W4A16 ? 0 : svdq::workspace_layout(M, w->K, w->rank).total;
+  *bytes = forward_workspace_bytes(w, M);
   return SVDQ_OK;
 }
 
@@ -480,7 +489,7 @@ svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const void* X, in
   if (!w) return fail(SVDQ_ERR_INVALID_ARG, "weights handle is NULL");
   if (M < 0) return fail(SVDQ_ERR_INVALID_ARG, "M=%d is negative", M);
   if (M == 0) return SVDQ_OK;
-  const size_t need = w->precision == SVDQ_W4A16 ? 0 : svdq::workspace_layout(M, w->K, w->rank).total;
+  const size_t need = forward_workspace_bytes(w, M);
   const size_t have = svdq::noalloc_scratch_bytes();
   if (need > have)
     return fail(SVDQ_ERR_INVALID_ARG,
