@@ -866,10 +866,11 @@ def run_sweep(args):
 
 
 def mlp_pair_leg(dev, stream, peaks, steps: int = 200):
-    """FLUX's MLP pair (4608 x 3072 -> 12288 -> GELU -> 3072, rank 32, NVFP4): the fused pair
+    """FLUX's MLP pair (4608 x 3072 -> 12288 -> GELU -> 3072, rank 32, NVFP4) three ways: fused
     (the up layer's epilogue emits the down layer's 4-bit operands; the hidden activation never
-    reaches memory) against the unfused sequence of the same layers (up forward writing bf16 Y,
-    GELU by torch, down forward), whole steps timed with CUDA events, two rotating buffer sets."""
+    reaches memory), GELU-fused (the up layer's GELU-output forward, then the down layer's
+    forward on the hidden activation) and unfused (up forward writing bf16 Y, GELU by torch, down
+    forward); whole steps timed with CUDA events, two rotating buffer sets."""
     import torch
 
     import synth
@@ -896,6 +897,12 @@ def mlp_pair_leg(dev, stream, peaks, steps: int = 200):
         S.svdq_mlp_forward(up, down, b["X"], M, b["X"].stride(0), b["Y"], b["Y"].stride(0), b["ws_up"],
                            b["ws_up"].numel(), b["mid"], b["mid"].numel(), stream)
 
+    def gelu_fused(b):
+        up.svdq_linear_forward_gelu(b["X"], M, b["X"].stride(0), b["H"], b["H"].stride(0), b["ws_up"],
+                                    b["ws_up"].numel(), stream)
+        down.svdq_linear_forward(b["H"], M, b["H"].stride(0), b["Y"], b["Y"].stride(0), b["ws_down"],
+                                 b["ws_down"].numel(), stream)
+
     def unfused(b):
         up.svdq_linear_forward(b["X"], M, b["X"].stride(0), b["H"], b["H"].stride(0), b["ws_up"], b["ws_up"].numel(),
                                stream)
@@ -904,7 +911,7 @@ def mlp_pair_leg(dev, stream, peaks, steps: int = 200):
                                  b["ws_down"].numel(), stream)
 
     out = {}
-    for name, fn in (("unfused", unfused), ("fused", fused), ("unfused", unfused), ("fused", fused)):
+    for name, fn in (("unfused", unfused), ("fused", fused), ("gelu_fused", gelu_fused)) * 2:
         for i in range(10):
             fn(sets[i % 2])
         a = torch.cuda.Event(enable_timing=True)
@@ -919,8 +926,10 @@ def mlp_pair_leg(dev, stream, peaks, steps: int = 200):
     S.svdq_get_device_error(stream)
     flops = up_spec.flops + down_spec.flops
     out.update({"tflops_fused": flops / (out["ms_fused"] / 1e3) / 1e12,
+                "tflops_gelu_fused": flops / (out["ms_gelu_fused"] / 1e3) / 1e12,
                 "tflops_unfused": flops / (out["ms_unfused"] / 1e3) / 1e12,
-                "speedup": out["ms_unfused"] / out["ms_fused"], "steps": steps,
+                "speedup": out["ms_unfused"] / out["ms_fused"],
+                "speedup_gelu_fused": out["ms_unfused"] / out["ms_gelu_fused"], "steps": steps,
                 "unfused_gelu": "torch.nn.functional.gelu on the bf16 hidden tensor (a library kernel)"})
     up.close()
     down.close()

@@ -224,8 +224,8 @@ svdq_status svdq_linear_forward_qkv_norm_rope(const svdq_weights* w, const void*
  * and writes, instead of its output, the down layer's activation codes and scales of h and the
  * fp32 partials of the down layer's T (warp-level bf16 MMAs per half tile); a small kernel adds
  * the partials in a fixed order into T; the down layer's kernel 2 then runs as usual.  GELU is
- * computed in fp32 (erff), so h can differ from an exact evaluation by one bf16 ulp where the
- * value sits on a rounding boundary.
+ * rounded correctly to bf16 (a shared-memory table of exact values for |x| in [2^-10, 16), closed
+ * forms outside it; svdq_selftest_gelu_bf16 runs the same path).
  * Both layers NVFP4, up->N == down->K, the down layer's rank 0, 16 or 32, same device.
  * ws_up: the up layer's workspace (svdq_workspace_size(up, M)).  ws_mid: the down layer's
  * workspace followed by the T partials, svdq_mlp_workspace_size(up, down, M) bytes, 256-byte
@@ -236,6 +236,16 @@ svdq_status svdq_mlp_workspace_size(const svdq_weights* up, const svdq_weights* 
 svdq_status svdq_mlp_forward(const svdq_weights* up, const svdq_weights* down, const void* X, int M, int ldx,
                              void* Y, int ldy, void* ws_up, size_t ws_up_bytes, void* ws_mid,
                              size_t ws_mid_bytes, void* stream);
+
+/* The forward with GELU on its output: Y = bf16(GELU(bf16(acc + bias))), GELU as in
+ * svdq_mlp_forward (correctly rounded).  The lighter of the two fusions of an MLP pair ([ND]
+ * "Introducing Nunchaku Lite" names fused GELU/MLP kernels): GELU in the up layer's kernel 2
+ * epilogue, Y (the hidden activation) written once and read by the down layer's own forward,
+ * whose kernel 1 quantizes it; svdq_mlp_forward instead keeps the hidden activation out of memory
+ * but does the quantization in the up layer's epilogue.  NVFP4 layers only (INVALID_ARG
+ * otherwise).  Arguments, workspace and errors as svdq_linear_forward. */
+svdq_status svdq_linear_forward_gelu(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
+                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* Kernel 1 alone (same arguments as the forward minus Y): fills the workspace. */
 svdq_status svdq_quant_down(const svdq_weights* w, const void* X, int M, int ldx, void* workspace,

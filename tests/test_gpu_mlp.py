@@ -8,7 +8,9 @@ activation codes and scales bit-exact against the oracle's quantizer applied to 
 layer's own bf16 output (the up layer's output is where the GPU's fp32 accumulation and the
 oracle's exact sum may round to neighbouring bf16 values, so both sides take the hidden value
 from the same up-layer output); its T within the per-element bound of the fp32 accumulation;
-two runs bit-identical.
+two runs bit-identical.  The GELU-output forward (the lighter fusion: GELU in the up layer's
+epilogue, the hidden activation through memory to the down layer's forward) equals the oracle's
+exact GELU of the plain forward on every element.
 """
 import numpy as np
 import pytest
@@ -141,3 +143,69 @@ def test_argument_checks():
         S.svdq_mlp_workspace_size(up, down_i4, 64)
     for lin in (up, down, up_bad, down64, down_i4):
         lin.close()
+
+
+def _plain_and_gelu(lin, X):
+    """The plain forward and the GELU-output forward of one layer on the same input."""
+    M = X.shape[0]
+    Xd = _bf16_dev(X)
+    ws = lin.new_workspace(M)
+    Yp = torch.full((M, lin.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    Yg = torch.full((M, lin.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lin.svdq_linear_forward(Xd, M, Xd.stride(0), Yp, Yp.stride(0), ws, ws.numel())
+    lin.svdq_linear_forward_gelu(Xd, M, Xd.stride(0), Yg, Yg.stride(0), ws, ws.numel())
+    S.svdq_get_device_error()
+    return Yp, Yg
+
+
+@pytest.mark.parametrize("M,K,N,r", [(300, 512, 768, 16), (1, 256, 256, 0), (4608, 3072, 12288, 32)])
+def test_gelu_forward_is_the_exact_gelu_of_the_plain_forward(M, K, N, r):
+    """The GELU-output forward: every element equals the oracle's correctly rounded bf16 GELU of the
+    plain forward's element (the same MMAs in the same order give the same bf16 output first)."""
+    spec = synth.custom(f"gelu_fwd_{M}_{N}", M=M, K=K, N=N, rank=r, seed=60 + M)
+    X = synth.activations_bf16(spec)
+    lin = S.SVDQLinear(synth.weight_bf16(spec), synth.bias_bf16(spec), synth.act_absmax(X), "nvfp4", r)
+    Yp, Yg = _plain_and_gelu(lin, X)
+    rows = np.arange(M) if M <= 512 else np.sort(np.random.default_rng(M).choice(M, 48, replace=False))
+    idx = torch.from_numpy(rows).cuda()
+    yp = Yp[idx].view(torch.int16).cpu().numpy().view(np.uint16)
+    yg = Yg[idx].view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(yg, O.gelu_bf16(yp))
+    lin.close()
+
+
+def test_mlp_pair_through_the_gelu_forward():
+    """The lighter fusion of FLUX's MLP pair: the up layer's GELU-output forward, then the down
+    layer's forward on that hidden activation; Y against the oracle's pair on sampled rows, and
+    the down layer's codes and scales bit-exact against the oracle's quantizer of the hidden rows."""
+    X, up, down = _layers(4608, 3072, 12288, 3072, 32, 32, seed=70)
+    M = X.shape[0]
+    _, H = _plain_and_gelu(up, X)
+    ws = down.new_workspace(M)
+    Y = torch.full((M, down.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    down.svdq_linear_forward(H, M, H.stride(0), Y, Y.stride(0), ws, ws.numel())
+    S.svdq_get_device_error()
+    rows = np.sort(np.random.default_rng(13).choice(M, 64, replace=False))
+    ref = O.mlp_pair(X[rows], up.export_weights(), down.export_weights(), "nvfp4")
+    got = _y64(Y[torch.from_numpy(rows).cuda()])
+    assert O.rel_fro(got, ref["Y"]) <= REL_FRO_TOL
+    assert np.max(np.abs(got - ref["Y"])) <= MAX_ABS_TOL * np.max(np.abs(ref["Y"]))
+    h = H[torch.from_numpy(rows).cuda()].view(torch.int16).cpu().numpy().view(np.uint16)
+    _, cx, sx = O.quantize_activations(h, down.export_weights()["inv_lambda"], "nvfp4")
+    act = down.svdq_export_activations(ws, M)
+    assert np.array_equal(act["codes_x"][rows], cx) and np.array_equal(act["scales_x"][rows], sx)
+    up.close()
+    down.close()
+
+
+def test_gelu_forward_refuses_int4():
+    spec = synth.custom("gelu_i4", M=16, K=256, N=256, rank=16, seed=95)
+    X = synth.activations_bf16(spec)
+    lin = S.SVDQLinear(synth.weight_bf16(spec), None, synth.act_absmax(X), "int4", 16)
+    Xd = _bf16_dev(X)
+    ws = lin.new_workspace(16)
+    Y = torch.empty((16, 256), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(S.SVDQError) as ei:
+        lin.svdq_linear_forward_gelu(Xd, 16, 256, Y, 256, ws, ws.numel())
+    assert ei.value.status == 1
+    lin.close()

@@ -60,6 +60,7 @@ def _load() -> ctypes.CDLL:
         "svdq_workspace_size": ([vp, i, ctypes.POINTER(sz)], i),
         "svdq_linear_forward": ([vp, vp, i, i, vp, i, vp, sz, vp], i),
         "svdq_linear_forward_noalloc": ([vp, vp, i, i, vp, i, vp], i),
+        "svdq_linear_forward_gelu": ([vp, vp, i, i, vp, i, vp, sz, vp], i),
         "svdq_linear_forward_qkv_norm_rope": ([vp, vp, i, i, vp, i, vp, vp, ctypes.c_float, vp, i, vp, sz, vp], i),
         "svdq_mlp_workspace_size": ([vp, vp, i, ctypes.POINTER(sz)], i),
         "svdq_mlp_forward": ([vp, vp, vp, i, i, vp, i, vp, sz, vp, sz, vp], i),
@@ -83,7 +84,7 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 DECLARED_SYMBOLS = tuple(sorted([
     "svdq_status_string", "svdq_last_error", "svdq_check_device", "svdq_get_device_error", "svdq_prepare_weights",
-    "svdq_free_weights", "svdq_clone_weights", "svdq_get_weights_info", "svdq_export_weights", "svdq_workspace_size", "svdq_linear_forward", "svdq_linear_forward_noalloc",
+    "svdq_free_weights", "svdq_clone_weights", "svdq_get_weights_info", "svdq_export_weights", "svdq_workspace_size", "svdq_linear_forward", "svdq_linear_forward_noalloc", "svdq_linear_forward_gelu",
     "svdq_linear_forward_qkv_norm_rope", "svdq_mlp_workspace_size", "svdq_mlp_forward",
     "svdq_quant_down", "svdq_gemm_up", "svdq_export_activations", "svdq_quantize_rows_host", "svdq_prepare_host",
     "svdq_selftest_wait_timeout", "svdq_selftest_gelu_bf16", "svdq_rope_packed_size", "svdq_pack_rope"]))
@@ -264,6 +265,12 @@ class SVDQLinear:
     def svdq_linear_forward(self, X, M: int, ldx: int, Y, ldy: int, workspace, workspace_bytes: int, stream=None):
         _check(_lib.svdq_linear_forward(self._h, _ptr(X), M, ldx, _ptr(Y), ldy, _ptr(workspace), workspace_bytes,
                                         _stream(stream)))
+
+    def svdq_linear_forward_gelu(self, X, M: int, ldx: int, Y, ldy: int, workspace, workspace_bytes: int,
+                                 stream=None):
+        """The forward with GELU on its output, Y = bf16(GELU(bf16(acc + bias))) (NVFP4 layers)."""
+        _check(_lib.svdq_linear_forward_gelu(self._h, _ptr(X), M, ldx, _ptr(Y), ldy, _ptr(workspace),
+                                             workspace_bytes, _stream(stream)))
 
     def svdq_linear_forward_noalloc(self, X, M: int, ldx: int, Y, ldy: int, stream=None):
         """The forward using the library's fixed device scratch instead of a caller workspace

@@ -1061,9 +1061,9 @@ static cudaError_t make_rows_map(CUtensorMap* map, const void* base, uint64_t by
 // stages before the k-blocks.  Kernel 2 is launched as a programmatic dependent of kernel 1.
 
 constexpr int kGStages = 5;
-// The fused MLP epilogue outlasts the k-loop, which then needs fewer stages in flight; its fourth
-// stage's shared memory holds the epilogue's GELU table instead.
-__host__ __device__ constexpr int gemm_stages(int epi) { return epi == 2 ? 4 : kGStages; }
+// The epilogues with GELU (fused MLP pair, GELU output) run four stages: the fifth stage's shared
+// memory holds the GELU table (the fused MLP epilogue outlasts the k-loop anyway).
+__host__ __device__ constexpr int gemm_stages(int epi) { return epi >= 2 ? 4 : kGStages; }
 // Warp roles, four warpgroups: 0 = the scale warps (warp w writes TMEM lane quadrant w); 1 = the
 // operand producer, the MMA issuer, the scale producer and one idle warp; 2 and 3 = the epilogue.
 constexpr int kGSfWarps = 4;
@@ -1300,6 +1300,37 @@ __device__ __forceinline__ float gelu_bf16_tab(float y, const uint16_t* tbl) {
   return gelu_bf16_outside_table(y);
 }
 
+// The same for the two bf16 values of a packed pair (low half first).
+__device__ __forceinline__ uint32_t gelu_bf16x2_tab(uint32_t w, const uint16_t* tbl) {
+  const float lo = gelu_bf16_tab(__uint_as_float(w << 16), tbl);
+  const float hi = gelu_bf16_tab(__uint_as_float(w & 0xFFFF0000u), tbl);
+  return (__float_as_uint(lo) >> 16) | (__float_as_uint(hi) & 0xFFFF0000u);
+}
+
+// The same for the eight bf16 values packed in w[0..3], in place; warp-collective (all 32 lanes call
+// it together).  When every value of every lane lies in the table's range (nearly always) each takes
+// one table load and no branch of its own; otherwise every value goes through gelu_bf16_tab.
+__device__ __forceinline__ void gelu_bf16x8_warp(uint32_t (&w)[4], const uint16_t* tbl) {
+  constexpr uint32_t kN = kGeluTblBinades * 128, kBase = static_cast<uint32_t>(kGeluTblE0) << 7;
+  uint32_t idx[8];
+  bool in = true;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const uint32_t b = (t & 1) ? (w[t >> 1] >> 16) : (w[t >> 1] & 0xFFFFu);
+    const uint32_t i = (b & 0x7FFFu) - kBase;  // wraps below the table
+    in &= i < kN;
+    idx[t] = (i < kN ? i : kN - 1) + (b >> 15) * kN;
+  }
+  if (__all_sync(0xffffffffu, in)) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      w[q] = static_cast<uint32_t>(tbl[idx[2 * q]]) | (static_cast<uint32_t>(tbl[idx[2 * q + 1]]) << 16);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) w[q] = gelu_bf16x2_tab(w[q], tbl);
+  }
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
@@ -1312,7 +1343,8 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
 
 // Staging box layout: 32 rows of 128 bytes (64 bf16); 16-byte unit u of row l sits at
 // u ^ (l % 8), the tensor map's 128-byte swizzle, so lanes 8i..8i+7 hit distinct bank groups.
-// kEpi: 0 = bias and bf16 Y; 1 = fused Q/K normalization and rotary embedding; 2 = fused MLP pair.
+// kEpi: 0 = bias and bf16 Y; 1 = fused Q/K normalization and rotary embedding; 2 = fused MLP pair;
+// 3 = bias, bf16, then GELU (Y = GELU(bf16(acc + bias)), each rounded to bf16).
 template <int kEpi>
 __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_constant__ GemmMaps maps,
                                                                     const GemmParams p) {
@@ -1329,7 +1361,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
   uint64_t* stg_free = lr_full + 1;         // (both) the epilogue's stores finished reading staging
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stg_free + 1);
   float* gamma_sm = reinterpret_cast<float*>(staging + kGStaging + 256);  // fused Q/K: gamma_q, gamma_k
-  uint16_t* gelu_tbl = reinterpret_cast<uint16_t*>(staging + kGStaging + 256);  // fused MLP: GELU table
+  uint16_t* gelu_tbl = reinterpret_cast<uint16_t*>(staging + kGStaging + 256);  // modes 2, 3: GELU table
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1372,7 +1404,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
     tmem_alloc2(tmem_slot, kTmemCols);
     tmem_relinquish2();
   }
-  if constexpr (kEpi == 2) fill_gelu_table(gelu_tbl, threadIdx.x, kGThreads);  // (before kernel 1 ends)
+  if constexpr (kEpi >= 2) fill_gelu_table(gelu_tbl, threadIdx.x, kGThreads);  // (before kernel 1 ends)
   tc_fence_before();
   cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
   tc_fence_after();
@@ -1499,7 +1531,10 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
             const uint32_t a0 = srow_swz ^ (static_cast<uint32_t>(2 * jg) << 4);
             const uint32_t a1 = srow_swz ^ (static_cast<uint32_t>(2 * jg + 1) << 4);
             const uint4 w0 = ld_shared_v4(a0), w1 = ld_shared_v4(a1);
-            const uint32_t wy[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            uint32_t g0[4] = {w0.x, w0.y, w0.z, w0.w}, g1[4] = {w1.x, w1.y, w1.z, w1.w};
+            gelu_bf16x8_warp(g0, gelu_tbl);  // GELU of the 16 bf16 values, each rounded to bf16
+            gelu_bf16x8_warp(g1, gelu_tbl);
+            const uint32_t wy[8] = {g0[0], g0[1], g0[2], g0[3], g1[0], g1[1], g1[2], g1[3]};
             const float* ilp = p.il_down + n0 + 64 * bx + 16 * jg;
             float il[16];
 #pragma unroll
@@ -1514,9 +1549,8 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
             float pm[8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
-              const float lo = live ? __fmul_rn(gelu_bf16_tab(__uint_as_float(wy[t] << 16), gelu_tbl), il[2 * t]) : 0.0f;
-              const float hi =
-                  live ? __fmul_rn(gelu_bf16_tab(__uint_as_float(wy[t] & 0xFFFF0000u), gelu_tbl), il[2 * t + 1]) : 0.0f;
+              const float lo = live ? __fmul_rn(__uint_as_float(wy[t] << 16), il[2 * t]) : 0.0f;
+              const float hi = live ? __fmul_rn(__uint_as_float(wy[t] & 0xFFFF0000u), il[2 * t + 1]) : 0.0f;
               xp[t >> 2][t & 3] = f2pack(lo, hi);
               pm[t] = fmaxf(fabsf(lo), fabsf(hi));
             }
@@ -1673,6 +1707,11 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_nvfp4_kernel(const __grid_c
               o.y = pack_bf16x2(__uint_as_float(v[bx][hh][c + 2]) + b0.z, __uint_as_float(v[bx][hh][c + 3]) + b0.w);
               o.z = pack_bf16x2(__uint_as_float(v[bx][hh][c + 4]) + b1.x, __uint_as_float(v[bx][hh][c + 5]) + b1.y);
               o.w = pack_bf16x2(__uint_as_float(v[bx][hh][c + 6]) + b1.z, __uint_as_float(v[bx][hh][c + 7]) + b1.w);
+              if constexpr (kEpi == 3) {  // GELU of each bf16 output, rounded to bf16 once more
+                uint32_t g4[4] = {o.x, o.y, o.z, o.w};
+                gelu_bf16x8_warp(g4, gelu_tbl);
+                o = make_uint4(g4[0], g4[1], g4[2], g4[3]);
+              }
             }
             st_shared_v4(srow_swz ^ (static_cast<uint32_t>(u) << 4), o);
           }
@@ -2430,7 +2469,7 @@ static cudaError_t launch_gemm_int4(const GemmArgs& a, int num_sms, cudaStream_t
 }
 
 static size_t gemm_smem_bytes(int mode) {
-  const size_t extra = mode == 2 ? kGeluTblSize * 2 : (mode == 1 ? 2 * kQkvHeadDim * 4 : 0);
+  const size_t extra = mode >= 2 ? kGeluTblSize * 2 : (mode == 1 ? 2 * kQkvHeadDim * 4 : 0);
   return 1024 + static_cast<size_t>(gemm_stages(mode)) * kGStage + kGStaging + 256 + extra;
 }
 
@@ -2481,9 +2520,11 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const int mode = a.mlp ? 2 : (a.qk_cols > 0 ? 1 : 0);
+  const int mode = a.mlp ? 2 : (a.qk_cols > 0 ? 1 : (a.gelu ? 3 : 0));
   const size_t smem = gemm_smem_bytes(mode);
-  auto kernel = mode == 2 ? gemm_nvfp4_kernel<2> : (mode == 1 ? gemm_nvfp4_kernel<1> : gemm_nvfp4_kernel<0>);
+  auto kernel = mode == 3   ? gemm_nvfp4_kernel<3>
+                : mode == 2 ? gemm_nvfp4_kernel<2>
+                            : (mode == 1 ? gemm_nvfp4_kernel<1> : gemm_nvfp4_kernel<0>);
   // The epilogue warpgroups' setmaxnreg.inc waits until the block's pool holds their share, and
   // the pool is the launch's registers a thread x threads: refuse to launch a build whose count
   // differs from the one the split was sized for (the wait would never end).
@@ -2497,7 +2538,8 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   static const cudaError_t regs_plain = check_regs(reinterpret_cast<const void*>(gemm_nvfp4_kernel<0>));
   static const cudaError_t regs_qkv = check_regs(reinterpret_cast<const void*>(gemm_nvfp4_kernel<1>));
   static const cudaError_t regs_mlp = check_regs(reinterpret_cast<const void*>(gemm_nvfp4_kernel<2>));
-  cudaError_t e = mode == 2 ? regs_mlp : (mode == 1 ? regs_qkv : regs_plain);
+  static const cudaError_t regs_gelu = check_regs(reinterpret_cast<const void*>(gemm_nvfp4_kernel<3>));
+  cudaError_t e = mode == 3 ? regs_gelu : (mode == 2 ? regs_mlp : (mode == 1 ? regs_qkv : regs_plain));
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -2641,20 +2683,30 @@ cudaError_t launch_rope_pack(const float* rope, int M, float* packed, cudaStream
 }
 
 // The fused MLP epilogue's bf16 GELU on a list of bf16 inputs (a test hook).
+// Eight values per thread through the epilogues' warp-collective path (every lane calls it).
 __global__ void selftest_gelu_kernel(const uint16_t* in, uint16_t* out, int n) {
   __shared__ uint16_t tbl[kGeluTblSize];
   fill_gelu_table(tbl, threadIdx.x, blockDim.x);
   __syncthreads();
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) {
-    const float g = gelu_bf16_tab(__uint_as_float(static_cast<uint32_t>(in[i]) << 16), tbl);
-    out[i] = static_cast<uint16_t>(__float_as_uint(g) >> 16);
+  const long long i0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t lo = i0 + 2 * q < n ? in[i0 + 2 * q] : 0u;
+    const uint32_t hi = i0 + 2 * q + 1 < n ? in[i0 + 2 * q + 1] : 0u;
+    w[q] = lo | (hi << 16);
+  }
+  gelu_bf16x8_warp(w, tbl);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (i0 + 2 * q < n) out[i0 + 2 * q] = static_cast<uint16_t>(w[q] & 0xFFFFu);
+    if (i0 + 2 * q + 1 < n) out[i0 + 2 * q + 1] = static_cast<uint16_t>(w[q] >> 16);
   }
 }
 
 cudaError_t launch_selftest_gelu(const uint16_t* in, uint16_t* out, int n, cudaStream_t stream) {
   if (n <= 0) return cudaSuccess;
-  selftest_gelu_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(in, out, n);
+  selftest_gelu_kernel<<<static_cast<unsigned>((n + 2047) / 2048), 256, 0, stream>>>(in, out, n);
   return cudaGetLastError();
 }
 

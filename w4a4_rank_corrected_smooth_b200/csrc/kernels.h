@@ -50,6 +50,9 @@ struct GemmArgs {
   float* tpart = nullptr;          // [M padded][2 column halves][mlp_smax][r_down] fp32 partials of T
   int mlp_smax = 0;                // slots per (row, column half): pairs meeting one 256-row block
   int mlp_pairs = 0;               // CTA pairs of the up layer's kernel 2 (the slots assume it)
+  // GELU output (NVFP4 only): Y = GELU(bf16(acc + bias)), rounded to bf16 (the first half of an MLP
+  // whose hidden activation goes through HBM to the next layer's forward).
+  bool gelu = false;
 };
 
 // The down layer's T from the fused MLP epilogue's partials (see the kernel), written in kernel 2's

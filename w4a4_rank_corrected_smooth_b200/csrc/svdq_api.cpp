@@ -185,7 +185,7 @@ struct QkvEpilogue {
 };
 
 svdq_status do_gemm(const svdq_weights* w, int M, void* Y, int ldy, const void* ws, cudaStream_t stream,
-                    const QkvEpilogue* qkv = nullptr, const MlpEpilogue* mlp = nullptr) {
+                    const QkvEpilogue* qkv = nullptr, const MlpEpilogue* mlp = nullptr, bool gelu = false) {
   if (!Y) return fail(SVDQ_ERR_INVALID_ARG, "Y is NULL");
   if (ldy < w->N || ldy % 8 != 0) return fail(SVDQ_ERR_INVALID_ARG, "ldy=%d must be >= N=%d and a multiple of 8", ldy, w->N);
   if (!aligned(Y, 16)) return fail(SVDQ_ERR_INVALID_ARG, "Y must be 16-byte aligned");
@@ -206,6 +206,7 @@ svdq_status do_gemm(const svdq_weights* w, int M, void* Y, int ldy, const void* 
   a.l2 = w->d_l2;
   a.bias = w->d_bias;
   a.Y = static_cast<uint16_t*>(Y);
+  a.gelu = gelu;
   if (qkv) {
     a.qk_cols = qkv->qk_cols;
     a.gamma_q = qkv->gamma_q;
@@ -671,6 +672,22 @@ svdq_status svdq_linear_forward(const svdq_weights* w, const void* X, int M, int
   s = do_quant_down(w, X, M, ldx, workspace, st);
   if (s != SVDQ_OK) return s;
   return do_gemm(w, M, Y, ldy, workspace, st);
+}
+
+svdq_status svdq_linear_forward_gelu(const svdq_weights* w, const void* X, int M, int ldx, void* Y, int ldy,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (w && w->precision != SVDQ_NVFP4)
+    return fail(SVDQ_ERR_INVALID_ARG, "the GELU-output forward runs on an NVFP4 layer (precision %d)", w->precision);
+  svdq_status s = check_forward_common(w, M, workspace, workspace_bytes);
+  if (s != SVDQ_OK || M == 0) return s;
+  if (!Y) return fail(SVDQ_ERR_INVALID_ARG, "Y is NULL");
+  if (ldy < w->N || ldy % 8 != 0 || !aligned(Y, 16))
+    return fail(SVDQ_ERR_INVALID_ARG, "Y must be 16-byte aligned with ldy >= N and a multiple of 8");
+  DeviceGuard guard(w->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = do_quant_down(w, X, M, ldx, workspace, st);
+  if (s != SVDQ_OK) return s;
+  return do_gemm(w, M, Y, ldy, workspace, st, nullptr, nullptr, true);
 }
 
 svdq_status svdq_export_activations(const svdq_weights* w, const void* workspace, size_t workspace_bytes, int M,

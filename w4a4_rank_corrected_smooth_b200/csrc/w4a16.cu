@@ -24,9 +24,10 @@ namespace svdq {
 // Weight-only 4-bit layers run where M is small (FLUX's modulation projections: one token per
 // image), so they are bound by reading the weights (half a byte an element) from HBM.  The weights
 // are streamed, not fetched into registers: one producer thread per CTA keeps a ring of stages in
-// flight with 1-D bulk copies (each stage: 8 groups of 64 along K of the CTA's R blocks of 16
-// weight rows, codes and scales, ~18 KB at R = 4), so an SM has 100-150 KB of weights in flight
-// without a register spent on them.  Eight consumer warps take one group each per stage.
+// flight with 1-D bulk copies (each stage: 16 groups of 64 along K of the CTA's R blocks of 16
+// weight rows, codes and scales, 36 KB at R = 4), so an SM has ~100-150 KB of weights in flight
+// without a register spent on them.  Sixteen consumer warps (four per scheduler, so that one
+// warp's chain of dependent MMAs hides behind the others') take one group each per stage.
 // The contraction runs on the warp-level bf16 tensor-core MMA (m16n8k16, fp32 accumulation) with A
 // from registers: a lane turns one 32-bit word of codes into four bf16x2 fragment registers with one
 // LOP3 each (the code, sign-flipped, into the mantissa of 128: 136 + q exactly) and one bf16x2
@@ -38,7 +39,7 @@ namespace svdq {
 // [blocks][groups][8 pairs (rows i, i + 8)] of fp32, so one (block, group) is 512 + 64 contiguous
 // bytes and a stage's share of one block is one copy of each.
 
-constexpr int kWWarps = 8;                      // consumer warps
+constexpr int kWWarps = 16;                     // consumer warps
 constexpr int kWProducerWarp = kWWarps;         // one more warp: the producer (one thread)
 constexpr int kWThreads = (kWWarps + 1) * 32;
 constexpr int kWConsumers = kWWarps * 32;
@@ -46,7 +47,7 @@ constexpr int kWGs = kWWarps;                   // groups per stage: one per con
 constexpr uint32_t kWCodeBytes = 512;           // one (block, group) of codes
 constexpr uint32_t kWScaleBytes = 64;           // one (block, group) of scales
 constexpr int kWMaxStages = 8;
-constexpr size_t kWSmemBudget = 220 * 1024;
+constexpr size_t kWSmemBudget = 226 * 1024;
 constexpr int kWBarrier = 1;                    // named barrier of the consumer warps
 
 struct W4A16Params {
@@ -317,15 +318,17 @@ static cudaError_t launch_w4a16_rm(const W4A16Params& p0, int num_sms, cudaStrea
   W4A16Params p = p0;
   const int nblocks = (p.N + kBN - 1) / kBN * (kBN / 16);  // the packed weights are padded to 256 rows
   p.nsets = nblocks / R;
-  // x_hat of all of K when it leaves room for at least four stages, else chunks of K
+  // x_hat of all of K with as many stages as fit (at least three), else chunks of K with two
   p.chunk_g = p.G;
-  if (w4a16_smem(R, MB, p.chunk_g, 4) > kWSmemBudget) {
-    const size_t fixed = w4a16_smem(R, MB, 0, 4);
+  int stages = kWMaxStages;
+  while (stages > 3 && w4a16_smem(R, MB, p.chunk_g, stages) > kWSmemBudget) --stages;
+  if (w4a16_smem(R, MB, p.chunk_g, stages) > kWSmemBudget) {
+    stages = 2;
+    const size_t fixed = w4a16_smem(R, MB, 0, stages);
+    if (fixed >= kWSmemBudget) return cudaErrorInvalidConfiguration;
     p.chunk_g = static_cast<int>((kWSmemBudget - fixed) / (static_cast<size_t>(MB) * 1024)) / kWGs * kWGs;
     if (p.chunk_g < kWGs) return cudaErrorInvalidConfiguration;
   }
-  int stages = kWMaxStages;
-  while (stages > 2 && w4a16_smem(R, MB, p.chunk_g, stages) > kWSmemBudget) --stages;
   p.stages = stages;
   const size_t smem = w4a16_smem(R, MB, p.chunk_g, stages);
   cudaError_t e = cudaFuncSetAttribute(w4a16_kernel<R, MB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
