@@ -386,7 +386,7 @@ def kernel_times(layers, sets, stream, launches: int = 200):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     evs = []
-    hold_gpu(stream, 40.0 * launches)
+    hold_gpu(stream, 100.0 * launches)
     start.record(stream)
     for i in range(launches):
         lin = layers[i % len(layers)]

@@ -1307,6 +1307,10 @@ __device__ __forceinline__ uint32_t gelu_bf16x2_tab(uint32_t w, const uint16_t* 
   return (__float_as_uint(lo) >> 16) | (__float_as_uint(hi) & 0xFFFF0000u);
 }
 
+// The rare branch of gelu_bf16x8_warp, out of line so that the epilogues' unrolled loops stay small
+// (their instruction fetch is a bottleneck of its own).
+__device__ __noinline__ uint32_t gelu_bf16x2_rare(uint32_t w, const uint16_t* tbl) { return gelu_bf16x2_tab(w, tbl); }
+
 // The same for the eight bf16 values packed in w[0..3], in place; warp-collective (all 32 lanes call
 // it together).  When every value of every lane lies in the table's range (nearly always) each takes
 // one table load and no branch of its own; otherwise every value goes through gelu_bf16_tab.
@@ -1327,7 +1331,7 @@ __device__ __forceinline__ void gelu_bf16x8_warp(uint32_t (&w)[4], const uint16_
       w[q] = static_cast<uint32_t>(tbl[idx[2 * q]]) | (static_cast<uint32_t>(tbl[idx[2 * q + 1]]) << 16);
   } else {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) w[q] = gelu_bf16x2_tab(w[q], tbl);
+    for (int q = 0; q < 4; ++q) w[q] = gelu_bf16x2_rare(w[q], tbl);
   }
 }
 
