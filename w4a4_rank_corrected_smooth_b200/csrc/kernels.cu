@@ -1009,12 +1009,14 @@ static cudaError_t launch_quant_down_warps(const QuantDownArgs& a, int num_sms, 
   return cudaGetLastError();
 }
 
-// The warp-level kernel when its 16-row blocks fit in one wave (two per SM) and the rank is at most
-// 32 (the FLUX QKV and MLP-up layers: X streamed with the most parallelism); the 128-row tiles
-// otherwise, and whenever the caller's workspace has room for their K-split partials only.
+// The warp-level kernel when its 16-row blocks fit in one wave (two per SM), the rank is at most 32
+// and K at most 4096 (the FLUX QKV and MLP-up layers: X streamed with the most parallelism); the
+// 128-row tiles otherwise.  Past K = 4096 the tiles win even at rank 0 (FLUX MLP-down, K = 12288:
+// 40 us against 50 us at rank 0, 54 us against 66 us at rank 32), since each warp-level CTA
+// walks all of K for its 16 rows and, with rank > 0, reads all of L1 from L2.
 cudaError_t launch_quant_down(const QuantDownArgs& a, int num_sms, cudaStream_t stream) {
   const int mpad = 2 * kBM * ((a.M + 2 * kBM - 1) / (2 * kBM));
-  if (a.rank <= 32 && mpad / kQdRows <= 2 * num_sms) return launch_quant_down_warps(a, num_sms, stream);
+  if (a.rank <= 32 && mpad / kQdRows <= 2 * num_sms && a.K <= 4096) return launch_quant_down_warps(a, num_sms, stream);
   return launch_quant_down_tile(a, num_sms, stream);
 }
 
