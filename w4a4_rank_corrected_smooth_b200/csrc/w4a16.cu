@@ -170,18 +170,20 @@ __global__ void __launch_bounds__(kWThreads, 1) w4a16_kernel(const W4A16Params p
   // (element pairs at k = 16 s + 2 (l % 4) + {0, 1} and that + 8).  Filled from 16-byte loads of
   // 8 consecutive elements of a row (item = row, 8-element unit; consecutive threads take
   // consecutive units): their four pairs are register j = 2 (s % 2) + (k % 16 >= 8) of the four
-  // lanes 4 (m % 8) + t, t = 0..3.
+  // lanes 4 (m % 8) + t, t = 0..3.  Only the pass's rows below M are staged (a single token per
+  // image is the common case); the lanes of the rows past M take zero fragments instead of reading.
   uint32_t* const xw = reinterpret_cast<uint32_t*>(xs);
+  const int rows_live = p.M - m0 < 8 * MB ? p.M - m0 : 8 * MB;
   auto stage_x = [&](int gc, int ng) {
     const int units = ng * 8;  // 8-element units of the chunk per row
-    const int items = MB * 8 * units;
+    const int items = rows_live * units;
 #pragma unroll 4
     for (int e = threadIdx.x; e < items; e += kWConsumers) {
       const int ml = e / units, u = e - ml * units;  // row of the pass, unit of the chunk
       const int m = m0 + ml;
       const int k0 = gc * 64 + 8 * u;
-      uint32_t v[4] = {0u, 0u, 0u, 0u};
-      if (m < p.M) {
+      uint32_t v[4];
+      {
         const uint4 xx = *reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(m) * p.ldx + k0);
         const float4 i0 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + k0));
         const float4 i1 = __ldg(reinterpret_cast<const float4*>(p.inv_lambda + k0 + 4));
@@ -238,7 +240,8 @@ __global__ void __launch_bounds__(kWThreads, 1) w4a16_kernel(const W4A16Params p
 #pragma unroll
         for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
-          for (int h = 0; h < 2; ++h) bq[mb][h] = xs[((mb * cng + gl) * 2 + h) * 32 + lane];
+          for (int h = 0; h < 2; ++h)
+            bq[mb][h] = 8 * mb + gid < rows_live ? xs[((mb * cng + gl) * 2 + h) * 32 + lane] : make_uint4(0u, 0u, 0u, 0u);
         const uint8_t* sb = ring + static_cast<size_t>(slot) * kStage;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
